@@ -1,0 +1,166 @@
+"""Torch-facing API of one TwoTower denoiser refinement step (device memory and streams only).
+
+Each function allocates its outputs with torch and calls the matching C-ABI entry point of
+libtt_denoise.so through `binding`; every step of the computation runs in the library's CUDA
+kernels. Workspaces are cached per (device, size) and zero-filled once, as the ABI requires.
+
+    denoise_attention    Eq. (1), layer-aligned denoiser attention       (tt_denoise_attn)
+    adaln_cond           adaLN-single: tau -> (shift, scale, gate)       (tt_adaln_modulate)
+    adaln_norm_modulate  modulated RMSNorm prologue                      (tt_adaln_modulate)
+    adaln_gated_residual h + gate * f                                    (tt_adaln_modulate)
+    unmask_step          ConfidenceSample, Algorithm 2 line 5            (tt_unmask_step)
+    RefinementStep       the whole step a1..a7 on one stream, from device or host buffers
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional, Tuple
+
+import torch
+
+from . import binding as B
+
+_WS: Dict[Tuple[int, str, int], torch.Tensor] = {}
+
+
+def workspace(nbytes: int, device: torch.device, tag: str) -> torch.Tensor:
+    """A cached zero-initialised workspace of at least nbytes for (device, tag)."""
+    dev = torch.device(device)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device(), tag, 0)
+    ws = _WS.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = B.new_workspace(nbytes, device=dev)
+        _WS[key] = ws
+    return ws
+
+
+def check_device_error(ws: torch.Tensor):
+    st, detail = B.tt_get_device_error(ws)
+    if st != B.TT_OK:
+        raise B.TTError(st, f"device-side error (detail {detail:#x})")
+
+
+def denoise_attention(q, k_blk, v_blk, k_ctx, v_ctx, ctx_lens, page_table=None, page_size: int = 0,
+                      ctx_stride: int = 0, softmax_scale: float = 1.0, return_lse: bool = False,
+                      out: Optional[torch.Tensor] = None, ws_tag: str = "attn"):
+    out = torch.empty_like(q) if out is None else out
+    lse = None
+    if return_lse:
+        Bn, S, Hq, _ = q.shape
+        lse = torch.empty((Bn, Hq, S), dtype=torch.float32, device=q.device)
+    args = B.attn_args(q, k_blk, v_blk, k_ctx, v_ctx, ctx_lens, out, page_table=page_table, page_size=page_size,
+                       ctx_stride=ctx_stride, softmax_scale=softmax_scale, lse=lse)
+    nbytes = B.tt_denoise_attn_workspace_bytes(args)
+    if nbytes == 0:
+        # invalid or unsupported arguments: let the launch report the exact status
+        nbytes = 256
+    ws = workspace(nbytes, q.device, ws_tag)
+    B.tt_denoise_attn(args, ws)
+    return (out, lse) if return_lse else out
+
+
+def adaln_cond(tau, w1, b1, w2, b2, w3, b3, layer_emb, ws_tag: str = "adaln"):
+    Bn = tau.shape[0]
+    D = layer_emb.shape[1]
+    mod = torch.empty((Bn, 3, D), dtype=torch.float32, device=tau.device)
+    args = B.adaln_args(B.TT_ADALN_COND, batch=Bn, hidden=D, freq_dim=w1.shape[1], mlp_width=w1.shape[0],
+                        tau=tau, w1=w1, b1=b1, w2=w2, b2=b2, w3=w3, b3=b3, layer_emb=layer_emb, mod=mod)
+    ws = workspace(max(256, B.tt_adaln_workspace_bytes(args)), tau.device, ws_tag)
+    B.tt_adaln_modulate(args, ws)
+    return mod
+
+
+def adaln_norm_modulate(h, norm_w, mod, eps: float = 1e-5, out=None, ws_tag: str = "adaln"):
+    Bn, S, D = h.shape
+    out = torch.empty_like(h) if out is None else out
+    args = B.adaln_args(B.TT_ADALN_NORM_MODULATE, batch=Bn, block_size=S, hidden=D, dtype=h.dtype, eps=eps,
+                        h=h, norm_w=norm_w, mod=mod, out=out)
+    ws = workspace(256, h.device, ws_tag)
+    B.tt_adaln_modulate(args, ws)
+    return out
+
+
+def adaln_gated_residual(h, f, mod, out=None, ws_tag: str = "adaln"):
+    Bn, S, D = h.shape
+    out = torch.empty_like(h) if out is None else out
+    args = B.adaln_args(B.TT_ADALN_GATED_RESIDUAL, batch=Bn, block_size=S, hidden=D, dtype=h.dtype, h=h, f=f,
+                        mod=mod, out=out)
+    ws = workspace(256, h.device, ws_tag)
+    B.tt_adaln_modulate(args, ws)
+    return out
+
+
+def unmask_step(logits, tokens, is_masked, *, gamma: float, inv_temperature: float = 1.0, mask_token_id: int = 3,
+                exclude_mask_token: bool = False, remaining_steps: int = 0, want_conf: bool = True,
+                ws_tag: str = "unmask"):
+    """Updates tokens / is_masked in place; returns (n_committed, n_masked, conf, argmax)."""
+    Bn, S, V = logits.shape
+    dev = logits.device
+    n_committed = torch.empty(Bn, dtype=torch.int32, device=dev)
+    n_masked = torch.empty(Bn, dtype=torch.int32, device=dev)
+    conf = torch.empty((Bn, S), dtype=torch.float32, device=dev) if want_conf else None
+    argmax = torch.empty((Bn, S), dtype=torch.int32, device=dev) if want_conf else None
+    args = B.unmask_args(logits, tokens, is_masked, n_committed, n_masked, gamma=gamma,
+                         inv_temperature=inv_temperature, mask_token_id=mask_token_id,
+                         exclude_mask_token=exclude_mask_token, remaining_steps=remaining_steps, conf=conf,
+                         argmax=argmax)
+    ws = workspace(max(256, B.tt_unmask_workspace_bytes(args)), dev, ws_tag)
+    B.tt_unmask_step(args, ws)
+    return n_committed, n_masked, conf, argmax
+
+
+@dataclasses.dataclass
+class StepBuffers:
+    """Device tensors of one refinement step (inputs and outputs)."""
+    tau: torch.Tensor
+    h: torch.Tensor
+    f: torch.Tensor
+    q: torch.Tensor
+    k_blk: torch.Tensor
+    v_blk: torch.Tensor
+    k_ctx: torch.Tensor
+    v_ctx: torch.Tensor
+    ctx_lens: torch.Tensor
+    page_table: Optional[torch.Tensor]
+    logits: torch.Tensor
+    tokens: torch.Tensor
+    is_masked: torch.Tensor
+
+
+class RefinementStep:
+    """One denoiser refinement step of TwoTower decoding on one GPU, one stream.
+
+    a2  mod = adaLN-single(tau)                 (tau = masked fraction, Algorithm 2 line 3)
+    a3  y = modulated RMSNorm(h)                (prologue; y feeds the out-of-scope QKV projection)
+    a4  O = Eq. (1) attention(q, [K_ctx; K_blk], [V_ctx; V_blk])
+    a5  h' = h + gate * f                       (f: the mixer output after its out-projection)
+    a6/a7  ConfidenceSample on the vocabulary logits (tokens / mask updated in place)
+    The weights (adaLN MLP, per-layer embedding, norm weight) live on the device.
+    """
+
+    def __init__(self, weights: Dict[str, torch.Tensor], *, gamma: float, inv_temperature: float = 1.0,
+                 mask_token_id: int = 3, page_size: int = 0, ctx_stride: int = 0, softmax_scale: float = 1.0,
+                 eps: float = 1e-5, remaining_steps: int = 0):
+        self.w = weights
+        self.gamma = gamma
+        self.inv_temperature = inv_temperature
+        self.mask_token_id = mask_token_id
+        self.page_size = page_size
+        self.ctx_stride = ctx_stride
+        self.softmax_scale = softmax_scale
+        self.eps = eps
+        self.remaining_steps = remaining_steps
+        self._args = None
+
+    def run(self, b: StepBuffers, out_attn: Optional[torch.Tensor] = None):
+        w = self.w
+        mod = adaln_cond(b.tau, w["w1"], w["b1"], w["w2"], w["b2"], w["w3"], w["b3"], w["layer_emb"])
+        y = adaln_norm_modulate(b.h, w["norm_w"], mod, eps=self.eps)
+        o = denoise_attention(b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
+                              page_size=self.page_size, ctx_stride=self.ctx_stride,
+                              softmax_scale=self.softmax_scale, out=out_attn)
+        h_new = adaln_gated_residual(b.h, b.f, mod)
+        nc, nm, _, _ = unmask_step(b.logits, b.tokens, b.is_masked, gamma=self.gamma,
+                                   inv_temperature=self.inv_temperature, mask_token_id=self.mask_token_id,
+                                   remaining_steps=self.remaining_steps, want_conf=False)
+        return {"mod": mod, "y": y, "attn": o, "h": h_new, "n_committed": nc, "n_masked": nm}

@@ -1,0 +1,236 @@
+"""ctypes binding of libtt_denoise.so: argument marshalling only.
+
+Every entry point of include/tt_denoise.h is exposed under the same name. The torch-facing
+wrappers take CUDA tensors, fill the C argument struct with their device pointers and sizes,
+and call the library on torch's current stream; all arithmetic runs in the library's kernels.
+There is no fallback: if the shared library is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtt_denoise.so")
+
+TT_OK = 0
+TT_ERR_INVALID_ARGUMENT = 1
+TT_ERR_UNSUPPORTED = 2
+TT_ERR_WORKSPACE_TOO_SMALL = 3
+TT_ERR_CUDA = 4
+TT_ERR_DEVICE = 5
+TT_ERR_DEVICE_TIMEOUT = 6
+
+TT_F32 = 0
+TT_BF16 = 1
+
+TT_ADALN_COND = 0
+TT_ADALN_NORM_MODULATE = 1
+TT_ADALN_GATED_RESIDUAL = 2
+
+EXPORTED = [
+    "tt_status_string", "tt_version",
+    "tt_denoise_attn_workspace_bytes", "tt_denoise_attn",
+    "tt_adaln_workspace_bytes", "tt_adaln_modulate",
+    "tt_unmask_workspace_bytes", "tt_unmask_step",
+    "tt_get_device_error",
+]
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_f32 = ctypes.c_float
+
+
+class AttnArgs(ctypes.Structure):
+    _fields_ = [
+        ("batch", _i32), ("block_size", _i32), ("num_q_heads", _i32), ("num_kv_heads", _i32),
+        ("head_dim", _i32), ("dtype", _i32), ("softmax_scale", _f32),
+        ("q", _vp), ("k_blk", _vp), ("v_blk", _vp), ("k_ctx", _vp), ("v_ctx", _vp),
+        ("ctx_lens", _vp), ("page_table", _vp),
+        ("page_size", _i32), ("max_pages_per_seq", _i32), ("num_pages", _i32), ("ctx_stride", _i32),
+        ("out", _vp), ("lse", _vp),
+    ]
+
+
+class AdalnArgs(ctypes.Structure):
+    _fields_ = [
+        ("op", _i32), ("batch", _i32), ("block_size", _i32), ("hidden", _i32), ("freq_dim", _i32),
+        ("mlp_width", _i32), ("dtype", _i32), ("eps", _f32),
+        ("tau", _vp), ("w1", _vp), ("b1", _vp), ("w2", _vp), ("b2", _vp), ("w3", _vp), ("b3", _vp),
+        ("layer_emb", _vp), ("mod", _vp), ("h", _vp), ("norm_w", _vp), ("f", _vp), ("out", _vp),
+    ]
+
+
+class UnmaskArgs(ctypes.Structure):
+    _fields_ = [
+        ("batch", _i32), ("block_size", _i32), ("vocab", _i32), ("dtype", _i32), ("logits", _vp),
+        ("gamma", _f32), ("inv_temperature", _f32), ("mask_token_id", _i32), ("exclude_mask_token", _i32),
+        ("remaining_steps", _i32), ("tokens", _vp), ("is_masked", _vp), ("conf", _vp), ("argmax", _vp),
+        ("n_committed", _vp), ("n_masked", _vp),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtt_denoise.so (raises if it is missing: there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with python -m denoiser_attention_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        L.tt_status_string.restype = ctypes.c_char_p
+        L.tt_status_string.argtypes = [ctypes.c_int]
+        L.tt_version.restype = ctypes.c_int
+        L.tt_denoise_attn_workspace_bytes.restype = ctypes.c_size_t
+        L.tt_denoise_attn_workspace_bytes.argtypes = [ctypes.POINTER(AttnArgs)]
+        L.tt_denoise_attn.restype = ctypes.c_int
+        L.tt_denoise_attn.argtypes = [ctypes.POINTER(AttnArgs), _vp, ctypes.c_size_t, _vp]
+        L.tt_adaln_workspace_bytes.restype = ctypes.c_size_t
+        L.tt_adaln_workspace_bytes.argtypes = [ctypes.POINTER(AdalnArgs)]
+        L.tt_adaln_modulate.restype = ctypes.c_int
+        L.tt_adaln_modulate.argtypes = [ctypes.POINTER(AdalnArgs), _vp, ctypes.c_size_t, _vp]
+        L.tt_unmask_workspace_bytes.restype = ctypes.c_size_t
+        L.tt_unmask_workspace_bytes.argtypes = [ctypes.POINTER(UnmaskArgs)]
+        L.tt_unmask_step.restype = ctypes.c_int
+        L.tt_unmask_step.argtypes = [ctypes.POINTER(UnmaskArgs), _vp, ctypes.c_size_t, _vp]
+        L.tt_get_device_error.restype = ctypes.c_int
+        L.tt_get_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+        _lib = L
+    return _lib
+
+
+class TTError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().tt_status_string(status).decode()}")
+
+
+def _check(status: int, what: str):
+    if status != TT_OK:
+        raise TTError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return TT_BF16
+    if dt == torch.float32:
+        return TT_F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def status_string(status: int) -> str:
+    return lib().tt_status_string(status).decode()
+
+
+# ------------------------------------------------------------------------------------------ attn
+def attn_args(q, k_blk, v_blk, k_ctx, v_ctx, ctx_lens, out, page_table=None, page_size=0,
+              ctx_stride=0, softmax_scale=1.0, lse=None) -> AttnArgs:
+    B, S, Hq, d = q.shape
+    Hkv = k_blk.shape[2]
+    a = AttnArgs()
+    a.batch, a.block_size, a.num_q_heads, a.num_kv_heads, a.head_dim = B, S, Hq, Hkv, d
+    a.dtype = _dtype_code(q.dtype)
+    a.softmax_scale = float(softmax_scale)
+    a.q, a.k_blk, a.v_blk = _ptr(q), _ptr(k_blk), _ptr(v_blk)
+    a.k_ctx, a.v_ctx = _ptr(k_ctx), _ptr(v_ctx)
+    a.ctx_lens = _ptr(ctx_lens)
+    a.page_table = _ptr(page_table)
+    if page_table is not None:
+        a.page_size = int(page_size)
+        a.max_pages_per_seq = int(page_table.shape[1])
+        a.num_pages = int(k_ctx.shape[0])
+    else:
+        a.ctx_stride = int(ctx_stride) if ctx_stride else int(k_ctx.shape[1])
+    a.out = _ptr(out)
+    a.lse = _ptr(lse)
+    return a
+
+
+def tt_denoise_attn_workspace_bytes(args: AttnArgs) -> int:
+    return int(lib().tt_denoise_attn_workspace_bytes(ctypes.byref(args)))
+
+
+def tt_denoise_attn(args: AttnArgs, workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().tt_denoise_attn(ctypes.byref(args), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream)), "tt_denoise_attn")
+
+
+# ------------------------------------------------------------------------------------------ adaLN
+def adaln_args(op: int, *, batch: int, hidden: int, block_size: int = 0, freq_dim: int = 256,
+               mlp_width: int = 256, dtype=torch.float32, eps: float = 1e-5, tau=None, w1=None, b1=None,
+               w2=None, b2=None, w3=None, b3=None, layer_emb=None, mod=None, h=None, norm_w=None, f=None,
+               out=None) -> AdalnArgs:
+    a = AdalnArgs()
+    a.op, a.batch, a.block_size, a.hidden = op, batch, block_size, hidden
+    a.freq_dim, a.mlp_width, a.dtype, a.eps = freq_dim, mlp_width, _dtype_code(dtype), float(eps)
+    a.tau, a.w1, a.b1, a.w2, a.b2 = _ptr(tau), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)
+    a.w3, a.b3, a.layer_emb, a.mod = _ptr(w3), _ptr(b3), _ptr(layer_emb), _ptr(mod)
+    a.h, a.norm_w, a.f, a.out = _ptr(h), _ptr(norm_w), _ptr(f), _ptr(out)
+    return a
+
+
+def tt_adaln_workspace_bytes(args: AdalnArgs) -> int:
+    return int(lib().tt_adaln_workspace_bytes(ctypes.byref(args)))
+
+
+def tt_adaln_modulate(args: AdalnArgs, workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().tt_adaln_modulate(ctypes.byref(args), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tt_adaln_modulate")
+
+
+# ------------------------------------------------------------------------------------------ unmask
+def unmask_args(logits, tokens, is_masked, n_committed, n_masked, *, gamma: float, inv_temperature: float = 1.0,
+                mask_token_id: int = 3, exclude_mask_token: bool = False, remaining_steps: int = 0,
+                conf=None, argmax=None) -> UnmaskArgs:
+    B, S, V = logits.shape
+    a = UnmaskArgs()
+    a.batch, a.block_size, a.vocab, a.dtype = B, S, V, _dtype_code(logits.dtype)
+    a.logits = _ptr(logits)
+    a.gamma, a.inv_temperature = float(gamma), float(inv_temperature)
+    a.mask_token_id, a.exclude_mask_token, a.remaining_steps = int(mask_token_id), int(bool(exclude_mask_token)), int(remaining_steps)
+    a.tokens, a.is_masked = _ptr(tokens), _ptr(is_masked)
+    a.conf, a.argmax = _ptr(conf), _ptr(argmax)
+    a.n_committed, a.n_masked = _ptr(n_committed), _ptr(n_masked)
+    return a
+
+
+def tt_unmask_workspace_bytes(args: UnmaskArgs) -> int:
+    return int(lib().tt_unmask_workspace_bytes(ctypes.byref(args)))
+
+
+def tt_unmask_step(args: UnmaskArgs, workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().tt_unmask_step(ctypes.byref(args), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream)), "tt_unmask_step")
+
+
+def tt_get_device_error(workspace: torch.Tensor, stream=None):
+    detail = ctypes.c_uint32(0)
+    st = lib().tt_get_device_error(_ptr(workspace), _stream(stream), ctypes.byref(detail))
+    return st, detail.value
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """Zero-filled device workspace of at least nbytes (256-byte granularity)."""
+    n = max(256, (int(nbytes) + 255) // 256 * 256)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")

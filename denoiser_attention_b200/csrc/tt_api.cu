@@ -1,0 +1,166 @@
+// C ABI entry points: host-side argument validation, workspace sizing and dispatch to the
+// sm_100a kernels. Nothing here allocates device memory or keeps mutable global state.
+#include <cstdio>
+#include <cstring>
+
+#include "tt_common.cuh"
+#include "tt_internal.h"
+
+namespace tt {
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int validate_attn(const tt_attn_args_t* a) {
+  if (!a) return TT_ERR_INVALID_ARGUMENT;
+  if (a->batch < 1 || a->block_size < 1 || a->num_q_heads < 1 || a->num_kv_heads < 1 || a->head_dim < 1)
+    return TT_ERR_INVALID_ARGUMENT;
+  if (a->num_q_heads % a->num_kv_heads != 0) return TT_ERR_INVALID_ARGUMENT;
+  if (a->dtype != TT_F32 && a->dtype != TT_BF16) return TT_ERR_INVALID_ARGUMENT;
+  if (!a->q || !a->k_blk || !a->v_blk || !a->k_ctx || !a->v_ctx || !a->ctx_lens || !a->out)
+    return TT_ERR_INVALID_ARGUMENT;
+  if (!(a->softmax_scale > 0.f) && !(a->softmax_scale < 0.f)) return TT_ERR_INVALID_ARGUMENT;
+  if (a->page_table) {
+    if (a->page_size < 1 || a->max_pages_per_seq < 1 || a->num_pages < 1) return TT_ERR_INVALID_ARGUMENT;
+  } else {
+    if (a->ctx_stride < 0) return TT_ERR_INVALID_ARGUMENT;
+  }
+  if (a->block_size > 64) return TT_ERR_UNSUPPORTED;
+  if (a->dtype == TT_BF16 && !attn_tc_supported(a)) return TT_ERR_UNSUPPORTED;
+  if (a->dtype == TT_F32 && !attn_simt_supported(a)) return TT_ERR_UNSUPPORTED;
+  return TT_OK;
+}
+
+static int validate_unmask(const tt_unmask_args_t* a) {
+  if (!a) return TT_ERR_INVALID_ARGUMENT;
+  if (a->batch < 1 || a->block_size < 1 || a->vocab < 1) return TT_ERR_INVALID_ARGUMENT;
+  if (a->dtype != TT_F32 && a->dtype != TT_BF16) return TT_ERR_INVALID_ARGUMENT;
+  if (!a->logits || !a->tokens || !a->is_masked || !a->n_committed || !a->n_masked) return TT_ERR_INVALID_ARGUMENT;
+  if (!(a->inv_temperature > 0.f)) return TT_ERR_INVALID_ARGUMENT;
+  if (a->remaining_steps < 0) return TT_ERR_INVALID_ARGUMENT;
+  if (a->exclude_mask_token && (a->mask_token_id < 0 || a->mask_token_id >= a->vocab)) return TT_ERR_INVALID_ARGUMENT;
+  if (a->block_size > 1024) return TT_ERR_UNSUPPORTED;
+  const int W = (a->dtype == TT_BF16) ? 8 : 4;
+  if (a->vocab % W != 0 || !aligned16(a->logits)) return TT_ERR_UNSUPPORTED;
+  return TT_OK;
+}
+
+static int validate_adaln(const tt_adaln_args_t* a) {
+  if (!a) return TT_ERR_INVALID_ARGUMENT;
+  if (a->batch < 1 || a->hidden < 1) return TT_ERR_INVALID_ARGUMENT;
+  if (a->dtype != TT_F32 && a->dtype != TT_BF16) return TT_ERR_INVALID_ARGUMENT;
+  switch (a->op) {
+    case TT_ADALN_COND:
+      if (!a->tau || !a->w1 || !a->b1 || !a->w2 || !a->b2 || !a->w3 || !a->b3 || !a->layer_emb || !a->mod)
+        return TT_ERR_INVALID_ARGUMENT;
+      if (a->freq_dim < 2 || (a->freq_dim & 1) || a->mlp_width < 1) return TT_ERR_INVALID_ARGUMENT;
+      if (a->freq_dim > 1024 || a->mlp_width > 1024) return TT_ERR_UNSUPPORTED;
+      return TT_OK;
+    case TT_ADALN_NORM_MODULATE:
+    case TT_ADALN_GATED_RESIDUAL: {
+      if (a->block_size < 1) return TT_ERR_INVALID_ARGUMENT;
+      if (!a->h || !a->mod || !a->out) return TT_ERR_INVALID_ARGUMENT;
+      if (a->op == TT_ADALN_NORM_MODULATE && !a->norm_w) return TT_ERR_INVALID_ARGUMENT;
+      if (a->op == TT_ADALN_GATED_RESIDUAL && !a->f) return TT_ERR_INVALID_ARGUMENT;
+      if (a->op == TT_ADALN_NORM_MODULATE && !(a->eps >= 0.f)) return TT_ERR_INVALID_ARGUMENT;
+      const int W = (a->dtype == TT_BF16) ? 8 : 4;
+      if (a->hidden % W != 0) return TT_ERR_UNSUPPORTED;
+      if (!aligned16(a->h) || !aligned16(a->out) || (a->f && !aligned16(a->f))) return TT_ERR_UNSUPPORTED;
+      return TT_OK;
+    }
+    default:
+      return TT_ERR_INVALID_ARGUMENT;
+  }
+}
+
+}  // namespace tt
+
+using namespace tt;
+
+extern "C" {
+
+const char* tt_status_string(int status) {
+  switch (status) {
+    case TT_OK: return "TT_OK";
+    case TT_ERR_INVALID_ARGUMENT: return "TT_ERR_INVALID_ARGUMENT";
+    case TT_ERR_UNSUPPORTED: return "TT_ERR_UNSUPPORTED";
+    case TT_ERR_WORKSPACE_TOO_SMALL: return "TT_ERR_WORKSPACE_TOO_SMALL";
+    case TT_ERR_CUDA: return "TT_ERR_CUDA";
+    case TT_ERR_DEVICE: return "TT_ERR_DEVICE";
+    case TT_ERR_DEVICE_TIMEOUT: return "TT_ERR_DEVICE_TIMEOUT";
+    default: return "TT_ERR_UNKNOWN";
+  }
+}
+
+int tt_version(void) { return 100; }
+
+size_t tt_denoise_attn_workspace_bytes(const tt_attn_args_t* a) {
+  if (validate_attn(a) != TT_OK) return 0;
+  const int sms = device_sm_count();
+  return a->dtype == TT_BF16 ? attn_tc_plan(a, sms).total : attn_simt_plan(a, sms).total;
+}
+
+int tt_denoise_attn(const tt_attn_args_t* a, void* ws, size_t ws_bytes, tt_stream_t stream) {
+  const int st = validate_attn(a);
+  if (st != TT_OK) return st;
+  if (!ws) return TT_ERR_INVALID_ARGUMENT;
+  const int sms = device_sm_count();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (a->dtype == TT_BF16) {
+    const AttnPlan pl = attn_tc_plan(a, sms);
+    if (ws_bytes < pl.total) return TT_ERR_WORKSPACE_TOO_SMALL;
+    return attn_tc_launch(a, pl, ws, s);
+  }
+  const AttnPlan pl = attn_simt_plan(a, sms);
+  if (ws_bytes < pl.total) return TT_ERR_WORKSPACE_TOO_SMALL;
+  return attn_simt_launch(a, pl, ws, s);
+}
+
+size_t tt_adaln_workspace_bytes(const tt_adaln_args_t* a) {
+  if (validate_adaln(a) != TT_OK) return 0;
+  return adaln_workspace_bytes(a);
+}
+
+int tt_adaln_modulate(const tt_adaln_args_t* a, void* ws, size_t ws_bytes, tt_stream_t stream) {
+  const int st = validate_adaln(a);
+  if (st != TT_OK) return st;
+  if (!ws) return TT_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < adaln_workspace_bytes(a)) return TT_ERR_WORKSPACE_TOO_SMALL;
+  return adaln_launch(a, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tt_unmask_workspace_bytes(const tt_unmask_args_t* a) {
+  if (validate_unmask(a) != TT_OK) return 0;
+  return unmask_plan(a, device_sm_count()).layout.total;
+}
+
+int tt_unmask_step(const tt_unmask_args_t* a, void* ws, size_t ws_bytes, tt_stream_t stream) {
+  const int st = validate_unmask(a);
+  if (st != TT_OK) return st;
+  if (!ws) return TT_ERR_INVALID_ARGUMENT;
+  const UnmaskPlan pl = unmask_plan(a, device_sm_count());
+  if (ws_bytes < pl.layout.total) return TT_ERR_WORKSPACE_TOO_SMALL;
+  return unmask_launch(a, pl, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int tt_get_device_error(void* ws, tt_stream_t stream, uint32_t* detail) {
+  if (!ws) return TT_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t host[2] = {0, 0};
+  if (cudaMemcpyAsync(host, ws, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return TT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TT_ERR_CUDA;
+  if (host[0] != 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof(host), s) != cudaSuccess) return TT_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TT_ERR_CUDA;
+  }
+  if (detail) *detail = host[1];
+  return (int)host[0];
+}
+
+}  // extern "C"

@@ -1,0 +1,50 @@
+// Host-side interfaces between the C ABI layer (tt_api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/tt_denoise.h"
+
+namespace tt {
+
+// ---------------------------------------------------------------- unmask
+struct UnmaskLayout {
+  size_t row_cnt, seq_cnt, partials, conf, argmax, total;
+};
+struct UnmaskPlan {
+  int chunks;
+  int chunk_elems;
+  UnmaskLayout layout;
+};
+UnmaskPlan unmask_plan(const tt_unmask_args_t* a, int num_sms);
+int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& plan, void* ws, cudaStream_t stream);
+
+// ---------------------------------------------------------------- adaLN
+size_t adaln_workspace_bytes(const tt_adaln_args_t* a);
+int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream);
+
+// ---------------------------------------------------------------- attention
+struct AttnPlan {
+  int grid;            // persistent CTAs
+  int qtiles;          // query-row tiles per (sequence, kv head)
+  int s_per_tile;      // block positions per query-row tile
+  int units;           // batch * kv heads * qtiles
+  size_t off_tickets;  // int32 [units]
+  size_t off_partials; // float [slots][rows][d]
+  size_t off_lse;      // float [slots][rows]
+  size_t slots;
+  size_t total;
+};
+bool attn_tc_supported(const tt_attn_args_t* a);
+AttnPlan attn_tc_plan(const tt_attn_args_t* a, int num_sms);
+int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& plan, void* ws, cudaStream_t stream);
+
+bool attn_simt_supported(const tt_attn_args_t* a);
+AttnPlan attn_simt_plan(const tt_attn_args_t* a, int num_sms);
+int attn_simt_launch(const tt_attn_args_t* a, const AttnPlan& plan, void* ws, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace tt

@@ -1,0 +1,330 @@
+// ConfidenceSample on sm_100a: the paper §2.2 "Sampling" and Algorithm 2 line 5 of
+// "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Context".
+//
+// One pass over the vocabulary logits computes, per block position, the softmax maximum
+// probability (confidence) and the argmax token; the last CTA to finish a sequence's positions
+// then applies the commit rule to that sequence. Logits are read once, with 128-bit loads.
+//
+// Grid: one CTA per (row, chunk) where a row is one (sequence, position) and a chunk is a
+// contiguous slice of the vocabulary, so that even 128 rows fill all SMs. Per thread the running
+// state is (m, s, idx): the largest raw logit seen, s = sum exp(c (x - m)) with
+// c = inv_temperature * log2(e) evaluated as exp2, and the lowest index attaining m. States merge
+// associatively; ties keep the lower token index at every level.
+#include <cmath>
+#include <cstdio>
+#include <algorithm>
+
+#include "tt_common.cuh"
+#include "tt_internal.h"
+
+namespace tt {
+
+struct UnmaskPartial {
+  float m;
+  float s;
+  int32_t idx;
+  int32_t pad;
+};
+
+struct RedState {
+  float m;
+  float s;
+  int32_t idx;
+};
+
+__device__ __forceinline__ RedState red_combine(RedState a, RedState b, float c) {
+  RedState r;
+  const bool take_b = (b.m > a.m) || (b.m == a.m && b.idx < a.idx);
+  r.idx = take_b ? b.idx : a.idx;
+  r.m = fmaxf(a.m, b.m);
+  const float sa = (a.m == -INFINITY) ? 0.f : a.s * ex2(c * (a.m - r.m));
+  const float sb = (b.m == -INFINITY) ? 0.f : b.s * ex2(c * (b.m - r.m));
+  r.s = sa + sb;
+  return r;
+}
+
+template <typename T>
+struct VecTraits;
+template <>
+struct VecTraits<float> {
+  static constexpr int kN = 4;
+  __device__ static void to_float(const uint4& v, float* x) {
+    x[0] = __uint_as_float(v.x);
+    x[1] = __uint_as_float(v.y);
+    x[2] = __uint_as_float(v.z);
+    x[3] = __uint_as_float(v.w);
+  }
+};
+template <>
+struct VecTraits<__nv_bfloat16> {
+  static constexpr int kN = 8;
+  __device__ static void to_float(const uint4& v, float* x) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
+struct UnmaskParams {
+  const void* logits;
+  int32_t vocab;
+  int32_t chunk_elems;   // multiple of the vector width
+  int32_t chunks;        // C
+  int32_t rows;          // B*S
+  int32_t block_size;    // S
+  float c;               // inv_temperature * log2(e)
+  float gamma;
+  int32_t mask_token_id;
+  int32_t exclude_mask_token;
+  int32_t remaining_steps;
+  int32_t* tokens;
+  uint8_t* is_masked;
+  float* conf_out;
+  int32_t* argmax_out;
+  int32_t* n_committed;
+  int32_t* n_masked;
+  uint8_t* ws;
+  size_t off_row_cnt, off_seq_cnt, off_partials, off_conf, off_argmax;
+};
+
+constexpr int kUnmaskThreads = 256;
+constexpr int kUnmaskUnroll = 4;
+
+// Commit rule for one sequence, run by the whole CTA.
+__device__ void commit_sequence(const UnmaskParams& p, int b, const float* conf_ws, const int32_t* arg_ws) {
+  __shared__ float s_conf[1024];
+  __shared__ uint8_t s_masked[1024];
+  __shared__ int s_counts[2];
+  const int S = p.block_size;
+  const int tid = threadIdx.x;
+  if (tid < 2) s_counts[tid] = 0;
+  __syncthreads();
+  int my_masked = 0, my_ge = 0;
+  for (int l = tid; l < S; l += blockDim.x) {
+    const float cf = __ldcg(conf_ws + (size_t)b * S + l);
+    const uint8_t mk = p.is_masked[(size_t)b * S + l] ? 1 : 0;
+    s_conf[l] = cf;
+    s_masked[l] = mk;
+    my_masked += mk;
+    my_ge += (mk && cf >= p.gamma) ? 1 : 0;
+  }
+  atomicAdd(&s_counts[0], my_masked);
+  atomicAdd(&s_counts[1], my_ge);
+  __syncthreads();
+  const int n_masked = s_counts[0];
+  const int n_ge = s_counts[1];
+  int need = 0;
+  if (n_masked > 0) need = (p.remaining_steps > 0) ? (n_masked + p.remaining_steps - 1) / p.remaining_steps : 1;
+  const int K = max(need, n_ge);
+  // a masked position commits iff its rank among masked positions (confidence descending,
+  // position ascending) is below K; every position >= gamma ranks below n_ge <= K.
+  for (int l = tid; l < S; l += blockDim.x) {
+    if (!s_masked[l]) continue;
+    const float cl = s_conf[l];
+    int rank = 0;
+    for (int j = 0; j < S; ++j) {
+      if (!s_masked[j]) continue;
+      const float cj = s_conf[j];
+      rank += (cj > cl || (cj == cl && j < l)) ? 1 : 0;
+    }
+    if (rank < K) {
+      p.tokens[(size_t)b * S + l] = __ldcg(arg_ws + (size_t)b * S + l);
+      p.is_masked[(size_t)b * S + l] = 0;
+    }
+  }
+  if (tid == 0) {
+    const int committed = min(K, n_masked);
+    p.n_committed[b] = committed;
+    p.n_masked[b] = n_masked - committed;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskParams p) {
+  using VT = VecTraits<T>;
+  constexpr int N = VT::kN;
+  const int row = blockIdx.x / p.chunks;
+  const int chunk = blockIdx.x - row * p.chunks;
+  const int tid = threadIdx.x;
+  const T* rowp = reinterpret_cast<const T*>(p.logits) + (size_t)row * p.vocab;
+  const int begin = chunk * p.chunk_elems;
+  const int end = min(p.vocab, begin + p.chunk_elems);
+  const int nvec = (end - begin) / N;
+  const uint4* vp = reinterpret_cast<const uint4*>(rowp + begin);
+  const float c = p.c;
+
+  float m = -INFINITY, s = 0.f;
+  int32_t idx = 0x7fffffff;
+
+  auto consume = [&](const uint4& raw, int vbase) {
+    float x[N];
+    VT::to_float(raw, x);
+    if (p.exclude_mask_token) {
+      const int r = p.mask_token_id - vbase;
+      if (r >= 0 && r < N) x[r] = -INFINITY;
+    }
+    float vm = x[0];
+    int vi = 0;
+#pragma unroll
+    for (int k = 1; k < N; ++k) {
+      if (x[k] > vm) { vm = x[k]; vi = k; }
+    }
+    if (vm > m) {
+      s = (m == -INFINITY) ? 0.f : s * ex2(c * (m - vm));
+      m = vm;
+      idx = vbase + vi;
+    }
+    const float nmc = -c * m;
+#pragma unroll
+    for (int k = 0; k < N; ++k) s += ex2(fmaf(x[k], c, nmc));
+  };
+
+  int v = tid;
+  for (; v + (kUnmaskUnroll - 1) * kUnmaskThreads < nvec; v += kUnmaskUnroll * kUnmaskThreads) {
+    uint4 raw[kUnmaskUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnmaskUnroll; ++u) raw[u] = __ldcs(vp + v + u * kUnmaskThreads);
+#pragma unroll
+    for (int u = 0; u < kUnmaskUnroll; ++u) consume(raw[u], begin + (v + u * kUnmaskThreads) * N);
+  }
+  for (; v < nvec; v += kUnmaskThreads) consume(__ldcs(vp + v), begin + v * N);
+
+  // ---- CTA reduction (warp shuffles, then across warps), keeping the lowest index on ties
+  RedState st{m, s, idx};
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    RedState o;
+    o.m = __shfl_xor_sync(0xffffffffu, st.m, off);
+    o.s = __shfl_xor_sync(0xffffffffu, st.s, off);
+    o.idx = __shfl_xor_sync(0xffffffffu, st.idx, off);
+    st = red_combine(st, o, c);
+  }
+  __shared__ RedState s_red[kUnmaskThreads / 32];
+  __shared__ int s_flag;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (lane == 0) s_red[warp] = st;
+  __syncthreads();
+
+  float* conf_ws = reinterpret_cast<float*>(p.ws + p.off_conf);
+  int32_t* arg_ws = reinterpret_cast<int32_t*>(p.ws + p.off_argmax);
+  int* row_cnt = reinterpret_cast<int*>(p.ws + p.off_row_cnt);
+  int* seq_cnt = reinterpret_cast<int*>(p.ws + p.off_seq_cnt);
+  UnmaskPartial* parts = reinterpret_cast<UnmaskPartial*>(p.ws + p.off_partials);
+
+  if (tid == 0) {
+    RedState r = s_red[0];
+    for (int w = 1; w < kUnmaskThreads / 32; ++w) r = red_combine(r, s_red[w], c);
+    bool row_done = true;
+    if (p.chunks > 1) {
+      parts[(size_t)row * p.chunks + chunk] = UnmaskPartial{r.m, r.s, r.idx, 0};
+      __threadfence();
+      const int old = atomicAdd(row_cnt + row, 1);
+      row_done = (old == p.chunks - 1);
+      if (row_done) {
+        row_cnt[row] = 0;
+        __threadfence();
+        const float4* pp = reinterpret_cast<const float4*>(parts + (size_t)row * p.chunks);
+        float4 q = __ldcg(pp);
+        r = RedState{q.x, q.y, __float_as_int(q.z)};
+        for (int k = 1; k < p.chunks; ++k) {
+          q = __ldcg(pp + k);
+          r = red_combine(r, RedState{q.x, q.y, __float_as_int(q.z)}, c);
+        }
+      }
+    }
+    int last_of_seq = 0;
+    if (row_done) {
+      const float conf = 1.0f / r.s;
+      conf_ws[row] = conf;
+      arg_ws[row] = r.idx;
+      if (p.conf_out) p.conf_out[row] = conf;
+      if (p.argmax_out) p.argmax_out[row] = r.idx;
+      __threadfence();
+      const int b = row / p.block_size;
+      const int old = atomicAdd(seq_cnt + b, 1);
+      if (old == p.block_size - 1) {
+        seq_cnt[b] = 0;
+        __threadfence();
+        last_of_seq = 1;
+      }
+    }
+    s_flag = last_of_seq;
+  }
+  __syncthreads();
+  if (s_flag) commit_sequence(p, row / p.block_size, conf_ws, arg_ws);
+}
+
+static UnmaskLayout layout_for(int rows, int batch, int chunks) {
+  UnmaskLayout L{};
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return o;
+  };
+  L.row_cnt = take(sizeof(int) * (size_t)rows);
+  L.seq_cnt = take(sizeof(int) * (size_t)batch);
+  L.partials = take(sizeof(UnmaskPartial) * (size_t)rows * chunks);
+  L.conf = take(sizeof(float) * (size_t)rows);
+  L.argmax = take(sizeof(int32_t) * (size_t)rows);
+  L.total = off;
+  return L;
+}
+
+UnmaskPlan unmask_plan(const tt_unmask_args_t* a, int num_sms) {
+  UnmaskPlan pl{};
+  const int rows = a->batch * a->block_size;
+  const int W = (a->dtype == TT_BF16) ? 8 : 4;
+  const int target = 4 * std::max(num_sms, 1);
+  int chunks = (target + rows - 1) / rows;
+  const int max_chunks = std::max(1, a->vocab / 4096);
+  chunks = std::max(1, std::min(chunks, max_chunks));
+  // chunk length: a multiple of one CTA sweep (threads x vector width) where possible
+  const int sweep = kUnmaskThreads * W;
+  int chunk_elems = (a->vocab + chunks - 1) / chunks;
+  chunk_elems = ((chunk_elems + sweep - 1) / sweep) * sweep;
+  if (chunk_elems > a->vocab) chunk_elems = ((a->vocab + W - 1) / W) * W;
+  chunks = (a->vocab + chunk_elems - 1) / chunk_elems;
+  pl.chunks = chunks;
+  pl.chunk_elems = chunk_elems;
+  pl.layout = layout_for(rows, a->batch, chunks);
+  return pl;
+}
+
+int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cudaStream_t stream) {
+  UnmaskParams p{};
+  p.logits = a->logits;
+  p.vocab = a->vocab;
+  p.chunk_elems = pl.chunk_elems;
+  p.chunks = pl.chunks;
+  p.rows = a->batch * a->block_size;
+  p.block_size = a->block_size;
+  p.c = a->inv_temperature * 1.4426950408889634f;
+  p.gamma = a->gamma;
+  p.mask_token_id = a->mask_token_id;
+  p.exclude_mask_token = a->exclude_mask_token;
+  p.remaining_steps = a->remaining_steps;
+  p.tokens = a->tokens;
+  p.is_masked = a->is_masked;
+  p.conf_out = a->conf;
+  p.argmax_out = a->argmax;
+  p.n_committed = a->n_committed;
+  p.n_masked = a->n_masked;
+  p.ws = static_cast<uint8_t*>(ws);
+  p.off_row_cnt = pl.layout.row_cnt;
+  p.off_seq_cnt = pl.layout.seq_cnt;
+  p.off_partials = pl.layout.partials;
+  p.off_conf = pl.layout.conf;
+  p.off_argmax = pl.layout.argmax;
+  const unsigned grid = (unsigned)p.rows * (unsigned)pl.chunks;
+  if (a->dtype == TT_BF16)
+    unmask_kernel<__nv_bfloat16><<<grid, kUnmaskThreads, 0, stream>>>(p);
+  else
+    unmask_kernel<float><<<grid, kUnmaskThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
+}
+
+}  // namespace tt

@@ -1,0 +1,220 @@
+/*
+ * tt_denoise.h -- C ABI of the B200 (sm_100a) TwoTower denoiser refinement step.
+ *
+ * One refinement step of TwoTower block-autoregressive diffusion decoding, as described in
+ * "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Context" (arXiv 2606.26493,
+ * "the paper" below), has three GPU operations, each one entry point here:
+ *
+ *   tt_denoise_attn    layer-aligned denoiser attention, the paper §2.1 Eq. (1)
+ *   tt_adaln_modulate  adaLN-single time conditioning, the paper §2.1 "Time conditioning"
+ *   tt_unmask_step     confidence-threshold unmasking, the paper §2.2 "Sampling", Algorithm 2
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer named in an args struct is a DEVICE pointer (cudaMalloc'd or equivalent)
+ *     unless its comment says "host". The caller owns all memory; the library never allocates
+ *     or frees, keeps no mutable global state, and may be called from several host threads.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Tensors are dense, row-major, with the shapes written in brackets.
+ *   - Argument errors are found on the host and returned before anything is launched:
+ *     TT_ERR_INVALID_ARGUMENT (null pointer, bad size), TT_ERR_UNSUPPORTED (valid but not
+ *     implemented, e.g. a head_dim the kernels do not handle), TT_ERR_WORKSPACE_TOO_SMALL.
+ *   - A failed launch returns TT_ERR_CUDA (the CUDA error is left for cudaGetLastError()).
+ *   - Errors only the device can see (a page id outside the pool, a context length beyond the
+ *     page table or the contiguous stride, a wait that timed out) never trap: the kernel sets a
+ *     word in the caller's workspace, skips the offending work, and tt_get_device_error()
+ *     reports it as TT_ERR_DEVICE or TT_ERR_DEVICE_TIMEOUT.
+ *   - Inputs must be finite. NaN/Inf inputs give unspecified (but non-faulting) results.
+ *   - Workspaces must be zero-filled once before their first use (cudaMemset); the kernels
+ *     leave them ready for the next call. Calls that share a workspace must be stream-ordered.
+ */
+#ifndef TT_DENOISE_H_
+#define TT_DENOISE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* tt_stream_t;
+
+typedef enum {
+  TT_OK = 0,
+  TT_ERR_INVALID_ARGUMENT = 1,
+  TT_ERR_UNSUPPORTED = 2,
+  TT_ERR_WORKSPACE_TOO_SMALL = 3,
+  TT_ERR_CUDA = 4,
+  TT_ERR_DEVICE = 5,
+  TT_ERR_DEVICE_TIMEOUT = 6
+} tt_status_t;
+
+typedef enum { TT_F32 = 0, TT_BF16 = 1 } tt_dtype_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* tt_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int tt_version(void);
+
+/* ---------------------------------------------------------------------------------------------
+ * Eq. (1), the paper §2.1 "Bidirectional attention": the S queries of the noisy block b at
+ * denoiser layer i attend to the concatenation of the context tower's layer-i keys/values for
+ * the past blocks 0..b-1 (the prefix cache, L_b tokens) and the denoiser's own layer-i
+ * keys/values of block b (S tokens):
+ *     O = softmax(softmax_scale * Q [K_ctx; K_blk]^T) [V_ctx; V_blk]
+ * Inside the block attention is bidirectional; every past block precedes the block, so no
+ * query is masked from any key: the only mask is the ragged end of each context.
+ * Grouped-query layout: query head h reads key/value head h / (Hq / Hkv).
+ *
+ * Layouts (E = element type given by dtype: TT_BF16 = bfloat16, TT_F32 = float):
+ *   q       [B][S][Hq][d]   E
+ *   k_blk   [B][S][Hkv][d]  E      (v_blk likewise)
+ *   k_ctx   contiguous (page_table == NULL): [B][ctx_stride][Hkv][d] E, sequence b's token t at
+ *           row t of its slab; paged: [num_pages][page_size][Hkv][d] E, token t of sequence b at
+ *           page page_table[b][t / page_size], row t % page_size.  (v_ctx likewise)
+ *   ctx_lens [B] int32, L_b >= 0 (0 = the first block: attention over the block alone)
+ *   page_table [B][max_pages_per_seq] int32 or NULL
+ *   out     [B][S][Hq][d]   E, rounded to nearest from the fp32 result
+ *   lse     [B][Hq][S] float or NULL: natural-log log-sum-exp of the scaled scores per row
+ * Supported: TT_BF16 with d = 128 (tensor-core path, S*Hq/Hkv rows per tile, S <= 64,
+ * page_size a multiple of 64); TT_F32 with d in {64, 128}. Others: TT_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct {
+  int32_t batch;             /* B >= 1 */
+  int32_t block_size;        /* S, 1..64 */
+  int32_t num_q_heads;       /* Hq, multiple of Hkv */
+  int32_t num_kv_heads;      /* Hkv >= 1 */
+  int32_t head_dim;          /* d */
+  int32_t dtype;             /* tt_dtype_t */
+  float softmax_scale;       /* multiplies Q.K (1.0 when Q is pre-scaled) */
+  const void* q;
+  const void* k_blk;
+  const void* v_blk;
+  const void* k_ctx;
+  const void* v_ctx;
+  const int32_t* ctx_lens;
+  const int32_t* page_table; /* NULL => contiguous context */
+  int32_t page_size;         /* paged: tokens per page */
+  int32_t max_pages_per_seq; /* paged: row length of page_table */
+  int32_t num_pages;         /* paged: pages in the pool */
+  int32_t ctx_stride;        /* contiguous: rows per sequence slab (>= every L_b) */
+  void* out;
+  float* lse;                /* optional */
+} tt_attn_args_t;
+
+/* Bytes of workspace tt_denoise_attn needs for these arguments (0 if the args are invalid). */
+size_t tt_denoise_attn_workspace_bytes(const tt_attn_args_t* args);
+
+/* Launch Eq. (1). `workspace` (device, zero-filled once) holds the split-KV partial results,
+ * the merge tickets and the device error word. */
+int tt_denoise_attn(const tt_attn_args_t* args, void* workspace, size_t workspace_bytes,
+                    tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * adaLN-single, the paper §2.1 "Time conditioning": a global MLP maps the diffusion time to
+ * shared (shift, scale, gate) parameters and a per-layer learned embedding is added; the
+ * result modulates the layer's RMSNorm prologue and gates its residual.
+ *
+ * op TT_ADALN_COND (tau, weights -> mod):
+ *   phi(tau) = [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)), k < F/2
+ *   mod[b] = W3 SiLU(W2 SiLU(W1 phi(tau_b) + b1) + b2) + b3, viewed as [3][D], + layer_emb
+ *   tau [B] float; w1 [W][F], b1 [W], w2 [W][W], b2 [W], w3 [3D][W], b3 [3D], layer_emb [3][D]
+ *   (all float); mod [B][3][D] float (rows: shift, scale, gate). F even, 2..1024; W 1..1024.
+ *   Needs workspace of tt_adaln_workspace_bytes() bytes (the MLP's hidden activations).
+ * op TT_ADALN_NORM_MODULATE (h, norm_w, mod -> out):
+ *   out[b][s] = h[b][s] / sqrt(mean(h[b][s]^2) + eps) * norm_w * (1 + scale[b]) + shift[b]
+ *   h, out [B][S][D] E; norm_w [D] float.
+ * op TT_ADALN_GATED_RESIDUAL (h, f, mod -> out):
+ *   out[b][s] = h[b][s] + gate[b] * f[b][s]        h, f, out [B][S][D] E (out may alias h)
+ * D must be a multiple of 8 for TT_BF16 and of 4 for TT_F32.
+ * ------------------------------------------------------------------------------------------- */
+typedef enum {
+  TT_ADALN_COND = 0,
+  TT_ADALN_NORM_MODULATE = 1,
+  TT_ADALN_GATED_RESIDUAL = 2
+} tt_adaln_op_t;
+
+typedef struct {
+  int32_t op;                /* tt_adaln_op_t */
+  int32_t batch;             /* B */
+  int32_t block_size;        /* S (NORM_MODULATE, GATED_RESIDUAL) */
+  int32_t hidden;            /* D */
+  int32_t freq_dim;          /* F (COND) */
+  int32_t mlp_width;         /* W (COND) */
+  int32_t dtype;             /* tt_dtype_t of h, f, out */
+  float eps;                 /* RMSNorm epsilon */
+  const float* tau;
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+  const float* w3;
+  const float* b3;
+  const float* layer_emb;
+  float* mod;                /* COND: output; other ops: input */
+  const void* h;
+  const float* norm_w;
+  const void* f;
+  void* out;
+} tt_adaln_args_t;
+
+size_t tt_adaln_workspace_bytes(const tt_adaln_args_t* args);
+int tt_adaln_modulate(const tt_adaln_args_t* args, void* workspace, size_t workspace_bytes,
+                      tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * ConfidenceSample, the paper §2.2 "Sampling" and Algorithm 2 line 5: the denoiser predicts
+ * every masked position in parallel; predictions whose confidence reaches gamma are committed,
+ * the rest stay masked for later steps.
+ *   conf[b][l]   = max_v softmax(inv_temperature * logits[b][l])_v
+ *   argmax[b][l] = smallest v attaining max_v logits[b][l][v]
+ *   For each sequence b: every position with is_masked = 1 and conf >= gamma is committed
+ *   (tokens := argmax, is_masked := 0). If none qualifies and a position is still masked, the
+ *   single masked position with the largest conf is committed (lowest position on ties). With
+ *   remaining_steps > 0 (the T - r + 1 of Algorithm 2), at least ceil(n_masked/remaining_steps)
+ *   of the most confident masked positions are committed, so a block finishes within T steps.
+ *   Positions already committed are never changed.
+ * Layouts: logits [B][S][V] E; tokens [B][S] int32 (in/out); is_masked [B][S] uint8 (in/out,
+ *   0/1); conf [B][S] float and argmax [B][S] int32 (optional outputs, may be NULL);
+ *   n_committed, n_masked [B] int32 outputs. exclude_mask_token != 0 removes the logit of
+ *   mask_token_id from both the softmax and the argmax. V must be a multiple of 8 (bf16) or
+ *   4 (fp32); S <= 1024.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct {
+  int32_t batch;             /* B */
+  int32_t block_size;        /* S */
+  int32_t vocab;             /* V */
+  int32_t dtype;             /* tt_dtype_t of logits */
+  const void* logits;
+  float gamma;               /* confidence threshold */
+  float inv_temperature;     /* > 0 */
+  int32_t mask_token_id;
+  int32_t exclude_mask_token;
+  int32_t remaining_steps;   /* 0 => commit >= gamma, else the single most confident */
+  int32_t* tokens;
+  uint8_t* is_masked;
+  float* conf;               /* optional */
+  int32_t* argmax;           /* optional */
+  int32_t* n_committed;
+  int32_t* n_masked;
+} tt_unmask_args_t;
+
+size_t tt_unmask_workspace_bytes(const tt_unmask_args_t* args);
+int tt_unmask_step(const tt_unmask_args_t* args, void* workspace, size_t workspace_bytes,
+                   tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Device-side error word of a workspace (any of the three). Synchronises `stream`, reads the
+ * word and clears it. Returns TT_OK, TT_ERR_DEVICE (bad page id / context length) or
+ * TT_ERR_DEVICE_TIMEOUT (a bounded wait inside a kernel gave up). *detail (host, may be NULL)
+ * receives a kernel-specific code for diagnostics.
+ * ------------------------------------------------------------------------------------------- */
+int tt_get_device_error(void* workspace, tt_stream_t stream, uint32_t* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TT_DENOISE_H_ */

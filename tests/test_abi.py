@@ -1,0 +1,153 @@
+"""C ABI checks that need no GPU: the library loads, exports every function include/*.h
+declares, and rejects bad arguments on the host before anything is launched."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from denoiser_attention_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(tt_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from denoiser_attention_b200 import build
+    build.build()
+    return B.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("tt_denoise_attn", "tt_adaln_modulate", "tt_unmask_step", "tt_get_device_error"):
+        assert n in names
+    assert set(names) == set(B.EXPORTED), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in _declared_functions():
+        assert n in exported, n
+        getattr(lib, n)
+
+
+def test_status_strings(lib):
+    assert B.status_string(0) == "TT_OK"
+    assert B.status_string(6) == "TT_ERR_DEVICE_TIMEOUT"
+    assert lib.tt_version() >= 100
+
+
+def _attn_args(**kw):
+    a = B.AttnArgs()
+    a.batch, a.block_size, a.num_q_heads, a.num_kv_heads, a.head_dim = 2, 16, 32, 2, 128
+    a.dtype, a.softmax_scale = B.TT_BF16, 1.0
+    for f in ("q", "k_blk", "v_blk", "k_ctx", "v_ctx", "ctx_lens", "out"):
+        setattr(a, f, 4096)
+    a.ctx_stride = 4096
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(num_q_heads=31), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(q=None), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(ctx_lens=None), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(dtype=7), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(softmax_scale=0.0), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(block_size=65), B.TT_ERR_UNSUPPORTED),
+    (dict(head_dim=96), B.TT_ERR_UNSUPPORTED),
+    (dict(page_table=4096, page_size=100, max_pages_per_seq=4, num_pages=8), B.TT_ERR_UNSUPPORTED),
+    (dict(page_table=4096, page_size=0, max_pages_per_seq=4, num_pages=8), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(q=4098), B.TT_ERR_UNSUPPORTED),
+])
+def test_attn_host_validation(lib, kw, status):
+    a = _attn_args(**kw)
+    assert lib.tt_denoise_attn(ctypes.byref(a), 4096, 1 << 30, None) == status
+    assert lib.tt_denoise_attn_workspace_bytes(ctypes.byref(a)) == 0
+
+
+def test_attn_workspace_too_small(lib):
+    a = _attn_args()
+    need = lib.tt_denoise_attn_workspace_bytes(ctypes.byref(a))
+    assert need > 256
+    assert lib.tt_denoise_attn(ctypes.byref(a), 4096, need - 1, None) == B.TT_ERR_WORKSPACE_TOO_SMALL
+    assert lib.tt_denoise_attn(ctypes.byref(a), None, need, None) == B.TT_ERR_INVALID_ARGUMENT
+
+
+def _unmask_args(**kw):
+    a = B.UnmaskArgs()
+    a.batch, a.block_size, a.vocab, a.dtype = 2, 16, 1024, B.TT_BF16
+    a.logits = a.tokens = a.is_masked = a.n_committed = a.n_masked = 4096
+    a.gamma, a.inv_temperature = 0.8, 1.0
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(vocab=0), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(tokens=None), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(inv_temperature=0.0), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(remaining_steps=-1), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(exclude_mask_token=1, mask_token_id=5000), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(vocab=1001), B.TT_ERR_UNSUPPORTED),
+    (dict(block_size=1025), B.TT_ERR_UNSUPPORTED),
+])
+def test_unmask_host_validation(lib, kw, status):
+    a = _unmask_args(**kw)
+    assert lib.tt_unmask_step(ctypes.byref(a), 4096, 1 << 30, None) == status
+
+
+def test_unmask_workspace_sizes(lib):
+    a = _unmask_args(batch=8, vocab=131072)
+    need = lib.tt_unmask_workspace_bytes(ctypes.byref(a))
+    assert need >= 256 + 8 * 16 * (4 + 4 + 4)
+    assert lib.tt_unmask_step(ctypes.byref(a), 4096, need - 1, None) == B.TT_ERR_WORKSPACE_TOO_SMALL
+
+
+def _adaln_args(**kw):
+    a = B.AdalnArgs()
+    a.op, a.batch, a.block_size, a.hidden, a.freq_dim, a.mlp_width = B.TT_ADALN_COND, 2, 16, 256, 256, 256
+    a.dtype, a.eps = B.TT_F32, 1e-5
+    for f in ("tau", "w1", "b1", "w2", "b2", "w3", "b3", "layer_emb", "mod", "h", "norm_w", "f", "out"):
+        setattr(a, f, 4096)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(op=9), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(freq_dim=255), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(w3=None), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(mlp_width=2048), B.TT_ERR_UNSUPPORTED),
+    (dict(op=B.TT_ADALN_NORM_MODULATE, norm_w=None), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(op=B.TT_ADALN_NORM_MODULATE, hidden=6), B.TT_ERR_UNSUPPORTED),
+    (dict(op=B.TT_ADALN_GATED_RESIDUAL, f=None), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(op=B.TT_ADALN_GATED_RESIDUAL, dtype=B.TT_BF16, hidden=260), B.TT_ERR_UNSUPPORTED),
+])
+def test_adaln_host_validation(lib, kw, status):
+    a = _adaln_args(**kw)
+    assert lib.tt_adaln_modulate(ctypes.byref(a), 4096, 1 << 30, None) == status
+
+
+def test_adaln_workspace(lib):
+    a = _adaln_args(batch=8, mlp_width=256)
+    assert lib.tt_adaln_workspace_bytes(ctypes.byref(a)) == 256 + 4 * 8 * 256
+    assert lib.tt_adaln_modulate(ctypes.byref(a), 4096, 100, None) == B.TT_ERR_WORKSPACE_TOO_SMALL

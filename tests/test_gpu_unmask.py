@@ -1,0 +1,119 @@
+"""ConfidenceSample on the GPU (through the C ABI) against the CPU fp64 oracle: confidence within
+1e-5, argmax ids bit-exact (lowest id on ties), committed tokens/mask bit-exact except at
+positions whose oracle confidence is within 1e-5 of gamma (counted)."""
+import numpy as np
+import pytest
+import torch
+
+from denoiser_attention_b200 import api, synth
+from tests._parity import check_unmask, np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _state(B, S, seed, frac_masked=1.0, mask_id=3):
+    g = torch.Generator().manual_seed(seed)
+    masked = (torch.rand((B, S), generator=g) < frac_masked).to(torch.uint8)
+    tokens = torch.randint(0, 1000, (B, S), generator=g, dtype=torch.int32)
+    tokens[masked.bool()] = mask_id
+    return tokens, masked
+
+
+def _step(logits, tokens, masked, **kw):
+    dev = "cuda"
+    t = tokens.to(dev)
+    m = masked.to(dev)
+    nc, nm, conf, arg = api.unmask_step(logits.to(dev), t, m, **kw)
+    torch.cuda.synchronize()
+    return t.cpu(), m.cpu(), nc.cpu(), nm.cpu(), conf.cpu(), arg.cpu()
+
+
+@pytest.mark.parametrize("B,S,V,dtype,std,gamma,it,frac", [
+    (1, 16, 1024, torch.float32, 2.0, 0.8, 1.0, 1.0),
+    (2, 16, 1000, torch.float32, 0.5, 0.8, 10.0, 0.7),
+    (3, 8, 4096 + 8, torch.bfloat16, 3.0, 0.5, 4.0, 0.9),
+    (2, 64, 32000, torch.bfloat16, 3.0, 0.3, 3.0, 0.5),
+    (4, 16, 131072, torch.bfloat16, 3.0, 0.8, 1.0, 1.0),
+    (1, 1024, 256, torch.float32, 1.0, 0.05, 2.0, 0.8),
+])
+def test_unmask_matches_oracle(cuda_lib, B, S, V, dtype, std, gamma, it, frac):
+    logits = synth.logits_normal(V + S, B, S, V, std, dtype)
+    tokens, masked = _state(B, S, seed=V, frac_masked=frac)
+    t, m, nc, nm, conf, arg = _step(logits, tokens, masked, gamma=gamma, inv_temperature=it)
+    check_unmask(tokens, masked, logits, gamma, it, t, m, nc, nm, conf, arg)
+
+
+def test_decode_workload_logits(cuda_lib):
+    w = synth.workload("decode_bf16")
+    logits = synth.workload_logits(w)
+    tokens, masked = _state(8, 16, seed=1)
+    t, m, nc, nm, conf, arg = _step(logits, tokens, masked, gamma=w.gamma)
+    band = check_unmask(tokens, masked, logits, w.gamma, 1.0, t, m, nc, nm, conf, arg)
+    frac = float((np64(conf) >= w.gamma).mean())
+    print(f"positions above gamma: {frac:.2f}, in the 1e-5 band: {band}")
+    assert 0.15 < frac < 0.45
+
+
+def test_ties_take_lowest_token_id(cuda_lib):
+    B, S, V = 2, 4, 8192
+    logits = torch.zeros((B, S, V), dtype=torch.bfloat16)
+    logits[0, 0, [5000, 17, 8000]] = 2.0      # tie across chunks: lowest id 17
+    logits[0, 1, :] = 1.0                     # all equal: id 0
+    logits[1, 2, [8191, 4096]] = 3.0
+    tokens, masked = _state(B, S, seed=3)
+    t, m, nc, nm, conf, arg = _step(logits, tokens, masked, gamma=0.9)
+    assert arg[0, 0] == 17 and arg[0, 1] == 0 and arg[1, 2] == 4096
+    assert abs(float(conf[0, 1]) - 1.0 / V) < 1e-9
+    check_unmask(tokens, masked, logits, 0.9, 1.0, t, m, nc, nm, conf, arg)
+
+
+def test_exclude_mask_token(cuda_lib):
+    B, S, V = 2, 8, 2048
+    logits = synth.logits_normal(5, B, S, V, 1.0, torch.float32)
+    logits[:, :, 3] = 50.0                     # the [MASK] logit dominates unless excluded
+    tokens, masked = _state(B, S, seed=4)
+    t, m, nc, nm, conf, arg = _step(logits, tokens, masked, gamma=0.8, exclude_mask_token=True, mask_token_id=3)
+    assert (arg != 3).all()
+    check_unmask(tokens, masked, logits, 0.8, 1.0, t, m, nc, nm, conf, arg, exclude_token=3)
+
+
+@pytest.mark.parametrize("rem", [1, 2, 5])
+def test_remaining_steps_schedule(cuda_lib, rem):
+    B, S, V = 4, 32, 4096
+    logits = synth.logits_normal(6, B, S, V, 2.0, torch.bfloat16)
+    tokens, masked = _state(B, S, seed=5, frac_masked=0.8)
+    t, m, nc, nm, conf, arg = _step(logits, tokens, masked, gamma=0.99, remaining_steps=rem)
+    check_unmask(tokens, masked, logits, 0.99, 1.0, t, m, nc, nm, conf, arg, remaining_steps=rem)
+    n_in = masked.sum(1)
+    assert (nc.long() >= torch.clamp((n_in + rem - 1) // rem, max=S)).all()
+
+
+def test_fully_committed_sequence_unchanged(cuda_lib):
+    B, S, V = 3, 16, 1024
+    logits = synth.logits_normal(7, B, S, V, 2.0, torch.float32)
+    tokens, masked = _state(B, S, seed=6)
+    masked[1] = 0
+    t, m, nc, nm, conf, arg = _step(logits, tokens, masked, gamma=0.8)
+    assert nc[1] == 0 and nm[1] == 0 and torch.equal(t[1], tokens[1])
+    check_unmask(tokens, masked, logits, 0.8, 1.0, t, m, nc, nm, conf, arg)
+
+
+def test_block_loop_tiny_closes_in_T_steps(cuda_lib):
+    # Algorithm 2 on the device for the tiny workload: logits redrawn each step (seed r), tau is
+    # the masked fraction; with max probability ~0.1 << gamma every step commits exactly one
+    # position and the block finishes at r = T = 16 -- the same trajectory as the oracle's loop.
+    from oracle import tt_oracle as O
+    w = synth.workload("tiny_fp32")
+    S, T = w.attn.block_size, w.steps
+    dev = "cuda"
+    tokens = torch.full((1, S), 3, dtype=torch.int32, device=dev)
+    masked = torch.ones((1, S), dtype=torch.uint8, device=dev)
+    traj = []
+    for r in range(1, T + 1):
+        logits = synth.logits_normal(r, 1, S, w.vocab, w.logits_std, torch.float32).to(dev)
+        nc, nm, _, _ = api.unmask_step(logits, tokens, masked, gamma=w.gamma)
+        traj.append(int(nc.item()))
+    assert traj == [1] * T and int(masked.sum()) == 0
+    t_or, m_or, _ = O.refine_block(1, S, T, w.gamma, lambda r, tau: synth.logits_normal(
+        r, 1, S, w.vocab, w.logits_std, torch.float32).double().numpy())
+    np.testing.assert_array_equal(tokens.cpu().numpy(), t_or)
