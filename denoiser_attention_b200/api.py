@@ -20,13 +20,17 @@ import torch
 
 from . import binding as B
 
-_WS: Dict[Tuple[int, str, int], torch.Tensor] = {}
+_WS: Dict[Tuple, torch.Tensor] = {}
 
 
-def workspace(nbytes: int, device: torch.device, tag: str) -> torch.Tensor:
-    """A cached zero-initialised workspace of at least nbytes for (device, tag)."""
+def workspace(nbytes: int, device: torch.device, tag: str, signature: Tuple = ()) -> torch.Tensor:
+    """A cached zero-initialised workspace of at least nbytes for (device, tag, signature).
+
+    The layout of a workspace (where its merge tickets live) depends on the argument sizes, and
+    the kernels only restore the tickets of their own layout to zero, so a workspace is reused
+    only by calls with the same signature (the sizes that determine the layout)."""
     dev = torch.device(device)
-    key = (dev.index if dev.index is not None else torch.cuda.current_device(), tag, 0)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device(), tag, tuple(signature))
     ws = _WS.get(key)
     if ws is None or ws.numel() < nbytes:
         ws = B.new_workspace(nbytes, device=dev)
@@ -54,7 +58,7 @@ def denoise_attention(q, k_blk, v_blk, k_ctx, v_ctx, ctx_lens, page_table=None, 
     if nbytes == 0:
         # invalid or unsupported arguments: let the launch report the exact status
         nbytes = 256
-    ws = workspace(nbytes, q.device, ws_tag)
+    ws = workspace(nbytes, q.device, ws_tag, (tuple(q.shape), k_blk.shape[2], q.dtype))
     B.tt_denoise_attn(args, ws)
     return (out, lse) if return_lse else out
 
@@ -104,7 +108,7 @@ def unmask_step(logits, tokens, is_masked, *, gamma: float, inv_temperature: flo
                          inv_temperature=inv_temperature, mask_token_id=mask_token_id,
                          exclude_mask_token=exclude_mask_token, remaining_steps=remaining_steps, conf=conf,
                          argmax=argmax)
-    ws = workspace(max(256, B.tt_unmask_workspace_bytes(args)), dev, ws_tag)
+    ws = workspace(max(256, B.tt_unmask_workspace_bytes(args)), dev, ws_tag, (tuple(logits.shape), logits.dtype))
     B.tt_unmask_step(args, ws)
     return n_committed, n_masked, conf, argmax
 
@@ -164,3 +168,47 @@ class RefinementStep:
                                    inv_temperature=self.inv_temperature, mask_token_id=self.mask_token_id,
                                    remaining_steps=self.remaining_steps, want_conf=False)
         return {"mod": mod, "y": y, "attn": o, "h": h_new, "n_committed": nc, "n_masked": nm}
+
+
+class HostStep:
+    """RefinementStep driven from host buffers: each run() copies the step's inputs from (pinned)
+    host memory to the device, runs the step on the device and copies its results back -- the
+    attention output, the updated tokens and mask, the commit counts and the new residual."""
+
+    INPUTS = ("tau", "h", "f", "q", "k_blk", "v_blk", "k_ctx", "v_ctx", "ctx_lens", "logits", "tokens", "is_masked")
+
+    def __init__(self, step: RefinementStep, host: Dict[str, torch.Tensor], device, page_table=None):
+        self.step = step
+        self.host = {k: host[k] for k in self.INPUTS}
+        self.dev = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in self.host.items()}
+        self.page_table = None if page_table is None else page_table.to(device)
+        self.out_attn = torch.empty_like(self.dev["q"])
+        pin = torch.cuda.is_available()
+        Bn = self.host["q"].shape[0]
+        self.out_host = {
+            "attn": torch.empty(self.host["q"].shape, dtype=self.host["q"].dtype, pin_memory=pin),
+            "h": torch.empty(self.host["h"].shape, dtype=self.host["h"].dtype, pin_memory=pin),
+            "tokens": torch.empty(self.host["tokens"].shape, dtype=torch.int32, pin_memory=pin),
+            "is_masked": torch.empty(self.host["is_masked"].shape, dtype=torch.uint8, pin_memory=pin),
+            "n_committed": torch.empty(Bn, dtype=torch.int32, pin_memory=pin),
+            "n_masked": torch.empty(Bn, dtype=torch.int32, pin_memory=pin),
+        }
+        self.h2d_bytes = sum(v.numel() * v.element_size() for v in self.host.values())
+        self.d2h_bytes = sum(v.numel() * v.element_size() for v in self.out_host.values())
+
+    def run(self) -> Dict[str, torch.Tensor]:
+        for k, v in self.host.items():
+            self.dev[k].copy_(v, non_blocking=True)
+        d = self.dev
+        bufs = StepBuffers(tau=d["tau"], h=d["h"], f=d["f"], q=d["q"], k_blk=d["k_blk"], v_blk=d["v_blk"],
+                           k_ctx=d["k_ctx"], v_ctx=d["v_ctx"], ctx_lens=d["ctx_lens"], page_table=self.page_table,
+                           logits=d["logits"], tokens=d["tokens"], is_masked=d["is_masked"])
+        r = self.step.run(bufs, out_attn=self.out_attn)
+        o = self.out_host
+        o["attn"].copy_(self.out_attn, non_blocking=True)
+        o["h"].copy_(r["h"], non_blocking=True)
+        o["tokens"].copy_(d["tokens"], non_blocking=True)
+        o["is_masked"].copy_(d["is_masked"], non_blocking=True)
+        o["n_committed"].copy_(r["n_committed"], non_blocking=True)
+        o["n_masked"].copy_(r["n_masked"], non_blocking=True)
+        return o

@@ -100,8 +100,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(const SimtParam
       } else if (t < total) {
         src = -2 - (b * p.S + (t - L));
       }
-      s_row[tid] = (t < total) ? src : -1;
-      if (t < total && src == -1) s_row[tid] = -1;
+      s_row[tid] = src;
     }
     __syncthreads();
     for (int i = tid; i < kSimtKeys * D; i += blockDim.x) {
@@ -200,15 +199,24 @@ int attn_simt_launch(const tt_attn_args_t* a, const AttnPlan& /*plan*/, void* ws
   p.hdr = static_cast<WsHeader*>(ws);
   const int M = p.G * p.S;
   dim3 grid((M + kSimtRows - 1) / kSimtRows, p.Hkv, p.B);
-  if (p.d == 64) {
-    const size_t smem = sizeof(float) * (kSimtRows * 64 + 2 * kSimtKeys * 65);
-    cudaFuncSetAttribute(attn_simt_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_simt_kernel<64><<<grid, kSimtThreads, smem, stream>>>(p);
-  } else {
-    const size_t smem = sizeof(float) * (kSimtRows * 128 + 2 * kSimtKeys * 129);
-    cudaFuncSetAttribute(attn_simt_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_simt_kernel<128><<<grid, kSimtThreads, smem, stream>>>(p);
+  static unsigned long long attr_done = 0;   // bit per device ordinal (< 64), set once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  const size_t smem64 = sizeof(float) * (kSimtRows * 64 + 2 * kSimtKeys * 65);
+  const size_t smem128 = sizeof(float) * (kSimtRows * 128 + 2 * kSimtKeys * 129);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(attn_simt_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem64) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(attn_simt_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem128) !=
+            cudaSuccess)
+      return TT_ERR_CUDA;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
+  if (p.d == 64)
+    attn_simt_kernel<64><<<grid, kSimtThreads, smem64, stream>>>(p);
+  else
+    attn_simt_kernel<128><<<grid, kSimtThreads, smem128, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }
 

@@ -5,8 +5,8 @@
 // G query heads of the kv head times the block positions of the tile, packed as M rows
 // m = s * G + g (at most 256 = two 128-row MMA halves), so each key/value tile is read from HBM
 // once per unit. Its keys are ceil(L_b/64) context tiles of 64 tokens followed by one tile holding
-// the S block tokens. All units' tiles are laid end to end and cut into gridDim.x equal ranges,
-// one per persistent CTA (one CTA per SM), so ragged contexts are balanced to within a tile
+// the S block tokens. All units' tiles are laid end to end and cut into min(gridDim.x, tiles)
+// equal ranges, one per persistent CTA (one CTA per SM), so ragged contexts are balanced to within a tile
 // without any host-side knowledge of the lengths. A unit cut between CTAs is finished by the last
 // CTA to arrive (an atomic ticket; no spinning), which merges the per-CTA partial results
 // (O_j normalised, log2-sum-exp_j) into the output.
@@ -93,7 +93,7 @@ struct Smem {
   uint64_t ep_arrive[2], ep_flag[2], drain;
   uint32_t tmem_base;
   int abort_flag;
-  long long range_begin, range_end, total_tiles;
+  long long range_begin, range_end, total_tiles, p_eff;
   int u0;
   long long u0_start;
   int last_flag[2];
@@ -162,7 +162,7 @@ struct SegWalk {
   }
 };
 
-// CTA index owning global tile t when T tiles are cut into P ranges [c*T/P, (c+1)*T/P).
+// CTA index owning global tile t when T tiles are cut into P ranges [c*T/P, (c+1)*T/P), P <= T.
 __device__ __forceinline__ long long owner_cta(long long t, long long T, long long P) {
   return ((t + 1) * P - 1) / T;
 }
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   Smem& sm = *reinterpret_cast<Smem*>(smem + kSmemBar);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long P = gridDim.x, c = blockIdx.x;
+  const long long P = gridDim.x, cta = blockIdx.x;
 
   // ---- 1. this CTA's tile range and the unit where it starts (warp 0)
   if (warp == 0) {
@@ -186,7 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
       T += n;
     }
-    const long long rb = c * T / P, re = (c + 1) * T / P;
+    // with fewer tiles than CTAs only the first T CTAs work (one tile each), so every working
+    // CTA owns a non-empty range and the CTAs of a unit are consecutive
+    const long long Pe = T < P ? T : P;
+    const long long rb = cta < Pe ? cta * T / Pe : T, re = cta < Pe ? (cta + 1) * T / Pe : T;
     long long acc = 0;
     int u0 = -1;
     long long u0s = 0;
@@ -210,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
     if (lane == 0) {
       sm.total_tiles = T;
+      sm.p_eff = Pe;
       sm.range_begin = rb;
       sm.range_end = re;
       sm.u0 = u0;
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t s_tm0 = tmem + lane_off + 256u + (uint32_t)(128 * h);
     const uint32_t o_tm = tmem + lane_off + (uint32_t)(kRowsPerHalf * h);
     const float c = p.scale_log2;
-    const long long T = sm.total_tiles;
+    const long long T = sm.total_tiles, Pe = sm.p_eff;
     float* partials = reinterpret_cast<float*>(p.ws + p.off_partials);
     float* plse = reinterpret_cast<float*>(p.ws + p.off_lse);
     int* tickets = reinterpret_cast<int*>(p.ws + p.off_tickets);
@@ -544,9 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       long long c_lo = 0, c_hi = 0;
       size_t slot = 0;
       if (!whole) {
-        c_lo = owner_cta(ustart, T, P);
-        c_hi = owner_cta(ustart + ui.ntiles - 1, T, P);
-        slot = (size_t)w.u + (size_t)c;
+        c_lo = owner_cta(ustart, T, Pe);
+        c_hi = owner_cta(ustart + ui.ntiles - 1, T, Pe);
+        slot = (size_t)w.u + (size_t)cta;
       }
       __nv_bfloat16* orow = p.out + (((size_t)ui.b * p.S + s_idx) * p.Hq + hq) * kD;
       float* prow = partials + (slot * 256 + row) * kD;
@@ -756,9 +760,18 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   p.off_tickets = pl.off_tickets;
   p.off_partials = pl.off_partials;
   p.off_lse = pl.off_lse;
-  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-      cudaSuccess)
-    return TT_ERR_CUDA;
+  // the shared-memory opt-in is per device; set it once so no attribute call happens while a
+  // caller captures the stream into a CUDA graph
+  static unsigned long long attr_done = 0;   // bit per device ordinal (< 64)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+        cudaSuccess)
+      return TT_ERR_CUDA;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
   attn_tc_kernel<<<pl.grid, kThreads, kSmemBytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }

@@ -24,8 +24,10 @@
  *     word in the caller's workspace, skips the offending work, and tt_get_device_error()
  *     reports it as TT_ERR_DEVICE or TT_ERR_DEVICE_TIMEOUT.
  *   - Inputs must be finite. NaN/Inf inputs give unspecified (but non-faulting) results.
- *   - Workspaces must be zero-filled once before their first use (cudaMemset); the kernels
- *     leave them ready for the next call. Calls that share a workspace must be stream-ordered.
+ *   - Workspaces must be zero-filled (cudaMemset) before their first use. Their layout depends
+ *     on the argument sizes; the kernels restore the merge tickets of that layout to zero, so a
+ *     workspace can be reused without re-zeroing by calls with the same sizes. Zero it again
+ *     before a call with different sizes. Calls sharing a workspace must be stream-ordered.
  */
 #ifndef TT_DENOISE_H_
 #define TT_DENOISE_H_
