@@ -430,16 +430,66 @@ def cpu_baseline(w, inp, ad, logits):
             "sample": f"{k} query tokens of the workload (all heads, adaLN, unmask of that position), {el:.1f} s"}
 
 
+def run_kernel_only(args):
+    """Eager launches of one kernel of the step on the workload (for ncu captures): warmup + steps
+    launches, one input set, no graph; prints the mean launch time from CUDA events."""
+    import torch
+    from denoiser_attention_b200 import api, build, synth
+    build.build()
+    dev = torch.device("cuda", 0)
+    w = synth.workload(args.workload)
+    inp, ad, logits = host_inputs(w)
+    B, S = w.attn.batch, w.attn.block_size
+    q, kb, vb = inp.q.to(dev), inp.k_blk.to(dev), inp.v_blk.to(dev)
+    kc, vc, lens = inp.k_ctx.to(dev), inp.v_ctx.to(dev), inp.ctx_lens.to(dev)
+    table = None if inp.page_table is None else inp.page_table.to(dev)
+    lg = logits.to(dev)
+    tokens = torch.full((B, S), 3, dtype=torch.int32, device=dev)
+    masked = torch.ones((B, S), dtype=torch.uint8, device=dev)
+    weights = {k: getattr(ad, k).to(dev) for k in ("w1", "b1", "w2", "b2", "w3", "b3", "layer_emb", "norm_w")}
+    tau, h, f = ad.tau.to(dev), ad.h.to(dev), ad.f.to(dev)
+    out = torch.empty_like(q)
+
+    def once():
+        if args.kernel == "attn":
+            api.denoise_attention(q, kb, vb, kc, vc, lens, page_table=table, page_size=w.attn.page_size,
+                                  ctx_stride=inp.ctx_stride, out=out)
+        elif args.kernel == "unmask":
+            api.unmask_step(lg, tokens, masked, gamma=w.gamma, want_conf=False)
+        else:
+            mod = api.adaln_cond(tau, weights["w1"], weights["b1"], weights["w2"], weights["b2"], weights["w3"],
+                                 weights["b3"], weights["layer_emb"])
+            api.adaln_norm_modulate(h, weights["norm_w"], mod)
+            api.adaln_gated_residual(h, f, mod)
+
+    for _ in range(args.warmup):
+        once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "launches": args.steps,
+                      "mean_us_incl_host_gaps": 1e3 * e0.elapsed_time(e1) / args.steps}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--kernel", choices=["attn", "unmask", "adaln"], default=None,
+                    help="profiling mode: eager launches of one kernel only (not a bench line)")
+    ap.add_argument("--workload", default=WORKLOAD, help="workload of the --kernel profiling mode")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.kernel:
+        run_kernel_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -3,8 +3,8 @@
 // PixArt-alpha: one global MLP from the diffusion time to shared shift/scale/gate, plus a learned
 // per-layer embedding).
 //
-//   COND             tau -> mod[B][3][D]   two launches: the small F->W->W part per sequence,
-//                                          then the W->3D projection with W3 read once for all B
+//   COND             tau -> mod[B][3][D]   three batched-GEMV launches (F->W, W->W, W->3D), each
+//                                          reading its weight rows once for every sequence
 //   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one CTA per token row
 //   GATED_RESIDUAL   h + gate * f: a vectorised elementwise pass
 // All arithmetic is fp32 (the timestep sinusoid in fp64); bf16 tensors are widened on load and
@@ -26,74 +26,103 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Kernel A: per sequence b, phi(tau_b) -> a1 = SiLU(W1 phi + b1) -> a2 = SiLU(W2 a1 + b2).
-__global__ void __launch_bounds__(kAdalnThreads) adaln_cond_hidden_kernel(const float* __restrict__ tau,
-                                                                          const float* __restrict__ w1,
-                                                                          const float* __restrict__ b1,
-                                                                          const float* __restrict__ w2,
-                                                                          const float* __restrict__ b2, int F,
-                                                                          int W, float* __restrict__ a2_out) {
-  __shared__ float s_phi[1024];
-  __shared__ float s_a1[1024];
-  const int b = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Batched GEMV for the three layers of the conditioning MLP:
+//   y[b][o] = act(sum_i W[o][i] x[b][i] + bias[o]) (+ extra[o])
+// Each warp holds R rows of W in registers (float4 per lane, KW of them per row) and applies them
+// to every batch row; batch rows are staged in shared memory in chunks. kPhi: x is the timestep
+// sinusoid phi(tau_b), computed in the kernel (IN = F); otherwise x is read from global memory.
+constexpr int kGemvBatchChunk = 8;
+constexpr int kGemvMaxIn = 1024;
+
+__device__ __forceinline__ void phi_row(float tau, int F, float* dst, int tid, int nthreads) {
+  // [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)); the angle is reduced
+  // modulo 2 pi in double so that sincos always takes its small-argument path
   const int half = F / 2;
-  const double t = 1000.0 * (double)tau[b];
-  for (int k = tid; k < half; k += blockDim.x) {
-    const double w = exp(-log(10000.0) * (double)k / (double)half);
+  const double t = 1000.0 * (double)tau;
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int k = tid; k < half; k += nthreads) {
+    const double w = exp(-9.2103403719761836 * (double)k / (double)half);   // ln(10000) = 9.2103...
+    double a = t * w;
+    a -= two_pi * rint(a / two_pi);
     double sv, cv;
-    sincos(t * w, &sv, &cv);
-    s_phi[k] = (float)cv;
-    s_phi[half + k] = (float)sv;
-  }
-  __syncthreads();
-  const int nwarps = blockDim.x >> 5;
-  for (int j = warp; j < W; j += nwarps) {
-    const float* row = w1 + (size_t)j * F;
-    float acc = 0.f;
-    for (int i = lane; i < F; i += 32) acc = fmaf(row[i], s_phi[i], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) s_a1[j] = silu_f(acc + b1[j]);
-  }
-  __syncthreads();
-  for (int j = warp; j < W; j += nwarps) {
-    const float* row = w2 + (size_t)j * W;
-    float acc = 0.f;
-    for (int i = lane; i < W; i += 32) acc = fmaf(row[i], s_a1[i], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) a2_out[(size_t)b * W + j] = silu_f(acc + b2[j]);
+    sincos(a, &sv, &cv);
+    dst[k] = (float)cv;
+    dst[half + k] = (float)sv;
   }
 }
 
-// Kernel B: mod[b][o] = W3[o] . a2[b] + b3[o] + emb[o] for o < 3D; one warp per output row o,
-// reading the row once and reusing it for every sequence.
-__global__ void __launch_bounds__(kAdalnThreads) adaln_cond_out_kernel(const float* __restrict__ a2,
-                                                                       const float* __restrict__ w3,
-                                                                       const float* __restrict__ b3,
-                                                                       const float* __restrict__ emb, int B,
-                                                                       int W, int out_rows,
-                                                                       float* __restrict__ mod) {
-  const int lane = threadIdx.x & 31;
-  const int o = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (o >= out_rows) return;
-  float wr[32];
-  const float* row = w3 + (size_t)o * W;
+template <int KW, int R, bool kPhi, bool kSilu>
+__global__ void __launch_bounds__(kAdalnThreads) adaln_gemv_kernel(const float* __restrict__ Wt,
+                                                                   const float* __restrict__ bias,
+                                                                   const float* __restrict__ extra,
+                                                                   const float* __restrict__ x, int B, int IN,
+                                                                   int OUT, float* __restrict__ y) {
+  __shared__ __align__(16) float s_x[kGemvBatchChunk * kGemvMaxIn];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int o0 = (blockIdx.x * (kAdalnThreads / 32) + warp) * R;
+  float4 w[R][KW];
+  float bo[R];
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const int i = lane + 32 * k;
-    wr[k] = (i < W) ? row[i] : 0.f;
-  }
-  const float bias = b3[o] + emb[o];
-  for (int b = 0; b < B; ++b) {
-    const float* x = a2 + (size_t)b * W;
-    float acc = 0.f;
+  for (int r = 0; r < R; ++r) {
+    const int o = o0 + r;
+    bo[r] = 0.f;
+    if (o < OUT) bo[r] = bias[o] + (extra ? extra[o] : 0.f);
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int i = lane + 32 * k;
-      if (i < W) acc = fmaf(wr[k], x[i], acc);
+    for (int k = 0; k < KW; ++k) {
+      const int i = (lane + 32 * k) * 4;
+      w[r][k] = (o < OUT && i < IN) ? *reinterpret_cast<const float4*>(Wt + (size_t)o * IN + i)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    acc = warp_sum(acc);
-    if (lane == 0) mod[(size_t)b * out_rows + o] = acc + bias;
+  }
+  for (int b0 = 0; b0 < B; b0 += kGemvBatchChunk) {
+    const int nb = min(kGemvBatchChunk, B - b0);
+    __syncthreads();
+    if (kPhi) {
+      for (int bb = 0; bb < nb; ++bb) phi_row(x[b0 + bb], IN, s_x + bb * IN, threadIdx.x, blockDim.x);
+    } else {
+      for (int i = threadIdx.x; i < nb * IN; i += blockDim.x) s_x[i] = x[(size_t)b0 * IN + i];
+    }
+    __syncthreads();
+    for (int bb = 0; bb < nb; ++bb) {
+      float acc[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[r] = 0.f;
+#pragma unroll
+      for (int k = 0; k < KW; ++k) {
+        const int i = (lane + 32 * k) * 4;
+        if (i < IN) {
+          const float4 xv = *reinterpret_cast<const float4*>(s_x + bb * IN + i);
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+            acc[r] = fmaf(w[r][k].x, xv.x, fmaf(w[r][k].y, xv.y, fmaf(w[r][k].z, xv.z, fmaf(w[r][k].w, xv.w, acc[r]))));
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float v = warp_sum(acc[r]) + bo[r];
+        if (lane == 0 && o0 + r < OUT) y[(size_t)(b0 + bb) * OUT + o0 + r] = kSilu ? silu_f(v) : v;
+      }
+    }
+  }
+}
+
+template <bool kPhi, bool kSilu>
+static void launch_gemv(const float* Wt, const float* bias, const float* extra, const float* x, int B, int IN, int OUT,
+                        float* y, cudaStream_t stream) {
+  const int kw = (IN + 127) / 128;   // float4 per lane per row
+  const int warps = kAdalnThreads / 32;
+  if (kw <= 1) {
+    adaln_gemv_kernel<1, 4, kPhi, kSilu><<<(OUT + warps * 4 - 1) / (warps * 4), kAdalnThreads, 0, stream>>>(
+        Wt, bias, extra, x, B, IN, OUT, y);
+  } else if (kw <= 2) {
+    adaln_gemv_kernel<2, 4, kPhi, kSilu><<<(OUT + warps * 4 - 1) / (warps * 4), kAdalnThreads, 0, stream>>>(
+        Wt, bias, extra, x, B, IN, OUT, y);
+  } else if (kw <= 4) {
+    adaln_gemv_kernel<4, 2, kPhi, kSilu><<<(OUT + warps * 2 - 1) / (warps * 2), kAdalnThreads, 0, stream>>>(
+        Wt, bias, extra, x, B, IN, OUT, y);
+  } else {
+    adaln_gemv_kernel<8, 1, kPhi, kSilu><<<(OUT + warps - 1) / warps, kAdalnThreads, 0, stream>>>(
+        Wt, bias, extra, x, B, IN, OUT, y);
   }
 }
 
@@ -197,20 +226,19 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_gated_residual_kernel(con
 }
 
 size_t adaln_workspace_bytes(const tt_adaln_args_t* a) {
-  if (a->op == TT_ADALN_COND) return kHeaderBytes + sizeof(float) * (size_t)a->batch * a->mlp_width;
+  if (a->op == TT_ADALN_COND) return kHeaderBytes + 2 * sizeof(float) * (size_t)a->batch * a->mlp_width;
   return kHeaderBytes;
 }
 
 int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
   const int B = a->batch, D = a->hidden;
   if (a->op == TT_ADALN_COND) {
-    float* a2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
-    adaln_cond_hidden_kernel<<<B, kAdalnThreads, 0, stream>>>(a->tau, a->w1, a->b1, a->w2, a->b2, a->freq_dim,
-                                                              a->mlp_width, a2);
-    const int rows = 3 * D;
-    const int per_cta = kAdalnThreads / 32;
-    adaln_cond_out_kernel<<<(rows + per_cta - 1) / per_cta, kAdalnThreads, 0, stream>>>(
-        a2, a->w3, a->b3, a->layer_emb, B, a->mlp_width, rows, a->mod);
+    float* a1 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+    float* a2 = a1 + (size_t)B * a->mlp_width;
+    const int F = a->freq_dim, W = a->mlp_width;
+    launch_gemv<true, true>(a->w1, a->b1, nullptr, a->tau, B, F, W, a1, stream);
+    launch_gemv<false, true>(a->w2, a->b2, nullptr, a1, B, W, W, a2, stream);
+    launch_gemv<false, false>(a->w3, a->b3, a->layer_emb, a2, B, W, 3 * D, a->mod, stream);
   } else if (a->op == TT_ADALN_NORM_MODULATE) {
     const int rows = B * a->block_size;
     if (a->dtype == TT_BF16)

@@ -5,11 +5,13 @@
 // G query heads of the kv head times the block positions of the tile, packed as M rows
 // m = s * G + g (at most 256 = two 128-row MMA halves), so each key/value tile is read from HBM
 // once per unit. Its keys are ceil(L_b/64) context tiles of 64 tokens followed by one tile holding
-// the S block tokens. All units' tiles are laid end to end and cut into min(gridDim.x, tiles)
-// equal ranges, one per persistent CTA (one CTA per SM), so ragged contexts are balanced to within a tile
-// without any host-side knowledge of the lengths. A unit cut between CTAs is finished by the last
-// CTA to arrive (an atomic ticket; no spinning), which merges the per-CTA partial results
-// (O_j normalised, log2-sum-exp_j) into the output.
+// the S block tokens. All units' tiles are laid end to end and cut into Pe = min(gridDim.x, tiles)
+// equal ranges, one per persistent CTA (one CTA per SM), so ragged contexts are balanced to within
+// a tile without any host-side knowledge of the lengths. A CTA that holds a whole unit writes its
+// output directly; a unit cut between CTAs leaves one normalised partial (O_j / l_j and the
+// log2-sum-exp) per CTA, and a second, wide kernel merges them (flash-decoding combine). The
+// merge kernel is launched as a programmatic dependent of the attention kernel, so its launch
+// overlaps the attention tail and it starts reading partials as soon as they are complete.
 //
 // Inside a CTA (384 threads):
 //   warp 0      TMA producer: Q tile of the unit, then K/V tiles into a 4-stage ring
@@ -23,7 +25,7 @@
 // The softmax works in the exp2 domain with the scale folded in; the running maximum used for
 // the exponentials is only raised when a tile's maximum exceeds it by more than 8 (a factor 256),
 // which keeps the O rescale off the common path and stays exact because numerator and
-// denominator use the same stale maximum.
+// denominator use the same stale maximum. Only a rescale waits for the previous PV product.
 #include <cstdio>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -53,6 +55,8 @@ constexpr uint32_t kSmemV = kSmemK + kStages * kKBytesPerStage;
 constexpr uint32_t kSmemBar = kSmemV + kStages * kKBytesPerStage;
 constexpr uint32_t kSmemBytes = kSmemBar + 1024 + 1024;        // barriers/scratch + alignment slack
 
+constexpr int kMergeRows = 32;    // rows per merge CTA (8 warps x 4 rows)
+
 // Instruction descriptors (kind::f16): D fp32, A/B bf16, A K-major.
 constexpr uint32_t make_idesc(int M, int N, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
@@ -72,6 +76,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Workspace: header | meta (total tiles, working CTAs) | unit_start[units + 1] | partials | lse
+struct AttnMeta {
+  long long total_tiles;
+  long long p_eff;
+};
+
 struct TcParams {
   CUtensorMap tm_q, tm_kc, tm_vc, tm_kb, tm_vb;
   const int32_t* ctx_lens;
@@ -83,33 +96,33 @@ struct TcParams {
   __nv_bfloat16* out;
   float* lse;
   uint8_t* ws;
-  size_t off_tickets, off_partials, off_lse;
+  size_t off_meta, off_ustart, off_partials, off_lse;
 };
 
 struct Smem {
   uint64_t q_full, q_empty;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2][2], p_full[2][2], pv_done[2];
-  uint64_t ep_arrive[2], ep_flag[2], drain;
+  uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
   long long range_begin, range_end, total_tiles, p_eff;
   int u0;
   long long u0_start;
-  int last_flag[2];
 };
 
 struct UnitInfo {
   int b, kvh, qt, L, nctx, ntiles;
 };
 
-__device__ __forceinline__ int clamp_len(const TcParams& p, int b, bool report, WsHeader* hdr) {
-  int L = p.ctx_lens[b];
+__device__ __forceinline__ int clamp_len(const int32_t* ctx_lens, int paged, int max_pages, int page_size,
+                                         int ctx_stride, int b, bool report, WsHeader* hdr) {
+  int L = ctx_lens[b];
   if (L < 0) {
     if (report) report_error(hdr, TT_ERR_DEVICE, kDetailNegativeLen);
     L = 0;
   }
-  const int cap = p.paged ? p.max_pages * p.page_size : p.ctx_stride;
+  const int cap = paged ? max_pages * page_size : ctx_stride;
   if (L > cap) {
     if (report) report_error(hdr, TT_ERR_DEVICE, kDetailCtxTooLong);
     L = cap;
@@ -123,7 +136,7 @@ __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int u, bool rep
   const int bk = u / p.qtiles;
   ui.kvh = bk % p.Hkv;
   ui.b = bk / p.Hkv;
-  ui.L = clamp_len(p, ui.b, report, hdr);
+  ui.L = clamp_len(p.ctx_lens, p.paged, p.max_pages, p.page_size, p.ctx_stride, ui.b, report, hdr);
   ui.nctx = (ui.L + kTile - 1) / kTile;
   ui.ntiles = ui.nctx + 1;
   return ui;
@@ -162,7 +175,7 @@ struct SegWalk {
   }
 };
 
-// CTA index owning global tile t when T tiles are cut into P ranges [c*T/P, (c+1)*T/P), P <= T.
+// CTA index owning global tile t when T tiles are cut into P <= T ranges [c*T/P, (c+1)*T/P).
 __device__ __forceinline__ long long owner_cta(long long t, long long T, long long P) {
   return ((t + 1) * P - 1) / T;
 }
@@ -175,7 +188,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long P = gridDim.x, cta = blockIdx.x;
 
-  // ---- 1. this CTA's tile range and the unit where it starts (warp 0)
+  // ---- 0. prologue that touches no input: barriers, TMEM, tensor-map prefetch. With a
+  // programmatic launch it overlaps the previous kernel; inputs are read after pdl_wait().
+  if (warp == 0 && lane == 0) {
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.kv_full[i], 1);
+      mbar_init(&sm.kv_empty[i], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      for (int bf = 0; bf < 2; ++bf) {
+        mbar_init(&sm.s_full[h][bf], 1);
+        mbar_init(&sm.p_full[h][bf], kRowsPerHalf);
+        mbar_init(&sm.pv_done[h][bf], 1);
+      }
+    }
+    mbar_init(&sm.drain, 1);
+    fence_barrier_init();
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_kc);
+    prefetch_tmap(&p.tm_vc);
+    prefetch_tmap(&p.tm_kb);
+    prefetch_tmap(&p.tm_vb);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  pdl_trigger();
+  pdl_wait();
+
+  // ---- 1. this CTA's tile range and the unit where it starts (warp 0); CTA 0 also records the
+  // partition for the merge kernel
   if (warp == 0) {
     long long T = 0;
     for (int base = 0; base < p.units; base += 32) {
@@ -193,7 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     long long acc = 0;
     int u0 = -1;
     long long u0s = 0;
-    for (int base = 0; base < p.units && u0 < 0; base += 32) {
+    int32_t* ustart_out = reinterpret_cast<int32_t*>(p.ws + p.off_ustart);
+    const bool record = (blockIdx.x == 0);
+    for (int base = 0; base < p.units && (u0 < 0 || record); base += 32) {
       const int u = base + lane;
       const int n = (u < p.units) ? unit_info(p, u, false, hdr).ntiles : 0;
       int incl = n;
@@ -203,8 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (lane >= o) incl += y;
       }
       const long long lo = acc + incl - n, hi = acc + incl;
+      if (record && u < p.units) ustart_out[u] = (int32_t)lo;
       const unsigned hit = __ballot_sync(0xffffffffu, u < p.units && lo <= rb && rb < hi);
-      if (hit) {
+      if (hit && u0 < 0) {
         const int src = __ffs(hit) - 1;
         u0 = base + src;
         u0s = __shfl_sync(0xffffffffu, lo, src);
@@ -219,43 +268,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       sm.u0 = u0;
       sm.u0_start = u0s;
       sm.abort_flag = 0;
-    }
-  }
-  __syncthreads();
-  if (sm.range_begin >= sm.range_end || sm.u0 < 0) return;   // uniform: nothing to do
-
-  const int M = p.G * p.s_per_tile;               // query rows per unit (<= 256)
-  const int nh = (M > kRowsPerHalf) ? 2 : 1;      // active 128-row halves
-
-  // ---- 2. barriers and TMEM
-  if (warp == 0 && lane == 0) {
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm.kv_full[i], 1);
-      mbar_init(&sm.kv_empty[i], 1);
-    }
-    for (int h = 0; h < 2; ++h) {
-      for (int bf = 0; bf < 2; ++bf) {
-        mbar_init(&sm.s_full[h][bf], 1);
-        mbar_init(&sm.p_full[h][bf], kRowsPerHalf);
+      if (record) {
+        ustart_out[p.units] = (int32_t)T;
+        AttnMeta* meta = reinterpret_cast<AttnMeta*>(p.ws + p.off_meta);
+        meta->total_tiles = T;
+        meta->p_eff = Pe;
       }
-      mbar_init(&sm.pv_done[h], 1);
-      mbar_init(&sm.ep_arrive[h], kRowsPerHalf);
-      mbar_init(&sm.ep_flag[h], 1);
     }
-    mbar_init(&sm.drain, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, kTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
+  const bool has_work = sm.range_begin < sm.range_end && sm.u0 >= 0;
+
+  const int M = p.G * p.s_per_tile;               // query rows per unit (<= 256)
+  const int nh = (M > kRowsPerHalf) ? 2 : 1;      // active 128-row halves
 
   auto fail = [&](uint32_t detail) {
     report_error(hdr, TT_ERR_DEVICE_TIMEOUT, detail);
@@ -266,14 +294,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const uint32_t sK = smem_u32(smem + kSmemK);
   const uint32_t sV = smem_u32(smem + kSmemV);
 
-  if (warp == 0) {
+  if (!has_work) {
+    // nothing to do (more CTAs than tiles)
+  } else if (warp == 0) {
     // ======================= TMA producer
     if (lane == 0) {
-      prefetch_tmap(&p.tm_q);
-      prefetch_tmap(&p.tm_kc);
-      prefetch_tmap(&p.tm_vc);
-      prefetch_tmap(&p.tm_kb);
-      prefetch_tmap(&p.tm_vb);
       SegWalk w;
       w.init(p, sm, hdr);
       long long f = 0;
@@ -377,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const uint64_t bdesc = sdesc_sw128(sV + stage * kKBytesPerStage + kk * 2048, kKVBoxBytes, 1024);
             mma_ts(d_tm, p_tm + 8u * kk, bdesc, kIdescPV, (first && kk == 0) ? 0u : 1u);
           }
-          tc_commit(&sm.pv_done[h]);
+          tc_commit(&sm.pv_done[h][bf]);
         }
         tc_commit(&sm.kv_empty[stage]);
         return true;
@@ -433,15 +458,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t s_tm0 = tmem + lane_off + 256u + (uint32_t)(128 * h);
     const uint32_t o_tm = tmem + lane_off + (uint32_t)(kRowsPerHalf * h);
-    const float c = p.scale_log2;
-    const long long T = sm.total_tiles, Pe = sm.p_eff;
+    const float sc = p.scale_log2;
     float* partials = reinterpret_cast<float*>(p.ws + p.off_partials);
     float* plse = reinterpret_cast<float*>(p.ws + p.off_lse);
-    int* tickets = reinterpret_cast<int*>(p.ws + p.off_tickets);
     SegWalk w;
     w.init(p, sm, hdr);
     long long f = 0;
-    int npart = 0;
     bool ok = true;
     while (ok && !w.done()) {
       int kb, ke;
@@ -457,18 +479,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           break;
         }
         tc_fence_after();
-        uint32_t sr[2][32];
-        tmem_ld32(s_tm0 + 64u * bf, sr[0]);
-        tmem_ld32(s_tm0 + 64u * bf + 32u, sr[1]);
+        uint32_t sr[64];
+        tmem_ld32(s_tm0 + 64u * bf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(s_tm0 + 64u * bf + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
-        float x[64];
+        // row maximum of the raw scores (the scale is positive, so it commutes with max)
         float mt = -INFINITY;
+        if (valid >= kTile) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float v = (j < valid) ? __uint_as_float(sr[j >> 5][j & 31]) * c : -INFINITY;
-          x[j] = v;
-          mt = fmaxf(mt, v);
+          for (int j = 0; j < 64; ++j) mt = fmaxf(mt, __uint_as_float(sr[j]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            if (j >= valid) sr[j] = __float_as_uint(-INFINITY);
+            mt = fmaxf(mt, __uint_as_float(sr[j]));
+          }
         }
+        mt *= sc;
         const bool first = (k == kb);
         bool resc = false;
         float m_new = m_used;
@@ -480,37 +507,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         const float factor = resc ? ex2(m_used - m_new) : 1.0f;
         uint32_t pk[32];
-        float psum = 0.f;
+        float psum0 = 0.f, psum1 = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float p0 = ex2(x[2 * j] - m_new);
-          const float p1 = ex2(x[2 * j + 1] - m_new);
-          psum += p0 + p1;
+          const float p0 = ex2(fmaf(__uint_as_float(sr[2 * j]), sc, -m_new));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[2 * j + 1]), sc, -m_new));
+          psum0 += p0;
+          psum1 += p1;
           pk[j] = pack_bf16x2(p0, p1);
         }
-        l = l * factor + psum;
+        l = l * factor + (psum0 + psum1);
         tmem_st32(s_tm0 + 64u * bf, pk);
-        tmem_wait_st();
-        if (!first) {
-          if (!mbar_wait_bounded(&sm.pv_done[h], (uint32_t)((f - 1) & 1), abort_flag)) {
+        if (resc) {
+          // O holds the sum up to tile f-1: wait for that PV product, then rescale it
+          const long long pf = f - 1;
+          if (!mbar_wait_bounded(&sm.pv_done[h][pf & 1], (uint32_t)((pf >> 1) & 1), abort_flag)) {
             fail(kDetailWaitPvDone);
             ok = false;
             break;
           }
           tc_fence_after();
-          if (resc) {
 #pragma unroll 1
-            for (int cb = 0; cb < kD / 32; ++cb) {
-              uint32_t orr[32];
-              tmem_ld32(o_tm + 32u * cb, orr);
-              tmem_wait_ld();
+          for (int cb = 0; cb < kD / 32; ++cb) {
+            uint32_t orr[32];
+            tmem_ld32(o_tm + 32u * cb, orr);
+            tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * factor);
-              tmem_st32(o_tm + 32u * cb, orr);
-            }
-            tmem_wait_st();
+            for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * factor);
+            tmem_st32(o_tm + 32u * cb, orr);
           }
         }
+        tmem_wait_st();
         if (h == 0 && k < ui.nctx && valid < kTile) {
           // Rows past the end of the context hold whatever the caller's slab or page holds
           // there; P is 0 for them, but 0 * NaN would still poison O, so zero those V rows
@@ -530,14 +557,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         mbar_arrive(&sm.p_full[h][bf]);
       }
       if (!ok) break;
-      // ---- epilogue of the segment: O / l for this row
-      if (!mbar_wait_bounded(&sm.pv_done[h], (uint32_t)((f - 1) & 1), abort_flag)) {
+      // ---- epilogue of the segment: wait for the last PV product, then O / l for this row
+      const long long lf = f - 1;
+      if (!mbar_wait_bounded(&sm.pv_done[h][lf & 1], (uint32_t)((lf >> 1) & 1), abort_flag)) {
         fail(kDetailWaitPvDone);
         ok = false;
         break;
       }
       tc_fence_after();
-      const long long ustart = w.ustart;
       const bool whole = (kb == 0) && (ke == ui.ntiles);
       const int s_cnt = min(p.s_per_tile, p.S - ui.qt * p.s_per_tile);
       const bool row_valid = row < p.G * s_cnt;
@@ -545,13 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int hq = ui.kvh * p.G + row % p.G;
       const float inv_l = 1.0f / l;
       const float lse2 = m_used + log2f(l);
-      long long c_lo = 0, c_hi = 0;
-      size_t slot = 0;
-      if (!whole) {
-        c_lo = owner_cta(ustart, T, Pe);
-        c_hi = owner_cta(ustart + ui.ntiles - 1, T, Pe);
-        slot = (size_t)w.u + (size_t)cta;
-      }
+      const size_t slot = (size_t)w.u + (size_t)cta;   // unique per (unit, CTA) pair
       __nv_bfloat16* orow = p.out + (((size_t)ui.b * p.S + s_idx) * p.Hq + hq) * kD;
       float* prow = partials + (slot * 256 + row) * kD;
 #pragma unroll 1
@@ -580,75 +601,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
       }
-      if (whole) {
-        if (row_valid && p.lse) p.lse[((size_t)ui.b * p.Hq + hq) * p.S + s_idx] = lse2 * 0.69314718055994531f;
-      } else {
-        // hand this CTA's share to the unit's last-arriving CTA (per half; bounded waits only)
-        if (row_valid) plse[slot * 256 + row] = lse2;
-        __threadfence();
-        mbar_arrive(&sm.ep_arrive[h]);
-        if (t == 0) {
-          int last = 0;
-          if (mbar_wait_bounded(&sm.ep_arrive[h], (uint32_t)(npart & 1), abort_flag)) {
-            const int old = atomicAdd(tickets + 2 * w.u + h, 1);
-            last = (old == (int)(c_hi - c_lo)) ? 1 : 0;
-            if (last) tickets[2 * w.u + h] = 0;
-            __threadfence();
-          } else {
-            fail(kDetailWaitTicket);
-          }
-          sm.last_flag[h] = last;
-          mbar_arrive(&sm.ep_flag[h]);
-        }
-        if (!mbar_wait_bounded(&sm.ep_flag[h], (uint32_t)(npart & 1), abort_flag)) {
-          fail(kDetailWaitTicket);
-          ok = false;
-          break;
-        }
-        ++npart;
-        if (sm.last_flag[h] && row_valid) {
-          // merge the partials of every CTA that worked on this unit
-          float mx = -INFINITY;
-          for (long long cc = c_lo; cc <= c_hi; ++cc)
-            mx = fmaxf(mx, __ldcg(plse + ((size_t)w.u + (size_t)cc) * 256 + row));
-          float wsum = 0.f;
-          for (long long cc = c_lo; cc <= c_hi; ++cc) wsum += ex2(__ldcg(plse + ((size_t)w.u + (size_t)cc) * 256 + row) - mx);
-          const float inv_w = 1.0f / wsum;
-#pragma unroll 1
-          for (int cb = 0; cb < kD / 8; ++cb) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (long long cc = c_lo; cc <= c_hi; ++cc) {
-              const size_t sl = (size_t)w.u + (size_t)cc;
-              const float wj = ex2(__ldcg(plse + sl * 256 + row) - mx) * inv_w;
-              const float4* src = reinterpret_cast<const float4*>(partials + (sl * 256 + row) * kD + cb * 8);
-              const float4 a = __ldcg(src), bq = __ldcg(src + 1);
-              acc[0] = fmaf(wj, a.x, acc[0]);
-              acc[1] = fmaf(wj, a.y, acc[1]);
-              acc[2] = fmaf(wj, a.z, acc[2]);
-              acc[3] = fmaf(wj, a.w, acc[3]);
-              acc[4] = fmaf(wj, bq.x, acc[4]);
-              acc[5] = fmaf(wj, bq.y, acc[5]);
-              acc[6] = fmaf(wj, bq.z, acc[6]);
-              acc[7] = fmaf(wj, bq.w, acc[7]);
-            }
-            uint4 v;
-            v.x = pack_bf16x2(acc[0], acc[1]);
-            v.y = pack_bf16x2(acc[2], acc[3]);
-            v.z = pack_bf16x2(acc[4], acc[5]);
-            v.w = pack_bf16x2(acc[6], acc[7]);
-            reinterpret_cast<uint4*>(orow)[cb] = v;
-          }
-          if (p.lse) p.lse[((size_t)ui.b * p.Hq + hq) * p.S + s_idx] = (mx + log2f(wsum)) * 0.69314718055994531f;
+      if (row_valid) {
+        if (whole) {
+          if (p.lse) p.lse[((size_t)ui.b * p.Hq + hq) * p.S + s_idx] = lse2 * 0.69314718055994531f;
+        } else {
+          plse[slot * 256 + row] = lse2;
         }
       }
       w.advance(p, hdr);
     }
   }
 
-  // ---- 3. teardown: every MMA has completed before the epilogues read O; on an abort path make
-  // sure nothing is still in flight before TMEM is released.
+  // ---- 3. teardown: all tensor-core work issued by the MMA thread completes before TMEM is
+  // released (on the normal path it already has; on an abort path this drains it)
   if (warp == 1 && lane == 0) {
-    // all tensor-core work issued by this thread completes before TMEM is released
     tc_commit(&sm.drain);
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
@@ -658,6 +624,94 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Merges the partials of units cut between CTAs. One CTA per (unit, 32 query rows); a warp
+// merges 4 rows, each lane 4 of the 128 dims, reading every contributor's row with coalesced
+// 512-byte loads: O = sum_j 2^(lse_j - M) O_j / sum_j 2^(lse_j - M), M = max_j lse_j.
+struct MergeParams {
+  int32_t S, Hq, Hkv, G, qtiles, s_per_tile, units;
+  __nv_bfloat16* out;
+  float* lse;
+  const uint8_t* ws;
+  size_t off_meta, off_ustart, off_partials, off_lse;
+};
+
+__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
+  pdl_wait();
+  const int u = blockIdx.x;
+  const AttnMeta* meta = reinterpret_cast<const AttnMeta*>(p.ws + p.off_meta);
+  const int32_t* ustart = reinterpret_cast<const int32_t*>(p.ws + p.off_ustart);
+  const long long T = meta->total_tiles, Pe = meta->p_eff;
+  if (T <= 0) return;
+  const long long us = ustart[u], ue = ustart[u + 1];
+  const long long c_lo = owner_cta(us, T, Pe), c_hi = owner_cta(ue - 1, T, Pe);
+  if (c_lo == c_hi) return;   // a whole unit: the attention kernel wrote it
+  const int qt = u % p.qtiles;
+  const int bk = u / p.qtiles;
+  const int kvh = bk % p.Hkv, b = bk / p.Hkv;
+  const int s_cnt = min(p.s_per_tile, p.S - qt * p.s_per_tile);
+  const int nrows = p.G * s_cnt;
+  const float* partials = reinterpret_cast<const float*>(p.ws + p.off_partials);
+  const float* plse = reinterpret_cast<const float*>(p.ws + p.off_lse);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = (int)(c_hi - c_lo + 1);
+  for (int rr = 0; rr < 4; ++rr) {
+    const int row = blockIdx.y * kMergeRows + warp * 4 + rr;
+    if (row >= nrows) break;
+    // per-contributor log2-sum-exp: lanes take contributors, then a warp max / sum
+    float mx = -INFINITY;
+    for (int j = lane; j < n; j += 32) mx = fmaxf(mx, plse[((size_t)u + (size_t)(c_lo + j)) * 256 + row]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const float wl = (j < n) ? ex2(plse[((size_t)u + (size_t)(c_lo + j)) * 256 + row] - mx) : 0.f;
+      float ws_part = wl;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ws_part += __shfl_xor_sync(0xffffffffu, ws_part, o);
+      wsum += ws_part;
+      const int cnt = min(32, n - j0);
+      int jj = 0;
+      for (; jj + 4 <= cnt; jj += 4) {
+        float4 v[4];
+        float wv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          wv[q] = __shfl_sync(0xffffffffu, wl, jj + q);
+          const size_t sl = (size_t)u + (size_t)(c_lo + j0 + jj + q);
+          v[q] = reinterpret_cast<const float4*>(partials + (sl * 256 + row) * kD)[lane];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc.x = fmaf(wv[q], v[q].x, acc.x);
+          acc.y = fmaf(wv[q], v[q].y, acc.y);
+          acc.z = fmaf(wv[q], v[q].z, acc.z);
+          acc.w = fmaf(wv[q], v[q].w, acc.w);
+        }
+      }
+      for (; jj < cnt; ++jj) {
+        const float wq = __shfl_sync(0xffffffffu, wl, jj);
+        const size_t sl = (size_t)u + (size_t)(c_lo + j0 + jj);
+        const float4 v = reinterpret_cast<const float4*>(partials + (sl * 256 + row) * kD)[lane];
+        acc.x = fmaf(wq, v.x, acc.x);
+        acc.y = fmaf(wq, v.y, acc.y);
+        acc.z = fmaf(wq, v.z, acc.z);
+        acc.w = fmaf(wq, v.w, acc.w);
+      }
+    }
+    const float inv = 1.0f / wsum;
+    const int s_idx = qt * p.s_per_tile + row / p.G;
+    const int hq = kvh * p.G + row % p.G;
+    __nv_bfloat16* orow = p.out + (((size_t)b * p.S + s_idx) * p.Hq + hq) * kD;
+    uint2 o;
+    o.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    o.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(orow)[lane] = o;
+    if (p.lse && lane == 0) p.lse[((size_t)b * p.Hq + hq) * p.S + s_idx] = (mx + log2f(wsum)) * 0.69314718055994531f;
   }
 }
 
@@ -687,6 +741,23 @@ bool make_map(CUtensorMap* m, const void* base, int heads, long long rows, int b
   return r == CUDA_SUCCESS;
 }
 
+// Launch with the programmatic-stream-serialization attribute: the kernel may start while the
+// previous kernel on the stream finishes; it reads no input before griddepcontrol.wait.
+template <typename Kern, typename Params>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const Params& prm) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, prm);
+}
+
 }  // namespace
 
 bool attn_tc_supported(const tt_attn_args_t* a) {
@@ -698,7 +769,7 @@ bool attn_tc_supported(const tt_attn_args_t* a) {
   // TMA needs 16-byte aligned bases
   const uintptr_t al = reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->k_blk) |
                        reinterpret_cast<uintptr_t>(a->v_blk) | reinterpret_cast<uintptr_t>(a->k_ctx) |
-                       reinterpret_cast<uintptr_t>(a->v_ctx);
+                       reinterpret_cast<uintptr_t>(a->v_ctx) | reinterpret_cast<uintptr_t>(a->out);
   if (al & 15) return false;
   return true;
 }
@@ -718,7 +789,8 @@ AttnPlan attn_tc_plan(const tt_attn_args_t* a, int num_sms) {
     off = (off + bytes + 255) & ~size_t(255);
     return o;
   };
-  pl.off_tickets = take(sizeof(int) * 2 * (size_t)pl.units);
+  pl.off_meta = take(sizeof(AttnMeta));
+  pl.off_ustart = take(sizeof(int32_t) * ((size_t)pl.units + 1));
   pl.off_partials = take(sizeof(float) * pl.slots * 256 * kD);
   pl.off_lse = take(sizeof(float) * pl.slots * 256);
   pl.total = off;
@@ -757,7 +829,8 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   p.out = static_cast<__nv_bfloat16*>(a->out);
   p.lse = a->lse;
   p.ws = static_cast<uint8_t*>(ws);
-  p.off_tickets = pl.off_tickets;
+  p.off_meta = pl.off_meta;
+  p.off_ustart = pl.off_ustart;
   p.off_partials = pl.off_partials;
   p.off_lse = pl.off_lse;
   // the shared-memory opt-in is per device; set it once so no attribute call happens while a
@@ -772,8 +845,27 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
       return TT_ERR_CUDA;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  attn_tc_kernel<<<pl.grid, kThreads, kSmemBytes, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
+  if (launch_pdl(attn_tc_kernel, dim3(pl.grid), dim3(kThreads), kSmemBytes, stream, p) != cudaSuccess)
+    return TT_ERR_CUDA;
+  MergeParams mp{};
+  mp.S = p.S;
+  mp.Hq = p.Hq;
+  mp.Hkv = p.Hkv;
+  mp.G = G;
+  mp.qtiles = pl.qtiles;
+  mp.s_per_tile = pl.s_per_tile;
+  mp.units = pl.units;
+  mp.out = p.out;
+  mp.lse = p.lse;
+  mp.ws = p.ws;
+  mp.off_meta = pl.off_meta;
+  mp.off_ustart = pl.off_ustart;
+  mp.off_partials = pl.off_partials;
+  mp.off_lse = pl.off_lse;
+  const int M = G * pl.s_per_tile;
+  const dim3 mgrid(pl.units, (M + kMergeRows - 1) / kMergeRows);
+  if (launch_pdl(attn_merge_kernel, mgrid, dim3(256), 0, stream, mp) != cudaSuccess) return TT_ERR_CUDA;
+  return TT_OK;
 }
 
 }  // namespace tt

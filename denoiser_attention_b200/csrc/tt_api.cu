@@ -25,7 +25,7 @@ static int validate_attn(const tt_attn_args_t* a) {
   if (a->dtype != TT_F32 && a->dtype != TT_BF16) return TT_ERR_INVALID_ARGUMENT;
   if (!a->q || !a->k_blk || !a->v_blk || !a->k_ctx || !a->v_ctx || !a->ctx_lens || !a->out)
     return TT_ERR_INVALID_ARGUMENT;
-  if (!(a->softmax_scale > 0.f) && !(a->softmax_scale < 0.f)) return TT_ERR_INVALID_ARGUMENT;
+  if (!(a->softmax_scale > 0.f) || !(a->softmax_scale < 3.0e38f)) return TT_ERR_INVALID_ARGUMENT;
   if (a->page_table) {
     if (a->page_size < 1 || a->max_pages_per_seq < 1 || a->num_pages < 1) return TT_ERR_INVALID_ARGUMENT;
   } else {
@@ -61,6 +61,8 @@ static int validate_adaln(const tt_adaln_args_t* a) {
         return TT_ERR_INVALID_ARGUMENT;
       if (a->freq_dim < 2 || (a->freq_dim & 1) || a->mlp_width < 1) return TT_ERR_INVALID_ARGUMENT;
       if (a->freq_dim > 1024 || a->mlp_width > 1024) return TT_ERR_UNSUPPORTED;
+      if ((a->freq_dim & 3) || (a->mlp_width & 3)) return TT_ERR_UNSUPPORTED;
+      if (!aligned16(a->w1) || !aligned16(a->w2) || !aligned16(a->w3)) return TT_ERR_UNSUPPORTED;
       return TT_OK;
     case TT_ADALN_NORM_MODULATE:
     case TT_ADALN_GATED_RESIDUAL: {

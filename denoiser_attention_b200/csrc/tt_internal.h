@@ -14,8 +14,7 @@ struct UnmaskLayout {
   size_t row_cnt, seq_cnt, partials, conf, argmax, total;
 };
 struct UnmaskPlan {
-  int chunks;
-  int chunk_elems;
+  int grid;            // CTAs, each streaming an equal share of the logits
   UnmaskLayout layout;
 };
 UnmaskPlan unmask_plan(const tt_unmask_args_t* a, int num_sms);
@@ -31,7 +30,8 @@ struct AttnPlan {
   int qtiles;          // query-row tiles per (sequence, kv head)
   int s_per_tile;      // block positions per query-row tile
   int units;           // batch * kv heads * qtiles
-  size_t off_tickets;  // int32 [units]
+  size_t off_meta;     // total tiles and working CTAs of the partition
+  size_t off_ustart;   // int32 [units + 1]: first global tile of each unit
   size_t off_partials; // float [slots][rows][d]
   size_t off_lse;      // float [slots][rows]
   size_t slots;

@@ -2,11 +2,15 @@
 // "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Context".
 //
 // One pass over the vocabulary logits computes, per block position, the softmax maximum
-// probability (confidence) and the argmax token; the last CTA to finish a sequence's positions
-// then applies the commit rule to that sequence. Logits are read once, with 128-bit loads.
+// probability (confidence) and the argmax token; the CTA that finishes the last position of a
+// sequence then applies the commit rule to that sequence. Logits are read once, with 128-bit
+// streaming loads, 8 in flight per thread.
 //
-// Grid: one CTA per (row, chunk) where a row is one (sequence, position) and a chunk is a
-// contiguous slice of the vocabulary, so that even 128 rows fill all SMs. Per thread the running
+// Work split: the logits of all positions are one flat array of 16-byte vectors, cut into equal
+// contiguous ranges, one per CTA (4 CTAs per SM), so every SM streams the same number of bytes
+// whatever the vocabulary size. A range covers the tail of one position and the head of the next
+// at most a few times; a position cut between CTAs is finished by the last of them to arrive (an
+// atomic ticket; no spinning), which merges the per-CTA partial states. Per thread the running
 // state is (m, s, idx): the largest raw logit seen, s = sum exp(c (x - m)) with
 // c = inv_temperature * log2(e) evaluated as exp2, and the lowest index attaining m. States merge
 // associatively; ties keep the lower token index at every level.
@@ -71,8 +75,9 @@ struct VecTraits<__nv_bfloat16> {
 struct UnmaskParams {
   const void* logits;
   int32_t vocab;
-  int32_t chunk_elems;   // multiple of the vector width
-  int32_t chunks;        // C
+  int32_t vec_per_row;   // vocab / vector width
+  long long total_vec;   // rows * vec_per_row
+  long long p_eff;       // working CTAs = min(gridDim.x, total_vec)
   int32_t rows;          // B*S
   int32_t block_size;    // S
   float c;               // inv_temperature * log2(e)
@@ -91,7 +96,13 @@ struct UnmaskParams {
 };
 
 constexpr int kUnmaskThreads = 256;
-constexpr int kUnmaskUnroll = 4;
+constexpr int kUnmaskUnroll = 8;
+constexpr int kUnmaskCtasPerSm = 4;
+
+// CTA owning vector v when E vectors are cut into P <= E ranges [c*E/P, (c+1)*E/P).
+__device__ __forceinline__ long long owner_of(long long v, long long E, long long P) {
+  return ((v + 1) * P - 1) / E;
+}
 
 // Commit rule for one sequence, run by the whole CTA.
 __device__ void commit_sequence(const UnmaskParams& p, int b, const float* conf_ws, const int32_t* arg_ws) {
@@ -146,118 +157,126 @@ template <typename T>
 __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskParams p) {
   using VT = VecTraits<T>;
   constexpr int N = VT::kN;
-  const int row = blockIdx.x / p.chunks;
-  const int chunk = blockIdx.x - row * p.chunks;
+  const long long cta = blockIdx.x;
+  if (cta >= p.p_eff) return;
   const int tid = threadIdx.x;
-  const T* rowp = reinterpret_cast<const T*>(p.logits) + (size_t)row * p.vocab;
-  const int begin = chunk * p.chunk_elems;
-  const int end = min(p.vocab, begin + p.chunk_elems);
-  const int nvec = (end - begin) / N;
-  const uint4* vp = reinterpret_cast<const uint4*>(rowp + begin);
   const float c = p.c;
-
-  float m = -INFINITY, s = 0.f;
-  int32_t idx = 0x7fffffff;
-
-  auto consume = [&](const uint4& raw, int vbase) {
-    float x[N];
-    VT::to_float(raw, x);
-    if (p.exclude_mask_token) {
-      const int r = p.mask_token_id - vbase;
-      if (r >= 0 && r < N) x[r] = -INFINITY;
-    }
-    float vm = x[0];
-    int vi = 0;
-#pragma unroll
-    for (int k = 1; k < N; ++k) {
-      if (x[k] > vm) { vm = x[k]; vi = k; }
-    }
-    if (vm > m) {
-      s = (m == -INFINITY) ? 0.f : s * ex2(c * (m - vm));
-      m = vm;
-      idx = vbase + vi;
-    }
-    const float nmc = -c * m;
-#pragma unroll
-    for (int k = 0; k < N; ++k) s += ex2(fmaf(x[k], c, nmc));
-  };
-
-  int v = tid;
-  for (; v + (kUnmaskUnroll - 1) * kUnmaskThreads < nvec; v += kUnmaskUnroll * kUnmaskThreads) {
-    uint4 raw[kUnmaskUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnmaskUnroll; ++u) raw[u] = __ldcs(vp + v + u * kUnmaskThreads);
-#pragma unroll
-    for (int u = 0; u < kUnmaskUnroll; ++u) consume(raw[u], begin + (v + u * kUnmaskThreads) * N);
-  }
-  for (; v < nvec; v += kUnmaskThreads) consume(__ldcs(vp + v), begin + v * N);
-
-  // ---- CTA reduction (warp shuffles, then across warps), keeping the lowest index on ties
-  RedState st{m, s, idx};
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    RedState o;
-    o.m = __shfl_xor_sync(0xffffffffu, st.m, off);
-    o.s = __shfl_xor_sync(0xffffffffu, st.s, off);
-    o.idx = __shfl_xor_sync(0xffffffffu, st.idx, off);
-    st = red_combine(st, o, c);
-  }
-  __shared__ RedState s_red[kUnmaskThreads / 32];
-  __shared__ int s_flag;
-  const int warp = tid >> 5, lane = tid & 31;
-  if (lane == 0) s_red[warp] = st;
-  __syncthreads();
+  const long long E = p.total_vec, Pe = p.p_eff;
+  const long long vbeg = cta * E / Pe, vend = (cta + 1) * E / Pe;
+  const uint4* base = reinterpret_cast<const uint4*>(p.logits);
 
   float* conf_ws = reinterpret_cast<float*>(p.ws + p.off_conf);
   int32_t* arg_ws = reinterpret_cast<int32_t*>(p.ws + p.off_argmax);
   int* row_cnt = reinterpret_cast<int*>(p.ws + p.off_row_cnt);
   int* seq_cnt = reinterpret_cast<int*>(p.ws + p.off_seq_cnt);
   UnmaskPartial* parts = reinterpret_cast<UnmaskPartial*>(p.ws + p.off_partials);
+  __shared__ RedState s_red[kUnmaskThreads / 32];
+  __shared__ int s_flag;
+  const int warp = tid >> 5, lane = tid & 31;
 
-  if (tid == 0) {
-    RedState r = s_red[0];
-    for (int w = 1; w < kUnmaskThreads / 32; ++w) r = red_combine(r, s_red[w], c);
-    bool row_done = true;
-    if (p.chunks > 1) {
-      parts[(size_t)row * p.chunks + chunk] = UnmaskPartial{r.m, r.s, r.idx, 0};
-      __threadfence();
-      const int old = atomicAdd(row_cnt + row, 1);
-      row_done = (old == p.chunks - 1);
-      if (row_done) {
-        row_cnt[row] = 0;
+  for (long long seg = vbeg; seg < vend;) {
+    const int row = (int)(seg / p.vec_per_row);
+    const long long row_beg = (long long)row * p.vec_per_row;
+    const long long seg_end = min(vend, row_beg + p.vec_per_row);
+    const int vb = (int)(seg - row_beg), ve = (int)(seg_end - row_beg);   // vectors of this row
+    const uint4* vp = base + row_beg;
+
+    float m = -INFINITY, s = 0.f;
+    int32_t idx = 0x7fffffff;
+    auto consume = [&](const uint4& raw, int vi_global) {
+      const int vbase = vi_global * N;
+      float x[N];
+      VT::to_float(raw, x);
+      if (p.exclude_mask_token) {
+        const int r = p.mask_token_id - vbase;
+        if (r >= 0 && r < N) x[r] = -INFINITY;
+      }
+      float vm = x[0];
+      int vi = 0;
+#pragma unroll
+      for (int k = 1; k < N; ++k) {
+        if (x[k] > vm) { vm = x[k]; vi = k; }
+      }
+      if (vm > m) {
+        s = (m == -INFINITY) ? 0.f : s * ex2(c * (m - vm));
+        m = vm;
+        idx = vbase + vi;
+      }
+      const float nmc = -c * m;
+#pragma unroll
+      for (int k = 0; k < N; ++k) s += ex2(fmaf(x[k], c, nmc));
+    };
+    int v = vb + tid;
+    for (; v + (kUnmaskUnroll - 1) * kUnmaskThreads < ve; v += kUnmaskUnroll * kUnmaskThreads) {
+      uint4 raw[kUnmaskUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnmaskUnroll; ++u) raw[u] = __ldcs(vp + v + u * kUnmaskThreads);
+#pragma unroll
+      for (int u = 0; u < kUnmaskUnroll; ++u) consume(raw[u], v + u * kUnmaskThreads);
+    }
+    for (; v < ve; v += kUnmaskThreads) consume(__ldcs(vp + v), v);
+
+    // ---- CTA reduction (warp shuffles, then across warps), lowest index on ties
+    RedState st{m, s, idx};
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      RedState o;
+      o.m = __shfl_xor_sync(0xffffffffu, st.m, off);
+      o.s = __shfl_xor_sync(0xffffffffu, st.s, off);
+      o.idx = __shfl_xor_sync(0xffffffffu, st.idx, off);
+      st = red_combine(st, o, c);
+    }
+    __syncthreads();   // s_red / s_flag reuse across segments
+    if (lane == 0) s_red[warp] = st;
+    __syncthreads();
+    if (tid == 0) {
+      RedState r = s_red[0];
+      for (int w = 1; w < kUnmaskThreads / 32; ++w) r = red_combine(r, s_red[w], c);
+      const long long c_lo = owner_of(row_beg, E, Pe), c_hi = owner_of(row_beg + p.vec_per_row - 1, E, Pe);
+      bool row_done = true;
+      if (c_hi > c_lo) {
+        const size_t slot = (size_t)row + (size_t)cta;   // unique per (row, CTA) pair
+        parts[slot] = UnmaskPartial{r.m, r.s, r.idx, 0};
         __threadfence();
-        const float4* pp = reinterpret_cast<const float4*>(parts + (size_t)row * p.chunks);
-        float4 q = __ldcg(pp);
-        r = RedState{q.x, q.y, __float_as_int(q.z)};
-        for (int k = 1; k < p.chunks; ++k) {
-          q = __ldcg(pp + k);
-          r = red_combine(r, RedState{q.x, q.y, __float_as_int(q.z)}, c);
+        const int old = atomicAdd(row_cnt + row, 1);
+        row_done = (old == (int)(c_hi - c_lo));
+        if (row_done) {
+          row_cnt[row] = 0;
+          __threadfence();
+          const float4* pp = reinterpret_cast<const float4*>(parts);
+          float4 q = __ldcg(pp + (size_t)row + (size_t)c_lo);
+          r = RedState{q.x, q.y, __float_as_int(q.z)};
+          for (long long k = c_lo + 1; k <= c_hi; ++k) {
+            q = __ldcg(pp + (size_t)row + (size_t)k);
+            r = red_combine(r, RedState{q.x, q.y, __float_as_int(q.z)}, c);
+          }
         }
       }
-    }
-    int last_of_seq = 0;
-    if (row_done) {
-      const float conf = 1.0f / r.s;
-      conf_ws[row] = conf;
-      arg_ws[row] = r.idx;
-      if (p.conf_out) p.conf_out[row] = conf;
-      if (p.argmax_out) p.argmax_out[row] = r.idx;
-      __threadfence();
-      const int b = row / p.block_size;
-      const int old = atomicAdd(seq_cnt + b, 1);
-      if (old == p.block_size - 1) {
-        seq_cnt[b] = 0;
+      int last_of_seq = 0;
+      if (row_done) {
+        const float conf = 1.0f / r.s;
+        conf_ws[row] = conf;
+        arg_ws[row] = r.idx;
+        if (p.conf_out) p.conf_out[row] = conf;
+        if (p.argmax_out) p.argmax_out[row] = r.idx;
         __threadfence();
-        last_of_seq = 1;
+        const int b = row / p.block_size;
+        const int old = atomicAdd(seq_cnt + b, 1);
+        if (old == p.block_size - 1) {
+          seq_cnt[b] = 0;
+          __threadfence();
+          last_of_seq = 1;
+        }
       }
+      s_flag = last_of_seq;
     }
-    s_flag = last_of_seq;
+    __syncthreads();
+    if (s_flag) commit_sequence(p, row / p.block_size, conf_ws, arg_ws);
+    seg = seg_end;
   }
-  __syncthreads();
-  if (s_flag) commit_sequence(p, row / p.block_size, conf_ws, arg_ws);
 }
 
-static UnmaskLayout layout_for(int rows, int batch, int chunks) {
+static UnmaskLayout layout_for(int rows, int batch, int grid) {
   UnmaskLayout L{};
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
@@ -267,7 +286,7 @@ static UnmaskLayout layout_for(int rows, int batch, int chunks) {
   };
   L.row_cnt = take(sizeof(int) * (size_t)rows);
   L.seq_cnt = take(sizeof(int) * (size_t)batch);
-  L.partials = take(sizeof(UnmaskPartial) * (size_t)rows * chunks);
+  L.partials = take(sizeof(UnmaskPartial) * ((size_t)rows + (size_t)grid));
   L.conf = take(sizeof(float) * (size_t)rows);
   L.argmax = take(sizeof(int32_t) * (size_t)rows);
   L.total = off;
@@ -278,29 +297,22 @@ UnmaskPlan unmask_plan(const tt_unmask_args_t* a, int num_sms) {
   UnmaskPlan pl{};
   const int rows = a->batch * a->block_size;
   const int W = (a->dtype == TT_BF16) ? 8 : 4;
-  const int target = 4 * std::max(num_sms, 1);
-  int chunks = (target + rows - 1) / rows;
-  const int max_chunks = std::max(1, a->vocab / 4096);
-  chunks = std::max(1, std::min(chunks, max_chunks));
-  // chunk length: a multiple of one CTA sweep (threads x vector width) where possible
-  const int sweep = kUnmaskThreads * W;
-  int chunk_elems = (a->vocab + chunks - 1) / chunks;
-  chunk_elems = ((chunk_elems + sweep - 1) / sweep) * sweep;
-  if (chunk_elems > a->vocab) chunk_elems = ((a->vocab + W - 1) / W) * W;
-  chunks = (a->vocab + chunk_elems - 1) / chunk_elems;
-  pl.chunks = chunks;
-  pl.chunk_elems = chunk_elems;
-  pl.layout = layout_for(rows, a->batch, chunks);
+  const long long E = (long long)rows * (a->vocab / W);
+  const long long P = (long long)std::max(num_sms, 1) * kUnmaskCtasPerSm;
+  pl.grid = (int)std::min(P, E);
+  pl.layout = layout_for(rows, a->batch, pl.grid);
   return pl;
 }
 
 int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cudaStream_t stream) {
   UnmaskParams p{};
+  const int W = (a->dtype == TT_BF16) ? 8 : 4;
   p.logits = a->logits;
   p.vocab = a->vocab;
-  p.chunk_elems = pl.chunk_elems;
-  p.chunks = pl.chunks;
+  p.vec_per_row = a->vocab / W;
   p.rows = a->batch * a->block_size;
+  p.total_vec = (long long)p.rows * p.vec_per_row;
+  p.p_eff = pl.grid;
   p.block_size = a->block_size;
   p.c = a->inv_temperature * 1.4426950408889634f;
   p.gamma = a->gamma;
@@ -319,11 +331,10 @@ int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cud
   p.off_partials = pl.layout.partials;
   p.off_conf = pl.layout.conf;
   p.off_argmax = pl.layout.argmax;
-  const unsigned grid = (unsigned)p.rows * (unsigned)pl.chunks;
   if (a->dtype == TT_BF16)
-    unmask_kernel<__nv_bfloat16><<<grid, kUnmaskThreads, 0, stream>>>(p);
+    unmask_kernel<__nv_bfloat16><<<pl.grid, kUnmaskThreads, 0, stream>>>(p);
   else
-    unmask_kernel<float><<<grid, kUnmaskThreads, 0, stream>>>(p);
+    unmask_kernel<float><<<pl.grid, kUnmaskThreads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }
 

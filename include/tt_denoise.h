@@ -90,7 +90,7 @@ typedef struct {
   int32_t num_kv_heads;      /* Hkv >= 1 */
   int32_t head_dim;          /* d */
   int32_t dtype;             /* tt_dtype_t */
-  float softmax_scale;       /* multiplies Q.K (1.0 when Q is pre-scaled) */
+  float softmax_scale;       /* > 0, multiplies Q.K (1.0 when Q is pre-scaled) */
   const void* q;
   const void* k_blk;
   const void* v_blk;
@@ -109,8 +109,9 @@ typedef struct {
 /* Bytes of workspace tt_denoise_attn needs for these arguments (0 if the args are invalid). */
 size_t tt_denoise_attn_workspace_bytes(const tt_attn_args_t* args);
 
-/* Launch Eq. (1). `workspace` (device, zero-filled once) holds the split-KV partial results,
- * the merge tickets and the device error word. */
+/* Launch Eq. (1): the attention kernel and, stream-ordered behind it, the kernel that merges the
+ * split-KV partial results. `workspace` (device) holds the partition of the tiles, the partial
+ * results and the device error word. */
 int tt_denoise_attn(const tt_attn_args_t* args, void* workspace, size_t workspace_bytes,
                     tt_stream_t stream);
 
@@ -123,7 +124,8 @@ int tt_denoise_attn(const tt_attn_args_t* args, void* workspace, size_t workspac
  *   phi(tau) = [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)), k < F/2
  *   mod[b] = W3 SiLU(W2 SiLU(W1 phi(tau_b) + b1) + b2) + b3, viewed as [3][D], + layer_emb
  *   tau [B] float; w1 [W][F], b1 [W], w2 [W][W], b2 [W], w3 [3D][W], b3 [3D], layer_emb [3][D]
- *   (all float); mod [B][3][D] float (rows: shift, scale, gate). F even, 2..1024; W 1..1024.
+ *   (all float); mod [B][3][D] float (rows: shift, scale, gate). F and W multiples of 4 up to
+ *   1024; w1, w2, w3 16-byte aligned.
  *   Needs workspace of tt_adaln_workspace_bytes() bytes (the MLP's hidden activations).
  * op TT_ADALN_NORM_MODULATE (h, norm_w, mod -> out):
  *   out[b][s] = h[b][s] / sqrt(mean(h[b][s]^2) + eps) * norm_w * (1 + scale[b]) + shift[b]

@@ -137,6 +137,9 @@ def _adaln_args(**kw):
     (dict(freq_dim=255), B.TT_ERR_INVALID_ARGUMENT),
     (dict(w3=None), B.TT_ERR_INVALID_ARGUMENT),
     (dict(mlp_width=2048), B.TT_ERR_UNSUPPORTED),
+    (dict(freq_dim=258), B.TT_ERR_UNSUPPORTED),
+    (dict(mlp_width=102), B.TT_ERR_UNSUPPORTED),
+    (dict(w2=4100), B.TT_ERR_UNSUPPORTED),
     (dict(op=B.TT_ADALN_NORM_MODULATE, norm_w=None), B.TT_ERR_INVALID_ARGUMENT),
     (dict(op=B.TT_ADALN_NORM_MODULATE, hidden=6), B.TT_ERR_UNSUPPORTED),
     (dict(op=B.TT_ADALN_GATED_RESIDUAL, f=None), B.TT_ERR_INVALID_ARGUMENT),
@@ -149,5 +152,5 @@ def test_adaln_host_validation(lib, kw, status):
 
 def test_adaln_workspace(lib):
     a = _adaln_args(batch=8, mlp_width=256)
-    assert lib.tt_adaln_workspace_bytes(ctypes.byref(a)) == 256 + 4 * 8 * 256
+    assert lib.tt_adaln_workspace_bytes(ctypes.byref(a)) == 256 + 2 * 4 * 8 * 256
     assert lib.tt_adaln_modulate(ctypes.byref(a), 4096, 100, None) == B.TT_ERR_WORKSPACE_TOO_SMALL
