@@ -34,20 +34,21 @@ __device__ __forceinline__ float warp_sum(float v) {
 constexpr int kGemvBatchChunk = 8;
 constexpr int kGemvMaxIn = 1024;
 
+// phi(tau) = [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)). The angle (up to
+// 1000 rad) is formed and reduced modulo 2 pi in double, so the single-precision sincos only sees
+// |angle| <= pi.
 __device__ __forceinline__ void phi_row(float tau, int F, float* dst, int tid, int nthreads) {
-  // [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)); the angle is reduced
-  // modulo 2 pi in double so that sincos always takes its small-argument path
   const int half = F / 2;
   const double t = 1000.0 * (double)tau;
   const double two_pi = 6.283185307179586476925286766559;
   for (int k = tid; k < half; k += nthreads) {
     const double w = exp(-9.2103403719761836 * (double)k / (double)half);   // ln(10000) = 9.2103...
     double a = t * w;
-    a -= two_pi * rint(a / two_pi);
-    double sv, cv;
-    sincos(a, &sv, &cv);
-    dst[k] = (float)cv;
-    dst[half + k] = (float)sv;
+    a -= two_pi * rint(a * (1.0 / two_pi));
+    float sv, cv;
+    sincosf((float)a, &sv, &cv);
+    dst[k] = cv;
+    dst[half + k] = sv;
   }
 }
 
@@ -58,6 +59,8 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_gemv_kernel(const float* 
                                                                    const float* __restrict__ x, int B, int IN,
                                                                    int OUT, float* __restrict__ y) {
   __shared__ __align__(16) float s_x[kGemvBatchChunk * kGemvMaxIn];
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int o0 = (blockIdx.x * (kAdalnThreads / 32) + warp) * R;
   float4 w[R][KW];
@@ -111,18 +114,28 @@ static void launch_gemv(const float* Wt, const float* bias, const float* extra, 
                         float* y, cudaStream_t stream) {
   const int kw = (IN + 127) / 128;   // float4 per lane per row
   const int warps = kAdalnThreads / 32;
+  // small layers: one row per warp (more CTAs); wide ones: four rows per warp
+  const bool wide = OUT > 2048;
   if (kw <= 1) {
-    adaln_gemv_kernel<1, 4, kPhi, kSilu><<<(OUT + warps * 4 - 1) / (warps * 4), kAdalnThreads, 0, stream>>>(
-        Wt, bias, extra, x, B, IN, OUT, y);
+    if (wide)
+      launch_pdl(adaln_gemv_kernel<1, 4, kPhi, kSilu>, dim3((OUT + warps * 4 - 1) / (warps * 4)), dim3(kAdalnThreads),
+                 0, stream, Wt, bias, extra, x, B, IN, OUT, y);
+    else
+      launch_pdl(adaln_gemv_kernel<1, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0,
+                 stream, Wt, bias, extra, x, B, IN, OUT, y);
   } else if (kw <= 2) {
-    adaln_gemv_kernel<2, 4, kPhi, kSilu><<<(OUT + warps * 4 - 1) / (warps * 4), kAdalnThreads, 0, stream>>>(
-        Wt, bias, extra, x, B, IN, OUT, y);
+    if (wide)
+      launch_pdl(adaln_gemv_kernel<2, 4, kPhi, kSilu>, dim3((OUT + warps * 4 - 1) / (warps * 4)), dim3(kAdalnThreads),
+                 0, stream, Wt, bias, extra, x, B, IN, OUT, y);
+    else
+      launch_pdl(adaln_gemv_kernel<2, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0,
+                 stream, Wt, bias, extra, x, B, IN, OUT, y);
   } else if (kw <= 4) {
-    adaln_gemv_kernel<4, 2, kPhi, kSilu><<<(OUT + warps * 2 - 1) / (warps * 2), kAdalnThreads, 0, stream>>>(
-        Wt, bias, extra, x, B, IN, OUT, y);
+    launch_pdl(adaln_gemv_kernel<4, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0, stream,
+               Wt, bias, extra, x, B, IN, OUT, y);
   } else {
-    adaln_gemv_kernel<8, 1, kPhi, kSilu><<<(OUT + warps - 1) / warps, kAdalnThreads, 0, stream>>>(
-        Wt, bias, extra, x, B, IN, OUT, y);
+    launch_pdl(adaln_gemv_kernel<8, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0, stream,
+               Wt, bias, extra, x, B, IN, OUT, y);
   }
 }
 
@@ -169,6 +182,8 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_norm_modulate_kernel(cons
                                                                             int S, int D, float eps,
                                                                             void* __restrict__ out) {
   constexpr int N = Io<T>::kN;
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x;
   const int b = row / S;
   const int nv = D / N;
@@ -210,6 +225,8 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_gated_residual_kernel(con
                                                                              int S, int D, size_t nvec,
                                                                              void* out) {
   constexpr int N = Io<T>::kN;
+  pdl_trigger();
+  pdl_wait();
   const int nv_row = D / N;
   for (size_t v = blockIdx.x * (size_t)blockDim.x + threadIdx.x; v < nvec; v += (size_t)gridDim.x * blockDim.x) {
     const size_t row = v / nv_row;
@@ -242,11 +259,11 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
   } else if (a->op == TT_ADALN_NORM_MODULATE) {
     const int rows = B * a->block_size;
     if (a->dtype == TT_BF16)
-      adaln_norm_modulate_kernel<__nv_bfloat16><<<rows, kAdalnThreads, 0, stream>>>(
-          a->h, a->norm_w, a->mod, a->block_size, D, a->eps, a->out);
+      launch_pdl(adaln_norm_modulate_kernel<__nv_bfloat16>, dim3(rows), dim3(kAdalnThreads), 0, stream, a->h,
+                 a->norm_w, (const float*)a->mod, a->block_size, D, a->eps, a->out);
     else
-      adaln_norm_modulate_kernel<float><<<rows, kAdalnThreads, 0, stream>>>(a->h, a->norm_w, a->mod,
-                                                                            a->block_size, D, a->eps, a->out);
+      launch_pdl(adaln_norm_modulate_kernel<float>, dim3(rows), dim3(kAdalnThreads), 0, stream, a->h, a->norm_w,
+                 (const float*)a->mod, a->block_size, D, a->eps, a->out);
   } else {
     const int N = (a->dtype == TT_BF16) ? 8 : 4;
     const size_t nvec = (size_t)B * a->block_size * D / N;
@@ -255,11 +272,11 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
     grid = grid < (size_t)sms * 8 ? grid : (size_t)sms * 8;
     if (grid == 0) grid = 1;
     if (a->dtype == TT_BF16)
-      adaln_gated_residual_kernel<__nv_bfloat16><<<(unsigned)grid, kAdalnThreads, 0, stream>>>(
-          a->h, a->f, a->mod, a->block_size, D, nvec, a->out);
+      launch_pdl(adaln_gated_residual_kernel<__nv_bfloat16>, dim3((unsigned)grid), dim3(kAdalnThreads), 0, stream,
+                 a->h, a->f, (const float*)a->mod, a->block_size, D, nvec, a->out);
     else
-      adaln_gated_residual_kernel<float><<<(unsigned)grid, kAdalnThreads, 0, stream>>>(
-          a->h, a->f, a->mod, a->block_size, D, nvec, a->out);
+      launch_pdl(adaln_gated_residual_kernel<float>, dim3((unsigned)grid), dim3(kAdalnThreads), 0, stream, a->h,
+                 a->f, (const float*)a->mod, a->block_size, D, nvec, a->out);
   }
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }

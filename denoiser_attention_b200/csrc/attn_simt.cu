@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(const SimtParam
   float* s_k = s_q + kSimtRows * D;                    // [32][DP]
   float* s_v = s_k + kSimtKeys * DP;                   // [32][DP]
   __shared__ int s_row[kSimtKeys];                     // source row of each tile key (-1: none)
+  pdl_trigger();
+  pdl_wait();
 
   const int b = blockIdx.z, kvh = blockIdx.y;
   const int row0 = blockIdx.x * kSimtRows;
@@ -214,9 +216,9 @@ int attn_simt_launch(const tt_attn_args_t* a, const AttnPlan& /*plan*/, void* ws
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
   if (p.d == 64)
-    attn_simt_kernel<64><<<grid, kSimtThreads, smem64, stream>>>(p);
+    launch_pdl(attn_simt_kernel<64>, grid, dim3(kSimtThreads), smem64, stream, p);
   else
-    attn_simt_kernel<128><<<grid, kSimtThreads, smem128, stream>>>(p);
+    launch_pdl(attn_simt_kernel<128>, grid, dim3(kSimtThreads), smem128, stream, p);
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }
 

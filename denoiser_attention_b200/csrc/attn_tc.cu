@@ -1,31 +1,36 @@
 // Eq. (1) of "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Context"
 // (§2.1 "Bidirectional attention") for bf16 tensors on the sm_100a tensor cores.
 //
-// Work decomposition. A "unit" is (sequence b, kv head, query-row tile). Its query rows are the
-// G query heads of the kv head times the block positions of the tile, packed as M rows
-// m = s * G + g (at most 256 = two 128-row MMA halves), so each key/value tile is read from HBM
-// once per unit. Its keys are ceil(L_b/64) context tiles of 64 tokens followed by one tile holding
-// the S block tokens. All units' tiles are laid end to end and cut into Pe = min(gridDim.x, tiles)
-// equal ranges, one per persistent CTA (one CTA per SM), so ragged contexts are balanced to within
-// a tile without any host-side knowledge of the lengths. A CTA that holds a whole unit writes its
-// output directly; a unit cut between CTAs leaves one normalised partial (O_j / l_j and the
-// log2-sum-exp) per CTA, and a second, wide kernel merges them (flash-decoding combine). The
-// merge kernel is launched as a programmatic dependent of the attention kernel, so its launch
-// overlaps the attention tail and it starts reading partials as soon as they are complete.
+// Work decomposition. A "group" is (sequence b, kv head): its keys are ceil(L_b/128) context
+// tiles of 128 tokens followed by one tile holding the S block tokens. Its query rows are the
+// G query heads of the kv head times the S block positions, packed as rows m = s * G + g and cut
+// into "query tiles" of at most 128 rows (one tcgen05 M=128 MMA). nq = number of query tiles per
+// group. The CTAs are organised in teams of nq; all groups' key tiles are laid end to end and cut
+// into Pe = min(teams, tiles) equal ranges, one per team, computed on the device from ctx_lens
+// (ragged contexts balance to within a tile, with no host knowledge of the lengths). Within a
+// team, CTA q handles query tile q of every group its range touches, and the team's CTAs walk the
+// same key tiles at the same time, so each K/V tile comes from HBM once and the other reads of it
+// hit L2. A CTA that holds a whole group writes its rows of the output directly; a group cut
+// between teams leaves a normalised partial (O_j / l_j and the log2-sum-exp) per CTA, and a second,
+// wide kernel merges them (flash-decoding combine), launched as a programmatic dependent.
 //
-// Inside a CTA (384 threads):
-//   warp 0      TMA producer: Q tile of the unit, then K/V tiles into a 4-stage ring
-//               (128B-swizzled boxes of 64 tokens x 64 dims; no multicast)
-//   warp 1      MMA issuer (one thread): S_h = Q_h K^T (M=128, N=64, K=128) into TMEM, then
-//               O_h += P_h V (M=128, N=128, K=64) with P read from TMEM; QK^T of tile f+1 is
-//               issued before PV of tile f so the tensor pipe works while the softmax runs
-//   warps 4-7   softmax + epilogue for rows 0..127 (thread = TMEM lane = row)
-//   warps 8-11  softmax + epilogue for rows 128..255
-// TMEM (512 columns): O_0 [0,128), O_1 [128,256), S/P double buffers of 64 columns per half.
-// The softmax works in the exp2 domain with the scale folded in; the running maximum used for
-// the exponentials is only raised when a tile's maximum exceeds it by more than 8 (a factor 256),
-// which keeps the O rescale off the common path and stays exact because numerator and
-// denominator use the same stale maximum. Only a rescale waits for the previous PV product.
+// Inside a CTA (320 threads):
+//   warp 0     TMA producer: the Q tile of the group, then K and V tiles of 128 tokens into a
+//              2-stage ring with separate K and V barriers (128B-swizzled boxes; no multicast)
+//   warp 1     MMA issuer (one thread): S[f%2] = Q K^T (M=128, N=128, K=128, both operands from
+//              shared memory) for tile f+1 is issued before O += P V for tile f (A = P from TMEM,
+//              B = V), so the tensor pipe computes the next scores while the softmax runs
+//   warps 2-9  softmax + epilogue: a thread owns query row = its TMEM lane (lane quadrant =
+//              warp % 4) and one half of the 128 key columns (warps 2-5 keys 0-63, warps 6-9
+//              keys 64-127); the two threads of a row exchange their partial maxima and sums
+//              through shared memory (bounded mbarrier handshakes)
+// TMEM (512 columns allocated): O [0,128), S/P double buffer [128,256), [256,384); each thread
+// writes its 64 P values (bf16) over the first 32 columns of its own S columns, and the PV
+// product reads P from TMEM.
+// The softmax works in the exp2 domain with the scale folded in and computes P against the
+// running maximum; only when a tile's maximum exceeds it by more than 8 (P > 256) is the tile
+// redone against the new maximum and O rescaled (exact: numerator and denominator share the
+// stale maximum).
 #include <cstdio>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -38,24 +43,23 @@ namespace tt {
 namespace {
 
 constexpr int kD = 128;           // head dim handled by this kernel
-constexpr int kTile = 64;         // keys per tile
-constexpr int kStages = 4;        // K/V ring depth
-constexpr int kThreads = 384;
-constexpr int kRowsPerHalf = 128;
+constexpr int kTile = 128;        // keys per tile
+constexpr int kStages = 2;        // K/V ring depth
+constexpr int kRows = 128;        // query rows per CTA (one M=128 MMA)
+constexpr int kThreads = 320;     // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kQBytesPerDh = 256 * 128;                   // 256 rows x 128 B
-constexpr uint32_t kQBytes = 2 * kQBytesPerDh;                 // 64 KB
-constexpr uint32_t kKVBoxBytes = kTile * 128;                  // 64 rows x 128 B = 8 KB
-constexpr uint32_t kKBytesPerStage = 2 * kKVBoxBytes;          // 16 KB
-constexpr uint32_t kStageBytes = 2 * kKBytesPerStage;          // K + V = 32 KB
+constexpr uint32_t kQBytesPerDh = kRows * 128;                 // 128 rows x 128 B = 16 KB
+constexpr uint32_t kQBytes = 2 * kQBytesPerDh;                 // 32 KB
+constexpr uint32_t kKVBoxBytes = kTile * 128;                  // 128 rows x 128 B = 16 KB
+constexpr uint32_t kKBytesPerStage = 2 * kKVBoxBytes;          // 32 KB (two 64-dim boxes)
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kQBytes;
 constexpr uint32_t kSmemV = kSmemK + kStages * kKBytesPerStage;
 constexpr uint32_t kSmemBar = kSmemV + kStages * kKBytesPerStage;
-constexpr uint32_t kSmemBytes = kSmemBar + 1024 + 1024;        // barriers/scratch + alignment slack
+constexpr uint32_t kSmemBytes = kSmemBar + 4096 + 1024;        // barriers/scratch + alignment slack
 
-constexpr int kMergeRows = 32;    // rows per merge CTA (8 warps x 4 rows)
+constexpr int kMergeRows = 8;     // rows per merge CTA (one per warp)
 
 // Instruction descriptors (kind::f16): D fp32, A/B bf16, A K-major.
 constexpr uint32_t make_idesc(int M, int N, bool b_mn_major) {
@@ -76,13 +80,10 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-// Workspace: header | meta (total tiles, working CTAs) | unit_start[units + 1] | partials | lse
+// Workspace: header | meta | group_start[groups + 1] | partials | lse
 struct AttnMeta {
   long long total_tiles;
-  long long p_eff;
+  long long p_eff;   // working teams
 };
 
 struct TcParams {
@@ -90,7 +91,7 @@ struct TcParams {
   const int32_t* ctx_lens;
   const int32_t* page_table;
   int32_t B, S, Hq, Hkv, G;
-  int32_t qtiles, s_per_tile, units;
+  int32_t nq, s_per_tile, groups, teams;
   int32_t page_size, max_pages, num_pages, ctx_stride, paged;
   float scale_log2;   // softmax_scale * log2(e)
   __nv_bfloat16* out;
@@ -101,9 +102,12 @@ struct TcParams {
 
 struct Smem {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2], pv_done;
+  uint64_t x_bar, l_bar;   // row-max and row-sum exchange between the two column halves
   uint64_t drain;
+  float xmax[2][2][kRows];  // [tile parity][column half][row]
+  float xsum[2][kRows];
   uint32_t tmem_base;
   int abort_flag;
   long long range_begin, range_end, total_tiles, p_eff;
@@ -111,18 +115,17 @@ struct Smem {
   long long u0_start;
 };
 
-struct UnitInfo {
-  int b, kvh, qt, L, nctx, ntiles;
+struct GroupInfo {
+  int b, kvh, L, nctx, ntiles;
 };
 
-__device__ __forceinline__ int clamp_len(const int32_t* ctx_lens, int paged, int max_pages, int page_size,
-                                         int ctx_stride, int b, bool report, WsHeader* hdr) {
-  int L = ctx_lens[b];
+__device__ __forceinline__ int clamp_len(const TcParams& p, int b, bool report, WsHeader* hdr) {
+  int L = p.ctx_lens[b];
   if (L < 0) {
     if (report) report_error(hdr, TT_ERR_DEVICE, kDetailNegativeLen);
     L = 0;
   }
-  const int cap = paged ? max_pages * page_size : ctx_stride;
+  const int cap = p.paged ? p.max_pages * p.page_size : p.ctx_stride;
   if (L > cap) {
     if (report) report_error(hdr, TT_ERR_DEVICE, kDetailCtxTooLong);
     L = cap;
@@ -130,53 +133,51 @@ __device__ __forceinline__ int clamp_len(const int32_t* ctx_lens, int paged, int
   return L;
 }
 
-__device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int u, bool report, WsHeader* hdr) {
-  UnitInfo ui;
-  ui.qt = u % p.qtiles;
-  const int bk = u / p.qtiles;
-  ui.kvh = bk % p.Hkv;
-  ui.b = bk / p.Hkv;
-  ui.L = clamp_len(p.ctx_lens, p.paged, p.max_pages, p.page_size, p.ctx_stride, ui.b, report, hdr);
-  ui.nctx = (ui.L + kTile - 1) / kTile;
-  ui.ntiles = ui.nctx + 1;
-  return ui;
+__device__ __forceinline__ GroupInfo group_info(const TcParams& p, int g, bool report, WsHeader* hdr) {
+  GroupInfo gi;
+  gi.kvh = g % p.Hkv;
+  gi.b = g / p.Hkv;
+  gi.L = clamp_len(p, gi.b, report, hdr);
+  gi.nctx = (gi.L + kTile - 1) / kTile;
+  gi.ntiles = gi.nctx + 1;
+  return gi;
 }
 
-// Walks the units overlapping this CTA's tile range, one segment (a maximal run of tiles of one
-// unit) at a time. Every role runs its own copy; all copies see the same sequence.
+// Walks the groups overlapping this team's tile range, one segment (a maximal run of tiles of one
+// group) at a time. Every role runs its own copy; all copies see the same sequence.
 struct SegWalk {
   int u;
   long long ustart;
   long long g, gend;
-  UnitInfo ui;
+  GroupInfo gi;
   __device__ void init(const TcParams& p, const Smem& sm, WsHeader* hdr) {
     u = sm.u0;
     ustart = sm.u0_start;
     g = sm.range_begin;
     gend = sm.range_end;
-    ui = unit_info(p, u, false, hdr);
+    gi = group_info(p, u, false, hdr);
   }
   __device__ bool done() const { return g >= gend; }
-  // tiles [kb, ke) of unit ui in the current segment
+  // tiles [kb, ke) of group gi in the current segment
   __device__ void segment(int& kb, int& ke) const {
     kb = (int)(g - ustart);
-    const long long uend = ustart + ui.ntiles;
+    const long long uend = ustart + gi.ntiles;
     ke = (int)((uend < gend ? uend : gend) - ustart);
   }
   __device__ void advance(const TcParams& p, WsHeader* hdr) {
     int kb, ke;
     segment(kb, ke);
     g = ustart + ke;
-    if (ke == ui.ntiles && g < gend) {
-      ustart += ui.ntiles;
+    if (ke == gi.ntiles && g < gend) {
+      ustart += gi.ntiles;
       ++u;
-      ui = unit_info(p, u, false, hdr);
+      gi = group_info(p, u, false, hdr);
     }
   }
 };
 
-// CTA index owning global tile t when T tiles are cut into P <= T ranges [c*T/P, (c+1)*T/P).
-__device__ __forceinline__ long long owner_cta(long long t, long long T, long long P) {
+// Team owning global tile t when T tiles are cut into P <= T ranges [c*T/P, (c+1)*T/P).
+__device__ __forceinline__ long long owner_team(long long t, long long T, long long P) {
   return ((t + 1) * P - 1) / T;
 }
 
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   Smem& sm = *reinterpret_cast<Smem*>(smem + kSmemBar);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long P = gridDim.x, cta = blockIdx.x;
+  const int team = blockIdx.x / p.nq, qt = blockIdx.x % p.nq;
 
   // ---- 0. prologue that touches no input: barriers, TMEM, tensor-map prefetch. With a
   // programmatic launch it overlaps the previous kernel; inputs are read after pdl_wait().
@@ -194,16 +195,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm.kv_full[i], 1);
-      mbar_init(&sm.kv_empty[i], 1);
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
+      mbar_init(&sm.v_full[i], 1);
+      mbar_init(&sm.v_empty[i], 1);
     }
-    for (int h = 0; h < 2; ++h) {
-      for (int bf = 0; bf < 2; ++bf) {
-        mbar_init(&sm.s_full[h][bf], 1);
-        mbar_init(&sm.p_full[h][bf], kRowsPerHalf);
-        mbar_init(&sm.pv_done[h][bf], 1);
-      }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.p_full[b], 2 * kRows);
     }
+    mbar_init(&sm.pv_done, 1);
+    mbar_init(&sm.x_bar, 2 * kRows);
+    mbar_init(&sm.l_bar, 2 * kRows);
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
     prefetch_tmap(&p.tm_q);
@@ -220,30 +223,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   pdl_trigger();
   pdl_wait();
 
-  // ---- 1. this CTA's tile range and the unit where it starts (warp 0); CTA 0 also records the
-  // partition for the merge kernel
+  // ---- 1. this team's tile range and the group where it starts (warp 0); CTA 0 also records
+  // the partition for the merge kernel
   if (warp == 0) {
     long long T = 0;
-    for (int base = 0; base < p.units; base += 32) {
+    for (int base = 0; base < p.groups; base += 32) {
       const int u = base + lane;
       int n = 0;
-      if (u < p.units) n = unit_info(p, u, blockIdx.x == 0, hdr).ntiles;
+      if (u < p.groups) n = group_info(p, u, blockIdx.x == 0, hdr).ntiles;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
       T += n;
     }
-    // with fewer tiles than CTAs only the first T CTAs work (one tile each), so every working
-    // CTA owns a non-empty range and the CTAs of a unit are consecutive
-    const long long Pe = T < P ? T : P;
-    const long long rb = cta < Pe ? cta * T / Pe : T, re = cta < Pe ? (cta + 1) * T / Pe : T;
+    // with fewer tiles than teams only the first T teams work (one tile each), so every working
+    // team owns a non-empty range and the teams of a group are consecutive
+    const long long Pe = T < p.teams ? T : p.teams;
+    const long long rb = team < Pe ? team * T / Pe : T, re = team < Pe ? (team + 1) * T / Pe : T;
     long long acc = 0;
     int u0 = -1;
     long long u0s = 0;
     int32_t* ustart_out = reinterpret_cast<int32_t*>(p.ws + p.off_ustart);
     const bool record = (blockIdx.x == 0);
-    for (int base = 0; base < p.units && (u0 < 0 || record); base += 32) {
+    for (int base = 0; base < p.groups && (u0 < 0 || record); base += 32) {
       const int u = base + lane;
-      const int n = (u < p.units) ? unit_info(p, u, false, hdr).ntiles : 0;
+      const int n = (u < p.groups) ? group_info(p, u, false, hdr).ntiles : 0;
       int incl = n;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -251,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (lane >= o) incl += y;
       }
       const long long lo = acc + incl - n, hi = acc + incl;
-      if (record && u < p.units) ustart_out[u] = (int32_t)lo;
-      const unsigned hit = __ballot_sync(0xffffffffu, u < p.units && lo <= rb && rb < hi);
+      if (record && u < p.groups) ustart_out[u] = (int32_t)lo;
+      const unsigned hit = __ballot_sync(0xffffffffu, u < p.groups && lo <= rb && rb < hi);
       if (hit && u0 < 0) {
         const int src = __ffs(hit) - 1;
         u0 = base + src;
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       sm.u0_start = u0s;
       sm.abort_flag = 0;
       if (record) {
-        ustart_out[p.units] = (int32_t)T;
+        ustart_out[p.groups] = (int32_t)T;
         AttnMeta* meta = reinterpret_cast<AttnMeta*>(p.ws + p.off_meta);
         meta->total_tiles = T;
         meta->p_eff = Pe;
@@ -280,10 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
-  const bool has_work = sm.range_begin < sm.range_end && sm.u0 >= 0;
-
-  const int M = p.G * p.s_per_tile;               // query rows per unit (<= 256)
-  const int nh = (M > kRowsPerHalf) ? 2 : 1;      // active 128-row halves
+  const bool has_work = team < p.teams && sm.range_begin < sm.range_end && sm.u0 >= 0;
 
   auto fail = [&](uint32_t detail) {
     report_error(hdr, TT_ERR_DEVICE_TIMEOUT, detail);
@@ -293,9 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const uint32_t sQ = smem_u32(smem + kSmemQ);
   const uint32_t sK = smem_u32(smem + kSmemK);
   const uint32_t sV = smem_u32(smem + kSmemV);
+  const int s_cnt = min(p.s_per_tile, p.S - qt * p.s_per_tile);   // block positions of this query tile
+  const int nrows = p.G * s_cnt;                                   // valid query rows (<= 128)
 
   if (!has_work) {
-    // nothing to do (more CTAs than tiles)
+    // nothing to do (more teams than tiles, or a CTA beyond the last full team)
   } else if (warp == 0) {
     // ======================= TMA producer
     if (lane == 0) {
@@ -308,54 +310,61 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       while (ok && !w.done()) {
         int kb, ke;
         w.segment(kb, ke);
-        const UnitInfo& ui = w.ui;
+        const GroupInfo& gi = w.gi;
         if (qn > 0 && !mbar_wait_bounded(&sm.q_empty, (qn - 1) & 1, abort_flag)) {
           fail(kDetailWaitQEmpty);
           ok = false;
           break;
         }
         mbar_arrive_expect_tx(&sm.q_full, q_bytes);
-        const int qrow = ui.b * p.S + ui.qt * p.s_per_tile;
-        tma_load_3d(smem + kSmemQ, &p.tm_q, &sm.q_full, 0, ui.kvh * p.G, qrow);
-        tma_load_3d(smem + kSmemQ + kQBytesPerDh, &p.tm_q, &sm.q_full, 64, ui.kvh * p.G, qrow);
+        const int qrow = gi.b * p.S + qt * p.s_per_tile;
+        tma_load_3d(smem + kSmemQ, &p.tm_q, &sm.q_full, 0, gi.kvh * p.G, qrow);
+        tma_load_3d(smem + kSmemQ + kQBytesPerDh, &p.tm_q, &sm.q_full, 64, gi.kvh * p.G, qrow);
         ++qn;
         for (int k = kb; k < ke; ++k, ++f) {
           const int stage = (int)(f % kStages);
-          const long long round = f / kStages;
-          if (round > 0 && !mbar_wait_bounded(&sm.kv_empty[stage], (uint32_t)((round - 1) & 1), abort_flag)) {
-            fail(kDetailWaitKvEmpty);
-            ok = false;
-            break;
-          }
+          const uint32_t round = (uint32_t)(f / kStages);
           const CUtensorMap* mk;
           const CUtensorMap* mv;
           int row;
-          if (k < ui.nctx) {
+          if (k < gi.nctx) {
             const int t0 = k * kTile;
             if (p.paged) {
-              int pg = p.page_table[(size_t)ui.b * p.max_pages + t0 / p.page_size];
+              int pg = p.page_table[(size_t)gi.b * p.max_pages + t0 / p.page_size];
               if (pg < 0 || pg >= p.num_pages) {
                 report_error(hdr, TT_ERR_DEVICE, kDetailBadPage);
                 pg = 0;   // read a valid page instead; the result is unspecified, the error is set
               }
               row = pg * p.page_size + t0 % p.page_size;
             } else {
-              row = ui.b * p.ctx_stride + t0;
+              row = gi.b * p.ctx_stride + t0;
             }
             mk = &p.tm_kc;
             mv = &p.tm_vc;
           } else {
-            row = ui.b * p.S;
+            row = gi.b * p.S;
             mk = &p.tm_kb;
             mv = &p.tm_vb;
           }
+          // K of a stage is free once its QK^T has run, V once its PV has run
+          if (round > 0 && !mbar_wait_bounded(&sm.k_empty[stage], (round - 1) & 1, abort_flag)) {
+            fail(kDetailWaitKvEmpty);
+            ok = false;
+            break;
+          }
           uint8_t* kdst = smem + kSmemK + stage * kKBytesPerStage;
+          mbar_arrive_expect_tx(&sm.k_full[stage], kKBytesPerStage);
+          tma_load_3d(kdst, mk, &sm.k_full[stage], 0, gi.kvh, row);
+          tma_load_3d(kdst + kKVBoxBytes, mk, &sm.k_full[stage], 64, gi.kvh, row);
+          if (round > 0 && !mbar_wait_bounded(&sm.v_empty[stage], (round - 1) & 1, abort_flag)) {
+            fail(kDetailWaitKvEmpty);
+            ok = false;
+            break;
+          }
           uint8_t* vdst = smem + kSmemV + stage * kKBytesPerStage;
-          mbar_arrive_expect_tx(&sm.kv_full[stage], kStageBytes);
-          tma_load_3d(kdst, mk, &sm.kv_full[stage], 0, ui.kvh, row);
-          tma_load_3d(kdst + kKVBoxBytes, mk, &sm.kv_full[stage], 64, ui.kvh, row);
-          tma_load_3d(vdst, mv, &sm.kv_full[stage], 0, ui.kvh, row);
-          tma_load_3d(vdst + kKVBoxBytes, mv, &sm.kv_full[stage], 64, ui.kvh, row);
+          mbar_arrive_expect_tx(&sm.v_full[stage], kKBytesPerStage);
+          tma_load_3d(vdst, mv, &sm.v_full[stage], 0, gi.kvh, row);
+          tma_load_3d(vdst + kKVBoxBytes, mv, &sm.v_full[stage], 64, gi.kvh, row);
         }
         if (!ok) break;
         w.advance(p, hdr);
@@ -364,9 +373,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const long long nf = f;
       for (long long j = (nf > kStages ? nf - kStages : 0); j < nf; ++j) {
         const int stage = (int)(j % kStages);
+        const uint32_t par = (uint32_t)((j / kStages) & 1);
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&sm.kv_full[stage], (uint32_t)((j / kStages) & 1)) &&
-               globaltimer_ns() - t0 < kWaitLimitNs) {
+        while (!mbar_try_wait(&sm.k_full[stage], par) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+        while (!mbar_try_wait(&sm.v_full[stage], par) && globaltimer_ns() - t0 < kWaitLimitNs) {
         }
       }
       if (qn > 0) {
@@ -380,172 +391,213 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (lane == 0) {
       SegWalk w;
       w.init(p, sm, hdr);
+      // descriptor bases; per-MMA descriptors add constant offsets to the start-address field
+      // (bits 0..13, 16-byte units), which shared-memory addresses below 256 KB never carry out of
+      const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sV, kKVBoxBytes, 1024);
       long long f = 0;
       int seg = 0;
       bool ok = true;
       bool have_prev = false;
-      long long prev_f = 0;
       bool prev_first = false;
-      auto issue_pv = [&](long long pf, bool first) -> bool {
+      // O (+)= P V for tile pf; P is in TMEM over S[pf % 2]
+      auto pv = [&](long long pf, bool first) -> bool {
         const int stage = (int)(pf % kStages);
-        const int bf = (int)(pf & 1);
-        for (int h = 0; h < nh; ++h) {
-          if (!mbar_wait_bounded(&sm.p_full[h][bf], (uint32_t)((pf >> 1) & 1), abort_flag)) {
-            fail(kDetailWaitPFull);
-            return false;
-          }
-          tc_fence_after();
-          const uint32_t d_tm = tmem + (uint32_t)(kRowsPerHalf * h);
-          const uint32_t p_tm = tmem + 256u + (uint32_t)(128 * h + 64 * bf);
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t bdesc = sdesc_sw128(sV + stage * kKBytesPerStage + kk * 2048, kKVBoxBytes, 1024);
-            mma_ts(d_tm, p_tm + 8u * kk, bdesc, kIdescPV, (first && kk == 0) ? 0u : 1u);
-          }
-          tc_commit(&sm.pv_done[h][bf]);
+        if (!mbar_wait_bounded(&sm.v_full[stage], (uint32_t)((pf / kStages) & 1), abort_flag)) {
+          fail(kDetailWaitKvFull);
+          return false;
         }
-        tc_commit(&sm.kv_empty[stage]);
+        if (!mbar_wait_bounded(&sm.p_full[pf & 1], (uint32_t)((pf >> 1) & 1), abort_flag)) {
+          fail(kDetailWaitPFull);
+          return false;
+        }
+        tc_fence_after();
+        const uint32_t p_tm = tmem + 128u + 128u * (uint32_t)(pf & 1);
+        const uint64_t vd = dv0 + (uint64_t)((stage * kKBytesPerStage) >> 4);
+        // keys 0-63: P columns 0-31; keys 64-127: P columns 64-95 (one block per column half)
+        mma_ts(tmem, p_tm, vd, kIdescPV, first ? 0u : 1u);
+#pragma unroll
+        for (int kk = 1; kk < kTile / 16; ++kk)
+          mma_ts(tmem, p_tm + 8u * (kk & 3) + 64u * (kk >> 2), vd + (uint64_t)((kk * 2048) >> 4), kIdescPV, 1u);
+        tc_commit(&sm.pv_done);
+        tc_commit(&sm.v_empty[stage]);
         return true;
+      };
+      // S[ff % 2] = Q K^T for tile ff
+      auto qk = [&](long long ff) {
+        const int stage = (int)(ff % kStages);
+        const uint32_t d_tm = tmem + 128u + 128u * (uint32_t)(ff & 1);
+        const uint64_t kd = dk0 + (uint64_t)((stage * kKBytesPerStage) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off_q = ((kk >> 2) * kQBytesPerDh + (kk & 3) * 32) >> 4;
+          const uint32_t off_k = ((kk >> 2) * kKVBoxBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d_tm, dq0 + off_q, kd + off_k, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&sm.s_full[ff & 1]);
+        tc_commit(&sm.k_empty[stage]);
       };
       while (ok && !w.done()) {
         int kb, ke;
         w.segment(kb, ke);
-        if (!mbar_wait_bounded(&sm.q_full, (uint32_t)(seg & 1), abort_flag)) {
-          fail(kDetailWaitQFull);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         for (int k = kb; k < ke; ++k, ++f) {
           const int stage = (int)(f % kStages);
-          if (!mbar_wait_bounded(&sm.kv_full[stage], (uint32_t)((f / kStages) & 1), abort_flag)) {
+          if (k == kb && !mbar_wait_bounded(&sm.q_full, (uint32_t)(seg & 1), abort_flag)) {
+            fail(kDetailWaitQFull);
+            ok = false;
+            break;
+          }
+          if (!mbar_wait_bounded(&sm.k_full[stage], (uint32_t)((f / kStages) & 1), abort_flag)) {
             fail(kDetailWaitKvFull);
             ok = false;
             break;
           }
           tc_fence_after();
-          const int bf = (int)(f & 1);
-          for (int h = 0; h < nh; ++h) {
-            const uint32_t d_tm = tmem + 256u + (uint32_t)(128 * h + 64 * bf);
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t qa = sQ + (kk >> 2) * kQBytesPerDh + h * (kRowsPerHalf * 128) + (kk & 3) * 32;
-              const uint32_t ka = sK + stage * kKBytesPerStage + (kk >> 2) * kKVBoxBytes + (kk & 3) * 32;
-              mma_ss(d_tm, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(&sm.s_full[h][bf]);
-          }
+          // S[f % 2] was last read as P of tile f-2, whose PV was issued before this QK^T
+          qk(f);
           if (k == ke - 1) tc_commit(&sm.q_empty);
-          if (have_prev && !issue_pv(prev_f, prev_first)) {
+          if (have_prev && !pv(f - 1, prev_first)) {
             ok = false;
             break;
           }
           have_prev = true;
-          prev_f = f;
           prev_first = (k == kb);
         }
         if (!ok) break;
         ++seg;
         w.advance(p, hdr);
       }
-      if (ok && have_prev) issue_pv(prev_f, prev_first);
+      if (ok && have_prev) pv(f - 1, prev_first);
     }
-  } else if (warp >= 4 && (warp - 4) / 4 < nh) {
-    // ======================= softmax + epilogue, half h
-    const int h = (warp - 4) / 4;
-    const int t = tid - 128 - 128 * h;             // 0..127: TMEM lane and row within the half
-    const int row = kRowsPerHalf * h + t;          // row within the unit's tile
+  } else {
+    // ======================= softmax + epilogue (warps 2-9)
+    const int t = 32 * (warp & 3) + lane;   // TMEM lane quadrant warp % 4 -> query row t
+    const int ch = (warp - 2) >> 2;         // column half: keys [64 ch, 64 ch + 64)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_tm0 = tmem + lane_off + 256u + (uint32_t)(128 * h);
-    const uint32_t o_tm = tmem + lane_off + (uint32_t)(kRowsPerHalf * h);
+    const uint32_t o_tm = tmem + lane_off + 64u * (uint32_t)ch;   // this thread's 64 output dims
     const float sc = p.scale_log2;
     float* partials = reinterpret_cast<float*>(p.ws + p.off_partials);
     float* plse = reinterpret_cast<float*>(p.ws + p.off_lse);
     SegWalk w;
     w.init(p, sm, hdr);
     long long f = 0;
+    int nseg = 0;
     bool ok = true;
+    // partial row maximum of this thread's 64 raw scores -> exchanged maximum of the row (scaled)
+    auto exchange_max = [&](float mine, long long ff, float& row_max) -> bool {
+      sm.xmax[ff & 1][ch][t] = mine;
+      mbar_arrive(&sm.x_bar);
+      if (!mbar_wait_bounded(&sm.x_bar, (uint32_t)(ff & 1), abort_flag)) {
+        fail(kDetailWaitTicket);
+        return false;
+      }
+      row_max = fmaxf(mine, sm.xmax[ff & 1][ch ^ 1][t]);
+      return true;
+    };
     while (ok && !w.done()) {
       int kb, ke;
       w.segment(kb, ke);
-      const UnitInfo ui = w.ui;
+      const GroupInfo gi = w.gi;
       float m_used = -INFINITY, l = 0.f;
       for (int k = kb; k < ke; ++k, ++f) {
-        const int bf = (int)(f & 1);
-        const int valid = (k < ui.nctx) ? min(kTile, ui.L - k * kTile) : p.S;
-        if (!mbar_wait_bounded(&sm.s_full[h][bf], (uint32_t)((f >> 1) & 1), abort_flag)) {
+        const int valid = (k < gi.nctx) ? min(kTile, gi.L - k * kTile) : p.S;
+        const int lim = valid - 64 * ch;    // valid columns among this thread's 64
+        const uint32_t s_tm = tmem + lane_off + 128u + 128u * (uint32_t)(f & 1) + 64u * (uint32_t)ch;
+        if (!mbar_wait_bounded(&sm.s_full[f & 1], (uint32_t)((f >> 1) & 1), abort_flag)) {
           fail(kDetailWaitSFull);
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sr[64];
-        tmem_ld32(s_tm0 + 64u * bf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(s_tm0 + 64u * bf + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(s_tm, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(s_tm + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
-        // row maximum of the raw scores (the scale is positive, so it commutes with max)
-        float mt = -INFINITY;
-        if (valid >= kTile) {
+        // The row's tile maximum (both column halves, exchanged through shared memory) decides the
+        // exponent base: a segment's first tile uses it; later tiles keep the running maximum
+        // m_used unless the tile exceeds it by more than 8 (P would exceed 256), in which case the
+        // base moves to the tile maximum and O is rescaled. Then one pass writes
+        // P = 2^(s*scale - base) in bf16 over this thread's S columns and sums P in fp32.
+        const bool first = (k == kb);
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (lim >= 64) {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) mt = fmaxf(mt, __uint_as_float(sr[j]));
+          for (int j = 0; j < 64; ++j) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sr[j]));
         } else {
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            if (j >= valid) sr[j] = __float_as_uint(-INFINITY);
-            mt = fmaxf(mt, __uint_as_float(sr[j]));
+            if (j >= lim) sr[j] = __float_as_uint(-INFINITY);
+            mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sr[j]));
           }
         }
-        mt *= sc;
-        const bool first = (k == kb);
-        bool resc = false;
+        float rm;
+        if (!exchange_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), f, rm)) {
+          ok = false;
+          break;
+        }
+        const float mt = rm * sc;
         float m_new = m_used;
+        bool resc = false;
         if (first) {
           m_new = mt;
         } else if (mt > m_used + 8.0f) {
           m_new = mt;
           resc = true;
         }
-        const float factor = resc ? ex2(m_used - m_new) : 1.0f;
-        uint32_t pk[32];
-        float psum0 = 0.f, psum1 = 0.f;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[2 * j]), sc, -m_new));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[2 * j + 1]), sc, -m_new));
-          psum0 += p0;
-          psum1 += p1;
-          pk[j] = pack_bf16x2(p0, p1);
+        for (int q = 0; q < 2; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = 16 * q + jj;
+            const float p0 = ex2(fmaf(__uint_as_float(sr[2 * j]), sc, -m_new));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[2 * j + 1]), sc, -m_new));
+            ps[j & 3] += p0 + p1;
+            pk[jj] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(s_tm + 16u * q, pk);
         }
-        l = l * factor + (psum0 + psum1);
-        tmem_st32(s_tm0 + 64u * bf, pk);
-        if (resc) {
-          // O holds the sum up to tile f-1: wait for that PV product, then rescale it
-          const long long pf = f - 1;
-          if (!mbar_wait_bounded(&sm.pv_done[h][pf & 1], (uint32_t)((pf >> 1) & 1), abort_flag)) {
+        const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        const float factor = resc ? ex2(m_used - m_new) : 1.0f;
+        l = l * factor + psum;
+        tmem_wait_st();
+        if (!first) {
+          // O holds the sum up to tile f-1: its PV product must be complete before O is rescaled
+          // and before P of this tile is handed over (so the pv_done phases stay one step apart)
+          if (!mbar_wait_bounded(&sm.pv_done, (uint32_t)((f - 1) & 1), abort_flag)) {
             fail(kDetailWaitPvDone);
             ok = false;
             break;
           }
           tc_fence_after();
+          if (resc) {
 #pragma unroll 1
-          for (int cb = 0; cb < kD / 32; ++cb) {
-            uint32_t orr[32];
-            tmem_ld32(o_tm + 32u * cb, orr);
-            tmem_wait_ld();
+            for (int cb = 0; cb < 2; ++cb) {
+              uint32_t orr[32];
+              tmem_ld32(o_tm + 32u * cb, orr);
+              tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * factor);
-            tmem_st32(o_tm + 32u * cb, orr);
+              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * factor);
+              tmem_st32(o_tm + 32u * cb, orr);
+            }
+            tmem_wait_st();
           }
         }
-        tmem_wait_st();
-        if (h == 0 && k < ui.nctx && valid < kTile) {
+        if (ch == 0 && k < gi.nctx && valid < kTile) {
           // Rows past the end of the context hold whatever the caller's slab or page holds
           // there; P is 0 for them, but 0 * NaN would still poison O, so zero those V rows
-          // before the PV product reads them (PV of half 1 is issued after half 0's).
+          // before the PV product reads them. The V tile must have landed first.
           const int stage = (int)(f % kStages);
+          if (!mbar_wait_bounded(&sm.v_full[stage], (uint32_t)((f / kStages) & 1), abort_flag)) {
+            fail(kDetailWaitKvFull);
+            ok = false;
+            break;
+          }
           uint8_t* vbase = smem + kSmemV + stage * kKBytesPerStage;
           const int chunks_per_box = (kTile - valid) * 8;   // 16-byte chunks
-          for (int i = t; i < 2 * chunks_per_box; i += kRowsPerHalf) {
+          for (int i = t; i < 2 * chunks_per_box; i += kRows) {
             const int box = i / chunks_per_box, r = i - box * chunks_per_box;
             *reinterpret_cast<uint4*>(vbase + box * kKVBoxBytes + (valid + r / 8) * 128 + (r % 8) * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
@@ -554,29 +606,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         m_used = m_new;
         tc_fence_before();
-        mbar_arrive(&sm.p_full[h][bf]);
+        mbar_arrive(&sm.p_full[f & 1]);
       }
       if (!ok) break;
-      // ---- epilogue of the segment: wait for the last PV product, then O / l for this row
+      // ---- epilogue of the segment: wait for the last PV product, combine the two column
+      // halves' sums, then O / l for this thread's 64 dims of its row
       const long long lf = f - 1;
-      if (!mbar_wait_bounded(&sm.pv_done[h][lf & 1], (uint32_t)((lf >> 1) & 1), abort_flag)) {
+      if (!mbar_wait_bounded(&sm.pv_done, (uint32_t)(lf & 1), abort_flag)) {
         fail(kDetailWaitPvDone);
         ok = false;
         break;
       }
       tc_fence_after();
-      const bool whole = (kb == 0) && (ke == ui.ntiles);
-      const int s_cnt = min(p.s_per_tile, p.S - ui.qt * p.s_per_tile);
-      const bool row_valid = row < p.G * s_cnt;
-      const int s_idx = ui.qt * p.s_per_tile + row / p.G;
-      const int hq = ui.kvh * p.G + row % p.G;
+      sm.xsum[ch][t] = l;
+      mbar_arrive(&sm.l_bar);
+      if (!mbar_wait_bounded(&sm.l_bar, (uint32_t)(nseg & 1), abort_flag)) {
+        fail(kDetailWaitTicket);
+        ok = false;
+        break;
+      }
+      l += sm.xsum[ch ^ 1][t];
+      ++nseg;
+      const bool whole = (kb == 0) && (ke == gi.ntiles);
+      const bool row_valid = t < nrows;
+      const int s_idx = qt * p.s_per_tile + t / p.G;
+      const int hq = gi.kvh * p.G + t % p.G;
       const float inv_l = 1.0f / l;
       const float lse2 = m_used + log2f(l);
-      const size_t slot = (size_t)w.u + (size_t)cta;   // unique per (unit, CTA) pair
-      __nv_bfloat16* orow = p.out + (((size_t)ui.b * p.S + s_idx) * p.Hq + hq) * kD;
-      float* prow = partials + (slot * 256 + row) * kD;
+      // partial slot unique per (group, team, query tile)
+      const size_t slot = ((size_t)w.u + (size_t)team) * (size_t)p.nq + (size_t)qt;
+      __nv_bfloat16* orow = p.out + (((size_t)gi.b * p.S + s_idx) * p.Hq + hq) * kD + 64 * ch;
+      float* prow = partials + (slot * kRows + t) * kD + 64 * ch;
 #pragma unroll 1
-      for (int cb = 0; cb < kD / 32; ++cb) {
+      for (int cb = 0; cb < 2; ++cb) {
         uint32_t orr[32];
         tmem_ld32(o_tm + 32u * cb, orr);
         tmem_wait_ld();
@@ -601,11 +663,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
       }
-      if (row_valid) {
+      if (row_valid && ch == 0) {
         if (whole) {
-          if (p.lse) p.lse[((size_t)ui.b * p.Hq + hq) * p.S + s_idx] = lse2 * 0.69314718055994531f;
+          if (p.lse) p.lse[((size_t)gi.b * p.Hq + hq) * p.S + s_idx] = lse2 * 0.69314718055994531f;
         } else {
-          plse[slot * 256 + row] = lse2;
+          plse[slot * kRows + t] = lse2;
         }
       }
       w.advance(p, hdr);
@@ -627,11 +689,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
-// Merges the partials of units cut between CTAs. One CTA per (unit, 32 query rows); a warp
-// merges 4 rows, each lane 4 of the 128 dims, reading every contributor's row with coalesced
-// 512-byte loads: O = sum_j 2^(lse_j - M) O_j / sum_j 2^(lse_j - M), M = max_j lse_j.
+// Merges the partials of groups cut between teams (flash-decoding combine). One warp per query
+// row, 8 rows per CTA; lane j reads contributor j's log2-sum-exp, and every lane reads 4 of the
+// 128 dims of every contributor's row (coalesced 512-byte rows), 8 contributors in flight:
+//   O = sum_j 2^(lse_j - M) O_j / sum_j 2^(lse_j - M),  M = max_j lse_j.
 struct MergeParams {
-  int32_t S, Hq, Hkv, G, qtiles, s_per_tile, units;
+  int32_t S, Hq, Hkv, G, nq, s_per_tile, groups;
   __nv_bfloat16* out;
   float* lse;
   const uint8_t* ws;
@@ -640,79 +703,62 @@ struct MergeParams {
 
 __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   pdl_wait();
-  const int u = blockIdx.x;
+  const int u = blockIdx.x;             // group
+  const int qt = blockIdx.z;            // query tile
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.y * kMergeRows + warp;
   const AttnMeta* meta = reinterpret_cast<const AttnMeta*>(p.ws + p.off_meta);
   const int32_t* ustart = reinterpret_cast<const int32_t*>(p.ws + p.off_ustart);
   const long long T = meta->total_tiles, Pe = meta->p_eff;
   if (T <= 0) return;
   const long long us = ustart[u], ue = ustart[u + 1];
-  const long long c_lo = owner_cta(us, T, Pe), c_hi = owner_cta(ue - 1, T, Pe);
-  if (c_lo == c_hi) return;   // a whole unit: the attention kernel wrote it
-  const int qt = u % p.qtiles;
-  const int bk = u / p.qtiles;
-  const int kvh = bk % p.Hkv, b = bk / p.Hkv;
+  const long long c_lo = owner_team(us, T, Pe), c_hi = owner_team(ue - 1, T, Pe);
+  if (c_lo == c_hi) return;   // a whole group: the attention kernel wrote it
+  const int kvh = u % p.Hkv, b = u / p.Hkv;
   const int s_cnt = min(p.s_per_tile, p.S - qt * p.s_per_tile);
-  const int nrows = p.G * s_cnt;
+  if (row >= p.G * s_cnt) return;
   const float* partials = reinterpret_cast<const float*>(p.ws + p.off_partials);
   const float* plse = reinterpret_cast<const float*>(p.ws + p.off_lse);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = (int)(c_hi - c_lo + 1);
-  for (int rr = 0; rr < 4; ++rr) {
-    const int row = blockIdx.y * kMergeRows + warp * 4 + rr;
-    if (row >= nrows) break;
-    // per-contributor log2-sum-exp: lanes take contributors, then a warp max / sum
-    float mx = -INFINITY;
-    for (int j = lane; j < n; j += 32) mx = fmaxf(mx, plse[((size_t)u + (size_t)(c_lo + j)) * 256 + row]);
+  auto slot_of = [&](int j) { return ((size_t)u + (size_t)(c_lo + j)) * (size_t)p.nq + (size_t)qt; };
+  float mx = -INFINITY;
+  for (int j = lane; j < n; j += 32) mx = fmaxf(mx, plse[slot_of(j) * kRows + row]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float wsum = 0.f;
-    for (int j0 = 0; j0 < n; j0 += 32) {
-      const int j = j0 + lane;
-      const float wl = (j < n) ? ex2(plse[((size_t)u + (size_t)(c_lo + j)) * 256 + row] - mx) : 0.f;
-      float ws_part = wl;
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int cnt = min(32, n - j0);
+    const float wl = (lane < cnt) ? ex2(plse[slot_of(j0 + lane) * kRows + row] - mx) : 0.f;
+    float part = wl;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ws_part += __shfl_xor_sync(0xffffffffu, ws_part, o);
-      wsum += ws_part;
-      const int cnt = min(32, n - j0);
-      int jj = 0;
-      for (; jj + 4 <= cnt; jj += 4) {
-        float4 v[4];
-        float wv[4];
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    wsum += part;
+    for (int jj = 0; jj < cnt; jj += 8) {
+      float4 v[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          wv[q] = __shfl_sync(0xffffffffu, wl, jj + q);
-          const size_t sl = (size_t)u + (size_t)(c_lo + j0 + jj + q);
-          v[q] = reinterpret_cast<const float4*>(partials + (sl * 256 + row) * kD)[lane];
-        }
+      for (int q = 0; q < 8; ++q)
+        v[q] = (jj + q < cnt) ? reinterpret_cast<const float4*>(partials + (slot_of(j0 + jj + q) * kRows + row) * kD)[lane]
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc.x = fmaf(wv[q], v[q].x, acc.x);
-          acc.y = fmaf(wv[q], v[q].y, acc.y);
-          acc.z = fmaf(wv[q], v[q].z, acc.z);
-          acc.w = fmaf(wv[q], v[q].w, acc.w);
-        }
-      }
-      for (; jj < cnt; ++jj) {
-        const float wq = __shfl_sync(0xffffffffu, wl, jj);
-        const size_t sl = (size_t)u + (size_t)(c_lo + j0 + jj);
-        const float4 v = reinterpret_cast<const float4*>(partials + (sl * 256 + row) * kD)[lane];
-        acc.x = fmaf(wq, v.x, acc.x);
-        acc.y = fmaf(wq, v.y, acc.y);
-        acc.z = fmaf(wq, v.z, acc.z);
-        acc.w = fmaf(wq, v.w, acc.w);
+      for (int q = 0; q < 8; ++q) {
+        const float wq = __shfl_sync(0xffffffffu, wl, (jj + q) & 31);
+        acc.x = fmaf(wq, v[q].x, acc.x);
+        acc.y = fmaf(wq, v[q].y, acc.y);
+        acc.z = fmaf(wq, v[q].z, acc.z);
+        acc.w = fmaf(wq, v[q].w, acc.w);
       }
     }
-    const float inv = 1.0f / wsum;
-    const int s_idx = qt * p.s_per_tile + row / p.G;
-    const int hq = kvh * p.G + row % p.G;
-    __nv_bfloat16* orow = p.out + (((size_t)b * p.S + s_idx) * p.Hq + hq) * kD;
-    uint2 o;
-    o.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    o.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(orow)[lane] = o;
-    if (p.lse && lane == 0) p.lse[((size_t)b * p.Hq + hq) * p.S + s_idx] = (mx + log2f(wsum)) * 0.69314718055994531f;
   }
+  const float inv = 1.0f / wsum;
+  const int s_idx = qt * p.s_per_tile + row / p.G;
+  const int hq = kvh * p.G + row % p.G;
+  __nv_bfloat16* orow = p.out + (((size_t)b * p.S + s_idx) * p.Hq + hq) * kD;
+  uint2 o;
+  o.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  o.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(orow)[lane] = o;
+  if (p.lse && lane == 0) p.lse[((size_t)b * p.Hq + hq) * p.S + s_idx] = (mx + log2f(wsum)) * 0.69314718055994531f;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -741,31 +787,14 @@ bool make_map(CUtensorMap* m, const void* base, int heads, long long rows, int b
   return r == CUDA_SUCCESS;
 }
 
-// Launch with the programmatic-stream-serialization attribute: the kernel may start while the
-// previous kernel on the stream finishes; it reads no input before griddepcontrol.wait.
-template <typename Kern, typename Params>
-cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const Params& prm) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, prm);
-}
-
 }  // namespace
 
 bool attn_tc_supported(const tt_attn_args_t* a) {
   if (a->dtype != TT_BF16 || a->head_dim != kD) return false;
   const int G = a->num_q_heads / a->num_kv_heads;
-  if (G > 256) return false;
+  if (G > kRows) return false;                       // one block position's heads fit one query tile
   if (a->block_size > kTile) return false;
-  if (a->page_table && (a->page_size % kTile) != 0) return false;
+  if (a->page_table && (a->page_size % kTile) != 0) return false;   // a tile never crosses a page
   // TMA needs 16-byte aligned bases
   const uintptr_t al = reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->k_blk) |
                        reinterpret_cast<uintptr_t>(a->v_blk) | reinterpret_cast<uintptr_t>(a->k_ctx) |
@@ -778,11 +807,13 @@ AttnPlan attn_tc_plan(const tt_attn_args_t* a, int num_sms) {
   AttnPlan pl{};
   const int G = a->num_q_heads / a->num_kv_heads;
   const int S = a->block_size;
-  pl.s_per_tile = std::min(S, 256 / G);
-  pl.qtiles = (S + pl.s_per_tile - 1) / pl.s_per_tile;
-  pl.units = a->batch * a->num_kv_heads * pl.qtiles;
-  pl.grid = std::max(1, num_sms);
-  pl.slots = (size_t)pl.units + (size_t)pl.grid;
+  pl.s_per_tile = std::min(S, kRows / G);
+  pl.qtiles = (S + pl.s_per_tile - 1) / pl.s_per_tile;        // nq, CTAs per team
+  pl.units = a->batch * a->num_kv_heads;                        // groups
+  const int sms = std::max(1, num_sms);
+  const int teams = std::max(1, sms / pl.qtiles);
+  pl.grid = teams * pl.qtiles;
+  pl.slots = ((size_t)pl.units + (size_t)teams) * (size_t)pl.qtiles;
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -791,8 +822,8 @@ AttnPlan attn_tc_plan(const tt_attn_args_t* a, int num_sms) {
   };
   pl.off_meta = take(sizeof(AttnMeta));
   pl.off_ustart = take(sizeof(int32_t) * ((size_t)pl.units + 1));
-  pl.off_partials = take(sizeof(float) * pl.slots * 256 * kD);
-  pl.off_lse = take(sizeof(float) * pl.slots * 256);
+  pl.off_partials = take(sizeof(float) * pl.slots * kRows * kD);
+  pl.off_lse = take(sizeof(float) * pl.slots * kRows);
   pl.total = off;
   return pl;
 }
@@ -817,9 +848,10 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   p.Hq = a->num_q_heads;
   p.Hkv = a->num_kv_heads;
   p.G = G;
-  p.qtiles = pl.qtiles;
+  p.nq = pl.qtiles;
   p.s_per_tile = pl.s_per_tile;
-  p.units = pl.units;
+  p.groups = pl.units;
+  p.teams = pl.grid / pl.qtiles;
   p.page_size = a->page_size;
   p.max_pages = a->max_pages_per_seq;
   p.num_pages = a->num_pages;
@@ -852,9 +884,9 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   mp.Hq = p.Hq;
   mp.Hkv = p.Hkv;
   mp.G = G;
-  mp.qtiles = pl.qtiles;
+  mp.nq = pl.qtiles;
   mp.s_per_tile = pl.s_per_tile;
-  mp.units = pl.units;
+  mp.groups = pl.units;
   mp.out = p.out;
   mp.lse = p.lse;
   mp.ws = p.ws;
@@ -863,7 +895,7 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   mp.off_partials = pl.off_partials;
   mp.off_lse = pl.off_lse;
   const int M = G * pl.s_per_tile;
-  const dim3 mgrid(pl.units, (M + kMergeRows - 1) / kMergeRows);
+  const dim3 mgrid(pl.units, (M + kMergeRows - 1) / kMergeRows, pl.qtiles);
   if (launch_pdl(attn_merge_kernel, mgrid, dim3(256), 0, stream, mp) != cudaSuccess) return TT_ERR_CUDA;
   return TT_OK;
 }

@@ -188,12 +188,53 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream serialization: it may start
+// while the previous kernel on the stream is finishing, runs a prologue that reads no input,
+// lets its own dependents start early, and waits for the previous kernel's memory before it
+// reads anything. Behind a kernel that does not allow early start, this is plain stream order.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename Kern, typename... Args>
+inline cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ------------------------------------------------------------------ arithmetic
 // Hardware base-2 exponential (MUFU.EX2 through the PTX ex2.approx instruction).
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for |x| <= 126: Cody-Waite split x = n + f with n = round(x) (taken
+// from the low mantissa bits of x + 1.5 * 2^23) and f in [-0.5, 0.5], then 2^f from a degree-4
+// polynomial fitted here to the relative error of 2^f on that interval (max 2.7e-6), and 2^n
+// added to the exponent field. Used for a share of the softmax exponentials so that they do not
+// all queue on the MUFU pipe.
+__device__ __forceinline__ float ex2_fma(float x) {
+  const float t = x + 12582912.0f;
+  const float fr = x - (t - 12582912.0f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  float p = 0.009570068679749966f;
+  p = fmaf(p, fr, 0.055917806923389435f);
+  p = fmaf(p, fr, 0.240247443318367f);
+  p = fmaf(p, fr, 0.6931218504905701f);
+  p = fmaf(p, fr, 0.9999992847442627f);
+  return __int_as_float(__float_as_int(p) + (n << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -157,6 +157,8 @@ template <typename T>
 __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskParams p) {
   using VT = VecTraits<T>;
   constexpr int N = VT::kN;
+  pdl_trigger();
+  pdl_wait();
   const long long cta = blockIdx.x;
   if (cta >= p.p_eff) return;
   const int tid = threadIdx.x;
@@ -189,7 +191,9 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
       VT::to_float(raw, x);
       if (p.exclude_mask_token) {
         const int r = p.mask_token_id - vbase;
-        if (r >= 0 && r < N) x[r] = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < N; ++k)   // static indices keep x[] in registers
+          if (k == r) x[k] = -INFINITY;
       }
       float vm = x[0];
       int vi = 0;
@@ -332,9 +336,9 @@ int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cud
   p.off_conf = pl.layout.conf;
   p.off_argmax = pl.layout.argmax;
   if (a->dtype == TT_BF16)
-    unmask_kernel<__nv_bfloat16><<<pl.grid, kUnmaskThreads, 0, stream>>>(p);
+    launch_pdl(unmask_kernel<__nv_bfloat16>, dim3(pl.grid), dim3(kUnmaskThreads), 0, stream, p);
   else
-    unmask_kernel<float><<<pl.grid, kUnmaskThreads, 0, stream>>>(p);
+    launch_pdl(unmask_kernel<float>, dim3(pl.grid), dim3(kUnmaskThreads), 0, stream, p);
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }
 

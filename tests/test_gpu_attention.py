@@ -60,7 +60,8 @@ CASES = [
     (2, 16, 64, 1, 128, [250, 10], torch.bfloat16, 0),
     (2, 5, 12, 4, 128, [77, 190], torch.bfloat16, 0),
     (3, 16, 32, 2, 128, [1000, 3000, 17], torch.bfloat16, 256),
-    (2, 16, 32, 2, 128, [4100, 64], torch.bfloat16, 64),
+    (2, 16, 32, 2, 128, [4100, 64], torch.bfloat16, 128),
+    (2, 16, 32, 2, 128, [130, 700], torch.bfloat16, 512),
     (1, 16, 4, 1, 64, [64], torch.float32, 0),
     (3, 7, 8, 2, 128, [0, 90, 300], torch.float32, 0),
     (2, 16, 4, 1, 64, [100, 37], torch.float32, 32),
