@@ -35,7 +35,7 @@ EXPORTED = [
     "tt_status_string", "tt_version",
     "tt_denoise_attn_workspace_bytes", "tt_denoise_attn",
     "tt_adaln_workspace_bytes", "tt_adaln_modulate",
-    "tt_unmask_workspace_bytes", "tt_unmask_step",
+    "tt_unmask_workspace_bytes", "tt_unmask_step", "tt_unmask_step_noalloc",
     "tt_get_device_error",
 ]
 
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.tt_unmask_workspace_bytes.argtypes = [ctypes.POINTER(UnmaskArgs)]
         L.tt_unmask_step.restype = ctypes.c_int
         L.tt_unmask_step.argtypes = [ctypes.POINTER(UnmaskArgs), _vp, ctypes.c_size_t, _vp]
+        L.tt_unmask_step_noalloc.restype = ctypes.c_int
+        L.tt_unmask_step_noalloc.argtypes = [ctypes.POINTER(UnmaskArgs), _vp]
         L.tt_get_device_error.restype = ctypes.c_int
         L.tt_get_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
@@ -222,6 +224,11 @@ def tt_unmask_workspace_bytes(args: UnmaskArgs) -> int:
 def tt_unmask_step(args: UnmaskArgs, workspace: torch.Tensor, stream=None) -> None:
     _check(lib().tt_unmask_step(ctypes.byref(args), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream)), "tt_unmask_step")
+
+
+def tt_unmask_step_noalloc(args: UnmaskArgs, stream=None) -> None:
+    """tt_unmask_step with the library's static scratch: no workspace, nothing allocated."""
+    _check(lib().tt_unmask_step_noalloc(ctypes.byref(args), _stream(stream)), "tt_unmask_step_noalloc")
 
 
 def tt_get_device_error(workspace: torch.Tensor, stream=None):

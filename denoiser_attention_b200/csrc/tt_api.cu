@@ -151,6 +151,12 @@ int tt_unmask_step(const tt_unmask_args_t* a, void* ws, size_t ws_bytes, tt_stre
   return unmask_launch(a, pl, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int tt_unmask_step_noalloc(const tt_unmask_args_t* a, tt_stream_t stream) {
+  const int st = validate_unmask(a);
+  if (st != TT_OK) return st;
+  return unmask_launch_static(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int tt_get_device_error(void* ws, tt_stream_t stream, uint32_t* detail) {
   if (!ws) return TT_ERR_INVALID_ARGUMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

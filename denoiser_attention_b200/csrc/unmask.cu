@@ -17,6 +17,7 @@
 #include <cmath>
 #include <cstdio>
 #include <algorithm>
+#include <mutex>
 
 #include "tt_common.cuh"
 #include "tt_internal.h"
@@ -340,6 +341,57 @@ int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cud
   else
     launch_pdl(unmask_kernel<float>, dim3(pl.grid), dim3(kUnmaskThreads), 0, stream, p);
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- no-allocation variant
+// The same kernel and launch as above, but its scratch is a fixed-size array in this module's
+// static device memory instead of a caller workspace. It serves callers that cannot allocate
+// device memory at the point of the call: a host runtime that has no CUDA allocator of its own
+// (it owns only the logits/token buffers handed to it), or a thread that must not enter an
+// allocator (e.g. one running under an allocator lock, or a real-time decode loop that forbids
+// allocation after start-up).
+//
+// The layout is the one layout_for() gives for the largest supported sizes, fixed once, so its
+// offsets never move between calls of different sizes; the kernel returns the merge tickets it
+// uses to zero, so after the one clearing at setup every later call finds them at zero.
+constexpr int kStaticMaxRows = 4096;   // batch * block_size
+constexpr int kStaticMaxGrid = 1024;   // CTAs (partial slots beyond the rows)
+constexpr size_t kStaticScratchBytes = 168 * 1024;
+
+static __device__ __align__(256) uint8_t g_unmask_scratch[kStaticScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+uint8_t* g_static_ptr[kMaxDevices] = {};
+}  // namespace
+
+int unmask_launch_static(const tt_unmask_args_t* a, cudaStream_t stream) {
+  const int rows = a->batch * a->block_size;
+  if (rows > kStaticMaxRows) return TT_ERR_WORKSPACE_TOO_SMALL;
+  const UnmaskLayout L = layout_for(kStaticMaxRows, kStaticMaxRows, kStaticMaxGrid);
+  if (L.total > kStaticScratchBytes) return TT_ERR_WORKSPACE_TOO_SMALL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TT_ERR_CUDA;
+  uint8_t* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    ws = g_static_ptr[dev];
+    if (!ws) {
+      // Setup, once per device, with that device current: resolve the array's address and clear
+      // the header and the ticket counters (everything before the partial slots), stream-ordered
+      // before the first launch.
+      void* sym = nullptr;
+      if (cudaGetSymbolAddress(&sym, g_unmask_scratch) != cudaSuccess || !sym) return TT_ERR_CUDA;
+      if (cudaMemsetAsync(sym, 0, L.partials, stream) != cudaSuccess) return TT_ERR_CUDA;
+      ws = static_cast<uint8_t*>(sym);
+      g_static_ptr[dev] = ws;
+    }
+  }
+  UnmaskPlan pl = unmask_plan(a, device_sm_count());
+  pl.grid = std::min(pl.grid, kStaticMaxGrid);
+  pl.layout = L;
+  return unmask_launch(a, pl, ws, stream);
 }
 
 }  // namespace tt

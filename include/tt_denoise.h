@@ -210,6 +210,29 @@ int tt_unmask_step(const tt_unmask_args_t* args, void* workspace, size_t workspa
                    tt_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * tt_unmask_step_noalloc: tt_unmask_step without a workspace and without any allocation.
+ *
+ * The paper has no counterpart: this is an interface variant of the confidence-threshold step
+ * above (same arguments, same kernel, same results) for callers that cannot allocate device
+ * memory when they call it, e.g. a host runtime with no CUDA allocator of its own that owns only
+ * the buffers handed to it, or a decode loop that forbids allocation once running. Its scratch
+ * is a fixed array in the library's static device memory (168 KiB per device).
+ *
+ *   - Limit: batch * block_size <= 4096. Larger sizes return TT_ERR_WORKSPACE_TOO_SMALL (the
+ *     built-in scratch is too small) before anything is launched; use tt_unmask_step instead.
+ *   - Setup: the first call on a device (with that device current) resolves the scratch address
+ *     and enqueues on `stream` the clearing of its counters; make that first call before any
+ *     stream capture begins. Later calls only launch the kernel, which leaves the counters at
+ *     zero again. A failure of the setup returns TT_ERR_CUDA.
+ *   - One scratch per device, shared by all callers: calls on the same device must be ordered
+ *     (one stream, or events between streams). Calls that overlap on the device race on the
+ *     scratch and give undefined results.
+ *   - This is the one entry point that keeps library state (the scratch and its address).
+ *   - The kernel sets no device error word; tt_get_device_error does not apply.
+ * ------------------------------------------------------------------------------------------- */
+int tt_unmask_step_noalloc(const tt_unmask_args_t* args, tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Device-side error word of a workspace (any of the three). Synchronises `stream`, reads the
  * word and clears it. Returns TT_OK, TT_ERR_DEVICE (bad page id / context length) or
  * TT_ERR_DEVICE_TIMEOUT (a bounded wait inside a kernel gave up). *detail (host, may be NULL)
