@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import re
 import math
 import os
 import statistics
@@ -247,16 +248,15 @@ def run_ours(args):
     # events recorded inside the graph must be "external" to become timestamped graph nodes
     mk = lambda: torch.cuda.Event(enable_timing=True, external=True)
     ev = [(mk(), mk(), mk(), mk()) for _ in range(M)]
-    timed_step = StepWithEvents(step)
     g = torch.cuda.CUDAGraph()
     cap_stream = torch.cuda.Stream(device=dev)
     cap_stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap_stream):
         with torch.cuda.graph(g, stream=cap_stream):
             for j in range(M):
-                timed_step.run(sets[j % n_sets], outs[j % n_sets], ev[j])
+                step.run(sets[j % n_sets], out_attn=outs[j % n_sets], events=ev[j])
     torch.cuda.current_stream().wait_stream(cap_stream)
-    launches_per_step = 6
+    launches_per_step = api.RefinementStep.LAUNCHES
 
     # warm-up: at least W steps and about half a second, untimed
     reps_w = max(1, math.ceil(args.warmup / M))
@@ -332,7 +332,7 @@ def run_ours(args):
             "config": {"workload": workload_desc(w), "global_batch": global_batch,
                        "seq_len": a.ctx_lens[0] + S, "parallelism": f"dp{world} (independent sequences)",
                        "l2": f"{n_sets} rotating input sets of {ws_bytes / 1e6:.1f} MB (> 4x L2)",
-                       "timing": f"CUDA graph of {M} steps replayed; events on the replay stream"},
+                       "timing": f"CUDA graph of {M} steps replayed (each step three concurrent branches on forked streams); per-kernel events on the streams the kernels run on"},
             "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                          "frac": attn_gbs / peak, "traffic": traffic, "kernel": "attn_tc_kernel",
                          "peak_source": peak_src, "algorithmic_bytes_per_launch": kv_bytes},
@@ -350,39 +350,23 @@ def run_ours(args):
     return result
 
 
-class StepWithEvents:
-    """RefinementStep.run with CUDA events around the attention and unmask launches."""
-
-    def __init__(self, step):
-        self.step = step
-
-    def run(self, b, out, ev):
-        from denoiser_attention_b200 import api
-        st = self.step
-        w = st.w
-        mod = api.adaln_cond(b.tau, w["w1"], w["b1"], w["w2"], w["b2"], w["w3"], w["b3"], w["layer_emb"])
-        api.adaln_norm_modulate(b.h, w["norm_w"], mod, eps=st.eps)
-        ev[0].record()
-        api.denoise_attention(b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
-                              page_size=st.page_size, ctx_stride=st.ctx_stride, softmax_scale=st.softmax_scale,
-                              out=out)
-        ev[1].record()
-        api.adaln_gated_residual(b.h, b.f, mod)
-        ev[2].record()
-        api.unmask_step(b.logits, b.tokens, b.is_masked, gamma=st.gamma, inv_temperature=st.inv_temperature,
-                        mask_token_id=st.mask_token_id, remaining_steps=st.remaining_steps, want_conf=False)
-        ev[3].record()
-
-
 def measured_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it matches the kernel."""
-    p = os.path.join(ROOT, "profiles", "attn_tc_kernel_decode_bf16.traffic.json")
-    if os.path.exists(p):
-        try:
-            return json.load(open(p)).get("dram_bytes_per_launch")
-        except Exception:
-            return None
-    return None
+    """DRAM bytes (read + write) per attention launch from the committed ncu summary of the decode
+    workload, or None when that summary is absent or was taken on another version of the kernel
+    source (its recorded sha256 differs from the current attn_tc.cu)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "attn_tc_kernel_decode_bf16.md")
+    src = os.path.join(ROOT, "denoiser_attention_b200", "csrc", "attn_tc.cu")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    if not (m_bytes and m_sha):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
+        return None
+    return int(m_bytes.group(1))
 
 
 def run_e2e(step, inp, ad, logits, w, dev, args, world):

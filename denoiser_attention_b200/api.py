@@ -9,7 +9,8 @@ kernels. Workspaces are cached per (device, size) and zero-filled once, as the A
     adaln_norm_modulate  modulated RMSNorm prologue                      (tt_adaln_modulate)
     adaln_gated_residual h + gate * f                                    (tt_adaln_modulate)
     unmask_step          ConfidenceSample, Algorithm 2 line 5            (tt_unmask_step)
-    RefinementStep       the whole step a1..a7 on one stream, from device or host buffers
+    RefinementStep       the whole step a2..a7 (three concurrent branches), device buffers
+    HostStep             the same step from pinned host buffers (copies included)
 """
 from __future__ import annotations
 
@@ -96,12 +97,15 @@ def adaln_gated_residual(h, f, mod, out=None, ws_tag: str = "adaln"):
 
 def unmask_step(logits, tokens, is_masked, *, gamma: float, inv_temperature: float = 1.0, mask_token_id: int = 3,
                 exclude_mask_token: bool = False, remaining_steps: int = 0, want_conf: bool = True,
-                ws_tag: str = "unmask"):
+                ws_tag: str = "unmask", n_committed: Optional[torch.Tensor] = None,
+                n_masked: Optional[torch.Tensor] = None):
     """Updates tokens / is_masked in place; returns (n_committed, n_masked, conf, argmax)."""
     Bn, S, V = logits.shape
     dev = logits.device
-    n_committed = torch.empty(Bn, dtype=torch.int32, device=dev)
-    n_masked = torch.empty(Bn, dtype=torch.int32, device=dev)
+    if n_committed is None:
+        n_committed = torch.empty(Bn, dtype=torch.int32, device=dev)
+    if n_masked is None:
+        n_masked = torch.empty(Bn, dtype=torch.int32, device=dev)
     conf = torch.empty((Bn, S), dtype=torch.float32, device=dev) if want_conf else None
     argmax = torch.empty((Bn, S), dtype=torch.int32, device=dev) if want_conf else None
     args = B.unmask_args(logits, tokens, is_masked, n_committed, n_masked, gamma=gamma,
@@ -132,7 +136,7 @@ class StepBuffers:
 
 
 class RefinementStep:
-    """One denoiser refinement step of TwoTower decoding on one GPU, one stream.
+    """One denoiser refinement step of TwoTower decoding on one GPU.
 
     a2  mod = adaLN-single(tau)                 (tau = masked fraction, Algorithm 2 line 3)
     a3  y = modulated RMSNorm(h)                (prologue; y feeds the out-of-scope QKV projection)
@@ -140,11 +144,21 @@ class RefinementStep:
     a5  h' = h + gate * f                       (f: the mixer output after its out-projection)
     a6/a7  ConfidenceSample on the vocabulary logits (tokens / mask updated in place)
     The weights (adaLN MLP, per-layer embedding, norm weight) live on the device.
+
+    The step has three independent branches: a2 -> a3 -> a5 (modulation), a4 (attention) and
+    a6/a7 (unmask). With concurrent=True (the default) the attention and the unmask run on two
+    side streams forked from the caller's stream and joined back into it before run() returns,
+    so the three branches overlap on the device (and appear as parallel branches of a CUDA graph
+    captured around run()). Every output is allocated on the caller's stream before the fork.
     """
+
+    # kernel launches per step: adaLN COND (3 batched GEMVs), RMSNorm prologue, attention +
+    # split-KV merge, gated residual, unmask
+    LAUNCHES = 8
 
     def __init__(self, weights: Dict[str, torch.Tensor], *, gamma: float, inv_temperature: float = 1.0,
                  mask_token_id: int = 3, page_size: int = 0, ctx_stride: int = 0, softmax_scale: float = 1.0,
-                 eps: float = 1e-5, remaining_steps: int = 0):
+                 eps: float = 1e-5, remaining_steps: int = 0, concurrent: bool = True):
         self.w = weights
         self.gamma = gamma
         self.inv_temperature = inv_temperature
@@ -154,20 +168,59 @@ class RefinementStep:
         self.softmax_scale = softmax_scale
         self.eps = eps
         self.remaining_steps = remaining_steps
-        self._args = None
+        self.concurrent = concurrent
+        self._streams = {}
 
-    def run(self, b: StepBuffers, out_attn: Optional[torch.Tensor] = None):
+    def _side(self, dev):
+        key = dev.index if dev.index is not None else torch.cuda.current_device()
+        if key not in self._streams:
+            mk = lambda: torch.cuda.Event()
+            self._streams[key] = (torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev), mk(), mk(), mk())
+        return self._streams[key]
+
+    def run(self, b: StepBuffers, out_attn: Optional[torch.Tensor] = None, events=None):
+        """Runs the step on the current stream. events: optional 4 timing events recorded around
+        the attention (0, 1) and the unmask (2, 3) launches, on the streams they run on."""
         w = self.w
-        mod = adaln_cond(b.tau, w["w1"], w["b1"], w["w2"], w["b2"], w["w3"], w["b3"], w["layer_emb"])
-        y = adaln_norm_modulate(b.h, w["norm_w"], mod, eps=self.eps)
-        o = denoise_attention(b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
+        dev = b.q.device
+        main = torch.cuda.current_stream(dev)
+        out_attn = torch.empty_like(b.q) if out_attn is None else out_attn
+        Bn = b.q.shape[0]
+        nc = torch.empty(Bn, dtype=torch.int32, device=dev)
+        nm = torch.empty(Bn, dtype=torch.int32, device=dev)
+        if self.concurrent:
+            s_attn, s_unm, fork, join_a, join_u = self._side(dev)
+            fork.record(main)
+            s_attn.wait_event(fork)
+            s_unm.wait_event(fork)
+        else:
+            s_attn = s_unm = main
+
+        with torch.cuda.stream(s_attn):
+            if events is not None:
+                events[0].record(s_attn)
+            denoise_attention(b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
                               page_size=self.page_size, ctx_stride=self.ctx_stride,
                               softmax_scale=self.softmax_scale, out=out_attn)
+            if events is not None:
+                events[1].record(s_attn)
+        with torch.cuda.stream(s_unm):
+            if events is not None:
+                events[2].record(s_unm)
+            unmask_step(b.logits, b.tokens, b.is_masked, gamma=self.gamma, inv_temperature=self.inv_temperature,
+                        mask_token_id=self.mask_token_id, remaining_steps=self.remaining_steps, want_conf=False,
+                        n_committed=nc, n_masked=nm)
+            if events is not None:
+                events[3].record(s_unm)
+        mod = adaln_cond(b.tau, w["w1"], w["b1"], w["w2"], w["b2"], w["w3"], w["b3"], w["layer_emb"])
+        y = adaln_norm_modulate(b.h, w["norm_w"], mod, eps=self.eps)
         h_new = adaln_gated_residual(b.h, b.f, mod)
-        nc, nm, _, _ = unmask_step(b.logits, b.tokens, b.is_masked, gamma=self.gamma,
-                                   inv_temperature=self.inv_temperature, mask_token_id=self.mask_token_id,
-                                   remaining_steps=self.remaining_steps, want_conf=False)
-        return {"mod": mod, "y": y, "attn": o, "h": h_new, "n_committed": nc, "n_masked": nm}
+        if self.concurrent:
+            join_a.record(s_attn)
+            join_u.record(s_unm)
+            main.wait_event(join_a)
+            main.wait_event(join_u)
+        return {"mod": mod, "y": y, "attn": out_attn, "h": h_new, "n_committed": nc, "n_masked": nm}
 
 
 class HostStep:

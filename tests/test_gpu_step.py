@@ -80,3 +80,27 @@ def test_graph_captured_step_matches_eager(cuda_lib):
     torch.cuda.synchronize()
     assert torch.equal(o_graph, o_eager)
     assert torch.equal(bufs.tokens, tok_eager)
+
+
+def test_concurrent_branches_match_sequential(cuda_lib):
+    # the three branches on forked streams give the bits of the one-stream order
+    w, inp, ad, logits = _workload_inputs("decode_bf16")
+    B, S = w.attn.batch, w.attn.block_size
+    dev = "cuda"
+    weights = {k: getattr(ad, k).to(dev) for k in ("w1", "b1", "w2", "b2", "w3", "b3", "layer_emb", "norm_w")}
+    results = []
+    for concurrent in (False, True, True):
+        bufs = api.StepBuffers(tau=ad.tau.to(dev), h=ad.h.to(dev), f=ad.f.to(dev), q=inp.q.to(dev),
+                               k_blk=inp.k_blk.to(dev), v_blk=inp.v_blk.to(dev), k_ctx=inp.k_ctx.to(dev),
+                               v_ctx=inp.v_ctx.to(dev), ctx_lens=inp.ctx_lens.to(dev), page_table=None,
+                               logits=logits.to(dev),
+                               tokens=torch.full((B, S), 3, dtype=torch.int32, device=dev),
+                               is_masked=torch.ones((B, S), dtype=torch.uint8, device=dev))
+        step = api.RefinementStep(weights, gamma=w.gamma, ctx_stride=inp.ctx_stride, concurrent=concurrent)
+        r = step.run(bufs)
+        torch.cuda.synchronize()
+        results.append({k: v.cpu() for k, v in r.items()} | {"tokens": bufs.tokens.cpu(),
+                                                               "is_masked": bufs.is_masked.cpu()})
+    for other in results[1:]:
+        for k, v in results[0].items():
+            assert torch.equal(v, other[k]), k
