@@ -492,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         fail(kDetailWaitTicket);
         return false;
       }
+      __syncwarp();
       row_max = fmaxf(mine, sm.xmax[ff & 1][ch ^ 1][t]);
       return true;
     };
@@ -509,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           ok = false;
           break;
         }
+        __syncwarp();   // lanes leave the wait one by one; the tcgen05 accesses are warp-collective
         tc_fence_after();
         uint32_t sr[64];
         tmem_ld32(s_tm, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -571,8 +573,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ok = false;
             break;
           }
+          __syncwarp();
           tc_fence_after();
-          if (resc) {
+          // rows decide separately; the O accesses are warp-collective, so the warp rescales when
+          // any of its rows needs it (factor is 1 for the others)
+          if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
             for (int cb = 0; cb < 2; ++cb) {
               uint32_t orr[32];
@@ -625,6 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         ok = false;
         break;
       }
+      __syncwarp();
       l += sm.xsum[ch ^ 1][t];
       ++nseg;
       const bool whole = (kb == 0) && (ke == gi.ntiles);
