@@ -11,6 +11,9 @@ kernels. Workspaces are cached per (device, size) and zero-filled once, as the A
     unmask_step          ConfidenceSample, Algorithm 2 line 5            (tt_unmask_step)
     RefinementStep       the whole step a2..a7 (three concurrent branches), device buffers
     HostStep             the same step from pinned host buffers (copies included)
+    block_tau            tau_b = masked fraction of sequence b, on the device  (tt_block_tau)
+    RefinementLoop       Algorithm 2: T steps of one block, tau from the mask on the device,
+                         capturable as one CUDA graph (no host round trip between steps)
 """
 from __future__ import annotations
 
@@ -221,6 +224,40 @@ class RefinementStep:
             main.wait_event(join_a)
             main.wait_event(join_u)
         return {"mod": mod, "y": y, "attn": out_attn, "h": h_new, "n_committed": nc, "n_masked": nm}
+
+
+def block_tau(is_masked: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """tau[b] = |{l : is_masked[b, l]}| / S on the device (Algorithm 2 line 3)."""
+    tau = torch.empty(is_masked.shape[0], dtype=torch.float32, device=is_masked.device) if out is None else out
+    B.tt_block_tau(is_masked, tau)
+    return tau
+
+
+class RefinementLoop:
+    """Algorithm 2 on the device: the T refinement steps of one block.
+
+    for r = 1..T:  tau = masked fraction (tt_block_tau, on the device)
+                   the RefinementStep with tau and step r's inputs
+                   (ConfidenceSample updates the shared tokens / mask in place)
+    Every step's inputs (q, K/V, logits, h, f) are the caller's, one StepBuffers per step; tokens
+    and is_masked are shared by all steps, and each step's tau buffer is written by the loop.
+    run() only enqueues work, so the whole loop can be captured in one CUDA graph and replayed
+    with no host synchronisation between steps. The per-step outputs (attention, modulation,
+    residual, commit counts) are returned for inspection.
+    """
+
+    def __init__(self, step: RefinementStep):
+        self.step = step
+
+    def run(self, steps: "list[StepBuffers]", tokens: torch.Tensor, is_masked: torch.Tensor,
+            out_attn: "Optional[list]" = None):
+        outs = []
+        for r, b in enumerate(steps):
+            block_tau(is_masked, out=b.tau)
+            b.tokens, b.is_masked = tokens, is_masked
+            o = self.step.run(b, out_attn=None if out_attn is None else out_attn[r])
+            outs.append(o)
+        return outs
 
 
 class HostStep:

@@ -35,7 +35,7 @@ EXPORTED = [
     "tt_status_string", "tt_version",
     "tt_denoise_attn_workspace_bytes", "tt_denoise_attn",
     "tt_adaln_workspace_bytes", "tt_adaln_modulate",
-    "tt_unmask_workspace_bytes", "tt_unmask_step", "tt_unmask_step_noalloc",
+    "tt_unmask_workspace_bytes", "tt_unmask_step", "tt_unmask_step_noalloc", "tt_block_tau",
     "tt_get_device_error",
 ]
 
@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         L.tt_unmask_step.restype = ctypes.c_int
         L.tt_unmask_step.argtypes = [ctypes.POINTER(UnmaskArgs), _vp, ctypes.c_size_t, _vp]
         L.tt_unmask_step_noalloc.restype = ctypes.c_int
+        L.tt_block_tau.restype = ctypes.c_int
+        L.tt_block_tau.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp]
         L.tt_unmask_step_noalloc.argtypes = [ctypes.POINTER(UnmaskArgs), _vp]
         L.tt_get_device_error.restype = ctypes.c_int
         L.tt_get_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -229,6 +231,14 @@ def tt_unmask_step(args: UnmaskArgs, workspace: torch.Tensor, stream=None) -> No
 def tt_unmask_step_noalloc(args: UnmaskArgs, stream=None) -> None:
     """tt_unmask_step with the library's static scratch: no workspace, nothing allocated."""
     _check(lib().tt_unmask_step_noalloc(ctypes.byref(args), _stream(stream)), "tt_unmask_step_noalloc")
+
+
+def tt_block_tau(is_masked: torch.Tensor, tau: torch.Tensor, stream=None) -> None:
+    """tau[b] = masked positions of sequence b / S, on the device."""
+    if is_masked.dtype != torch.uint8 or tau.dtype != torch.float32:
+        raise ValueError("is_masked must be uint8 and tau float32")
+    Bn, S = is_masked.shape
+    _check(lib().tt_block_tau(_ptr(is_masked), Bn, S, _ptr(tau), _stream(stream)), "tt_block_tau")
 
 
 def tt_get_device_error(workspace: torch.Tensor, stream=None):

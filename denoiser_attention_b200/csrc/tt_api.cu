@@ -157,6 +157,11 @@ int tt_unmask_step_noalloc(const tt_unmask_args_t* a, tt_stream_t stream) {
   return unmask_launch_static(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, tt_stream_t stream) {
+  if (!is_masked || !tau || batch < 1 || block_size < 1) return TT_ERR_INVALID_ARGUMENT;
+  return block_tau_launch(is_masked, batch, block_size, tau, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int tt_get_device_error(void* ws, tt_stream_t stream, uint32_t* detail) {
   if (!ws) return TT_ERR_INVALID_ARGUMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -394,4 +394,31 @@ int unmask_launch_static(const tt_unmask_args_t* a, cudaStream_t stream) {
   return unmask_launch(a, pl, ws, stream);
 }
 
+// ---------------------------------------------------------------- Algorithm 2 line 3
+// tau_b = |{l : position l of sequence b is masked}| / S, one warp per sequence, so a multi-step
+// refinement loop can feed the next step's time input from the mask on the device.
+constexpr int kTauThreads = 128;
+
+__global__ void __launch_bounds__(kTauThreads) block_tau_kernel(const uint8_t* __restrict__ is_masked, int B, int S,
+                                                                float* __restrict__ tau) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (kTauThreads / 32) + warp;
+  if (b >= B) return;
+  int n = 0;
+  for (int l = lane; l < S; l += 32) n += is_masked[(size_t)b * S + l] ? 1 : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+  if (lane == 0) tau[b] = (float)n / (float)S;
+}
+
+int block_tau_launch(const uint8_t* is_masked, int B, int S, float* tau, cudaStream_t stream) {
+  const int per = kTauThreads / 32;
+  return launch_pdl(block_tau_kernel, dim3((B + per - 1) / per), dim3(kTauThreads), 0, stream, is_masked, B, S, tau) ==
+                 cudaSuccess
+             ? TT_OK
+             : TT_ERR_CUDA;
+}
+
 }  // namespace tt

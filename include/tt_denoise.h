@@ -8,6 +8,7 @@
  *   tt_denoise_attn    layer-aligned denoiser attention, the paper §2.1 Eq. (1)
  *   tt_adaln_modulate  adaLN-single time conditioning, the paper §2.1 "Time conditioning"
  *   tt_unmask_step     confidence-threshold unmasking, the paper §2.2 "Sampling", Algorithm 2
+ *   tt_block_tau       the step's time input from the mask, Algorithm 2 line 3
  *
  * Conventions shared by every entry point
  *   - Every pointer named in an args struct is a DEVICE pointer (cudaMalloc'd or equivalent)
@@ -231,6 +232,17 @@ int tt_unmask_step(const tt_unmask_args_t* args, void* workspace, size_t workspa
  *   - The kernel sets no device error word; tt_get_device_error does not apply.
  * ------------------------------------------------------------------------------------------- */
 int tt_unmask_step_noalloc(const tt_unmask_args_t* args, tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * tt_block_tau: the time input of one refinement step, the paper §2.2 Algorithm 2 line 3:
+ * tau_b = |{l : z_l = [MASK]}| / S, computed on the device from the mask so that a multi-step
+ * loop (captured in one CUDA graph) needs no host round trip between steps.
+ *   is_masked  device u8 [batch][block_size], 1 = still masked
+ *   tau        device float [batch], written
+ * Errors: TT_ERR_INVALID_ARGUMENT (null pointer, batch < 1, block_size < 1); TT_ERR_CUDA on a
+ * failed launch. No workspace.
+ * ------------------------------------------------------------------------------------------- */
+int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, tt_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Device-side error word of a workspace (any of the three). Synchronises `stream`, reads the

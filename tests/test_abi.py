@@ -154,3 +154,17 @@ def test_adaln_workspace(lib):
     a = _adaln_args(batch=8, mlp_width=256)
     assert lib.tt_adaln_workspace_bytes(ctypes.byref(a)) == 256 + 2 * 4 * 8 * 256
     assert lib.tt_adaln_modulate(ctypes.byref(a), 4096, 100, None) == B.TT_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.parametrize("ptrs,batch,S", [
+    ((None, 0x1000), 2, 16),        # no mask
+    ((0x1000, None), 2, 16),        # no output
+    ((0x1000, 0x2000), 0, 16),      # empty batch
+    ((0x1000, 0x2000), 2, 0),       # empty block
+])
+def test_block_tau_host_validation(lib, ptrs, batch, S):
+    # rejected on the host before any launch (the pointers are never dereferenced)
+    f = lib.tt_block_tau
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    assert f(ptrs[0], batch, S, ptrs[1], None) == 1   # TT_ERR_INVALID_ARGUMENT
