@@ -309,6 +309,15 @@ def run_ours(args):
     unmask_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
     attn_ms = max_over_ranks(attn_ms, dev)
     unmask_ms = max_over_ranks(unmask_ms, dev)
+    # the same two kernels alone (own graphs over the same rotating input sets), for context: inside
+    # the step they share the GPU with the other branches
+    attn_iso_ms = max_over_ranks(isolated_ms(lambda b, o: api.denoise_attention(
+        b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
+        page_size=step.page_size, ctx_stride=step.ctx_stride, softmax_scale=step.softmax_scale, out=o),
+        sets, outs, cap_stream), dev)
+    unmask_iso_ms = max_over_ranks(isolated_ms(lambda b, o: api.unmask_step(
+        b.logits, b.tokens, b.is_masked, gamma=step.gamma, inv_temperature=step.inv_temperature,
+        mask_token_id=step.mask_token_id, want_conf=False), sets, outs, cap_stream), dev)
 
     a = w.attn
     kv_bytes = B * (a.ctx_lens[0] + S) * a.num_kv_heads * a.head_dim * 2 * 2
@@ -337,6 +346,9 @@ def run_ours(args):
                          "frac": attn_gbs / peak, "traffic": traffic, "kernel": "attn_tc_kernel",
                          "peak_source": peak_src, "algorithmic_bytes_per_launch": kv_bytes},
             "attn_us": attn_ms * 1e3, "attn_kv_gbs": attn_gbs, "attn_query_tok_s": B * S / (attn_ms * 1e-3),
+            "attn_isolated_us": attn_iso_ms * 1e3, "attn_isolated_kv_gbs": kv_bytes / (attn_iso_ms * 1e-3) / 1e9,
+            "attn_isolated_frac": kv_bytes / (attn_iso_ms * 1e-3) / 1e9 / peak,
+            "unmask_isolated_us": unmask_iso_ms * 1e3,
             "unmask_us": unmask_ms * 1e3, "unmask_steps_per_s": 1.0 / (unmask_ms * 1e-3),
             "unmask_logits_gbs": unmask_gbs, "unmask_frac": unmask_gbs / peak,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
@@ -367,6 +379,31 @@ def measured_traffic():
     if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
         return None
     return int(m_bytes.group(1))
+
+
+def isolated_ms(op, sets, outs, cap_stream, reps: int = 20):
+    """Mean device time of op(buffers, out) from a CUDA graph of one launch per rotating input set,
+    replayed back to back (the sets together exceed L2, so each launch reads from HBM)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    cap_stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap_stream):
+        with torch.cuda.graph(g, stream=cap_stream):
+            for b, o in zip(sets, outs):
+                op(b, o)
+    torch.cuda.current_stream().wait_stream(cap_stream)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * len(sets))
+    del g
+    return ms
 
 
 def run_e2e(step, inp, ad, logits, w, dev, args, world):

@@ -12,6 +12,7 @@ kernels. Workspaces are cached per (device, size) and zero-filled once, as the A
     RefinementStep       the whole step a2..a7 (three concurrent branches), device buffers
     HostStep             the same step from pinned host buffers (copies included)
     block_tau            tau_b = masked fraction of sequence b, on the device  (tt_block_tau)
+    append_block_kv      block commit: the block's context KV into the paged cache (tt_kv_append)
     RefinementLoop       Algorithm 2: T steps of one block, tau from the mask on the device,
                          capturable as one CUDA graph (no host round trip between steps)
 """
@@ -231,6 +232,18 @@ def block_tau(is_masked: torch.Tensor, out: Optional[torch.Tensor] = None) -> to
     tau = torch.empty(is_masked.shape[0], dtype=torch.float32, device=is_masked.device) if out is None else out
     B.tt_block_tau(is_masked, tau)
     return tau
+
+
+def append_block_kv(k_new, v_new, k_ctx, v_ctx, page_table, ctx_lens, free_pages, free_count,
+                    ws_tag: str = "kv_append") -> torch.Tensor:
+    """Appends the committed block's context K/V [B][S][Hkv][d] after each sequence's context in the
+    paged pool [num_pages][page_size][Hkv][d], taking pages from the free stack; page_table,
+    ctx_lens and free_count are updated in place. Returns the workspace (its error word reports a
+    sequence that could not be given pages)."""
+    args = B.kv_append_args(k_new, v_new, k_ctx, v_ctx, page_table, ctx_lens, free_pages, free_count)
+    ws = workspace(max(256, B.tt_kv_append_workspace_bytes(args)), k_new.device, ws_tag)
+    B.tt_kv_append(args, ws)
+    return ws
 
 
 class RefinementLoop:

@@ -36,6 +36,7 @@ EXPORTED = [
     "tt_denoise_attn_workspace_bytes", "tt_denoise_attn",
     "tt_adaln_workspace_bytes", "tt_adaln_modulate",
     "tt_unmask_workspace_bytes", "tt_unmask_step", "tt_unmask_step_noalloc", "tt_block_tau",
+    "tt_kv_append_workspace_bytes", "tt_kv_append",
     "tt_get_device_error",
 ]
 
@@ -73,6 +74,15 @@ class UnmaskArgs(ctypes.Structure):
     ]
 
 
+class KvAppendArgs(ctypes.Structure):
+    _fields_ = [
+        ("batch", _i32), ("block_size", _i32), ("num_kv_heads", _i32), ("head_dim", _i32), ("dtype", _i32),
+        ("k_new", _vp), ("v_new", _vp), ("k_ctx", _vp), ("v_ctx", _vp), ("page_table", _vp), ("ctx_lens", _vp),
+        ("free_pages", _vp), ("free_count", _vp), ("page_size", _i32), ("max_pages_per_seq", _i32),
+        ("num_pages", _i32),
+    ]
+
+
 _lib = None
 
 
@@ -100,6 +110,10 @@ def lib() -> ctypes.CDLL:
         L.tt_unmask_step.argtypes = [ctypes.POINTER(UnmaskArgs), _vp, ctypes.c_size_t, _vp]
         L.tt_unmask_step_noalloc.restype = ctypes.c_int
         L.tt_block_tau.restype = ctypes.c_int
+        L.tt_kv_append_workspace_bytes.restype = ctypes.c_size_t
+        L.tt_kv_append_workspace_bytes.argtypes = [ctypes.POINTER(KvAppendArgs)]
+        L.tt_kv_append.restype = ctypes.c_int
+        L.tt_kv_append.argtypes = [ctypes.POINTER(KvAppendArgs), _vp, ctypes.c_size_t, _vp]
         L.tt_block_tau.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp]
         L.tt_unmask_step_noalloc.argtypes = [ctypes.POINTER(UnmaskArgs), _vp]
         L.tt_get_device_error.restype = ctypes.c_int
@@ -239,6 +253,29 @@ def tt_block_tau(is_masked: torch.Tensor, tau: torch.Tensor, stream=None) -> Non
         raise ValueError("is_masked must be uint8 and tau float32")
     Bn, S = is_masked.shape
     _check(lib().tt_block_tau(_ptr(is_masked), Bn, S, _ptr(tau), _stream(stream)), "tt_block_tau")
+
+
+# ------------------------------------------------------------------------------------ block commit
+def kv_append_args(k_new, v_new, k_ctx, v_ctx, page_table, ctx_lens, free_pages, free_count) -> KvAppendArgs:
+    B, S, Hkv, d = k_new.shape
+    a = KvAppendArgs()
+    a.batch, a.block_size, a.num_kv_heads, a.head_dim = B, S, Hkv, d
+    a.dtype = _dtype_code(k_new.dtype)
+    a.k_new, a.v_new, a.k_ctx, a.v_ctx = _ptr(k_new), _ptr(v_new), _ptr(k_ctx), _ptr(v_ctx)
+    a.page_table, a.ctx_lens = _ptr(page_table), _ptr(ctx_lens)
+    a.free_pages, a.free_count = _ptr(free_pages), _ptr(free_count)
+    a.num_pages, a.page_size = int(k_ctx.shape[0]), int(k_ctx.shape[1])
+    a.max_pages_per_seq = int(page_table.shape[1])
+    return a
+
+
+def tt_kv_append_workspace_bytes(args: KvAppendArgs) -> int:
+    return int(lib().tt_kv_append_workspace_bytes(ctypes.byref(args)))
+
+
+def tt_kv_append(args: KvAppendArgs, workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().tt_kv_append(ctypes.byref(args), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)), "tt_kv_append")
 
 
 def tt_get_device_error(workspace: torch.Tensor, stream=None):

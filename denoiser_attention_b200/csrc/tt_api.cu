@@ -81,6 +81,21 @@ static int validate_adaln(const tt_adaln_args_t* a) {
   }
 }
 
+static int validate_kv_append(const tt_kv_append_args_t* a) {
+  if (!a) return TT_ERR_INVALID_ARGUMENT;
+  if (a->batch < 1 || a->block_size < 1 || a->num_kv_heads < 1 || a->head_dim < 1) return TT_ERR_INVALID_ARGUMENT;
+  if (a->dtype != TT_F32 && a->dtype != TT_BF16) return TT_ERR_INVALID_ARGUMENT;
+  if (!a->k_new || !a->v_new || !a->k_ctx || !a->v_ctx || !a->page_table || !a->ctx_lens || !a->free_pages ||
+      !a->free_count)
+    return TT_ERR_INVALID_ARGUMENT;
+  if (a->page_size < 1 || a->max_pages_per_seq < 1 || a->num_pages < 1) return TT_ERR_INVALID_ARGUMENT;
+  const int elt = (a->dtype == TT_BF16) ? 2 : 4;
+  if ((a->head_dim * elt) % 16 != 0) return TT_ERR_UNSUPPORTED;
+  if (!aligned16(a->k_new) || !aligned16(a->v_new) || !aligned16(a->k_ctx) || !aligned16(a->v_ctx))
+    return TT_ERR_UNSUPPORTED;
+  return TT_OK;
+}
+
 }  // namespace tt
 
 using namespace tt;
@@ -160,6 +175,18 @@ int tt_unmask_step_noalloc(const tt_unmask_args_t* a, tt_stream_t stream) {
 int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, tt_stream_t stream) {
   if (!is_masked || !tau || batch < 1 || block_size < 1) return TT_ERR_INVALID_ARGUMENT;
   return block_tau_launch(is_masked, batch, block_size, tau, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tt_kv_append_workspace_bytes(const tt_kv_append_args_t* a) {
+  return validate_kv_append(a) == TT_OK ? kHeaderBytes : 0;
+}
+
+int tt_kv_append(const tt_kv_append_args_t* a, void* ws, size_t ws_bytes, tt_stream_t stream) {
+  const int st = validate_kv_append(a);
+  if (st != TT_OK) return st;
+  if (!ws) return TT_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < kHeaderBytes) return TT_ERR_WORKSPACE_TOO_SMALL;
+  return kv_append_launch(a, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int tt_get_device_error(void* ws, tt_stream_t stream, uint32_t* detail) {

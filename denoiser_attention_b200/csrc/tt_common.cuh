@@ -26,6 +26,8 @@ enum : uint32_t {
   kDetailBadPage = 1,        // page id outside [0, num_pages)
   kDetailCtxTooLong = 2,     // context length beyond the page table / contiguous slab
   kDetailNegativeLen = 3,    // negative context length
+  kDetailOutOfPages = 4,     // block commit: the free-page stack cannot provide the pages needed
+  kDetailPageTableFull = 5,  // block commit: the context would outgrow max_pages_per_seq pages
   kDetailWaitQFull = 0x100,  // bounded waits: which wait gave up
   kDetailWaitKvFull = 0x101,
   kDetailWaitKvEmpty = 0x102,

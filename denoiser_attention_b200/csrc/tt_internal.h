@@ -24,6 +24,9 @@ int unmask_launch_static(const tt_unmask_args_t* a, cudaStream_t stream);
 // tau[b] = masked positions of sequence b / S.
 int block_tau_launch(const uint8_t* is_masked, int B, int S, float* tau, cudaStream_t stream);
 
+// ---------------------------------------------------------------- block commit (paged KV append)
+int kv_append_launch(const tt_kv_append_args_t* a, void* ws, cudaStream_t stream);
+
 // ---------------------------------------------------------------- adaLN
 size_t adaln_workspace_bytes(const tt_adaln_args_t* a);
 int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream);

@@ -9,6 +9,7 @@
  *   tt_adaln_modulate  adaLN-single time conditioning, the paper §2.1 "Time conditioning"
  *   tt_unmask_step     confidence-threshold unmasking, the paper §2.2 "Sampling", Algorithm 2
  *   tt_block_tau       the step's time input from the mask, Algorithm 2 line 3
+ *   tt_kv_append       block commit into the paged context cache, Algorithm 1 line 8
  *
  * Conventions shared by every entry point
  *   - Every pointer named in an args struct is a DEVICE pointer (cudaMalloc'd or equivalent)
@@ -232,6 +233,49 @@ int tt_unmask_step(const tt_unmask_args_t* args, void* workspace, size_t workspa
  *   - The kernel sets no device error word; tt_get_device_error does not apply.
  * ------------------------------------------------------------------------------------------- */
 int tt_unmask_step_noalloc(const tt_unmask_args_t* args, tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * tt_kv_append: block commit into the paged context cache, the paper §2.2 Algorithm 1 line 8
+ * ("update the AR context" once block b is committed): the context tower's K and V for the S
+ * tokens of the committed block are appended after each sequence's current context, taking new
+ * pages from a free-page stack as needed. The context tower that produces k_new / v_new is not
+ * part of this library.
+ *
+ * For sequence b with L = ctx_lens[b]: rows L .. L+S-1 of its context are written from
+ * k_new[b] / v_new[b] through page_table[b] (position p lives in page page_table[b][p / page_size],
+ * slot p % page_size); the pages holding positions >= ceil(L / page_size) * page_size are taken
+ * from the top of the free stack, in order, and entered in page_table[b]; ctx_lens[b] += S.
+ * Pages are allocated with one atomic per sequence, so which free pages a sequence receives
+ * depends on the order the sequences run in (the content each sequence sees does not).
+ *
+ *   k_new, v_new   device [batch][block_size][num_kv_heads][head_dim] (dtype)
+ *   k_ctx, v_ctx   device paged pool [num_pages][page_size][num_kv_heads][head_dim] (dtype), written
+ *   page_table     device int32 [batch][max_pages_per_seq], in/out
+ *   ctx_lens       device int32 [batch], in/out
+ *   free_pages     device int32 [>= *free_count]: entries [0, *free_count) are free page ids
+ *   free_count     device int32 scalar, in/out (decreases by the pages taken)
+ * Errors (host): TT_ERR_INVALID_ARGUMENT for null pointers or sizes < 1; TT_ERR_UNSUPPORTED unless
+ * head_dim * element size is a multiple of 16 bytes and the four tensors are 16-byte aligned.
+ * Errors (device, via tt_get_device_error; the sequence is left unchanged): the free stack is too
+ * short, or the context would need more than max_pages_per_seq pages.
+ * Workspace: tt_kv_append_workspace_bytes() (the error word), zero-filled before first use.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct {
+  int32_t batch, block_size, num_kv_heads, head_dim;
+  int32_t dtype;                  /* tt_dtype_t */
+  const void* k_new;
+  const void* v_new;
+  void* k_ctx;
+  void* v_ctx;
+  int32_t* page_table;
+  int32_t* ctx_lens;
+  const int32_t* free_pages;
+  int32_t* free_count;
+  int32_t page_size, max_pages_per_seq, num_pages;
+} tt_kv_append_args_t;
+
+size_t tt_kv_append_workspace_bytes(const tt_kv_append_args_t* args);
+int tt_kv_append(const tt_kv_append_args_t* args, void* workspace, size_t workspace_bytes, tt_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * tt_block_tau: the time input of one refinement step, the paper §2.2 Algorithm 2 line 3:

@@ -17,6 +17,7 @@ Source: "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Conte
   confidence_argmax,
   confidence_commit      the paper §2.2 "Sampling" and Algorithm 2 (ConfidenceSample)
   refine_block           the paper Algorithm 2 (single-block confidence unmasking loop)
+  append_block           the paper Algorithm 1 line 8 (the committed block joins the context)
 
 Readings of points the paper leaves open (each is also listed in the design notes):
   * attention mask: every block query sees all L_b context keys and all S block keys; the only
@@ -258,6 +259,18 @@ def refine_block(batch: int, block_size: int, steps: int, gamma: float,
                                                       inv_temperature, None, rem)
         records.append((r, tau.copy(), nc.copy()))
     return tokens, is_masked, records
+
+
+def append_block(ctx_k: Sequence[np.ndarray], ctx_v: Sequence[np.ndarray], k_new: np.ndarray,
+                 v_new: np.ndarray):
+    """Algorithm 1 line 8: after block b is committed, the context tower's K/V of its S tokens
+    follow the sequence's existing context. ctx_k[b] / ctx_v[b] are [L_b][Hkv][d] (the logical
+    context, e.g. from gather_context); k_new / v_new are [B][S][Hkv][d]. Returns the new
+    per-sequence contexts [L_b + S][Hkv][d] and lengths. Storage (pages) is not modelled: a paged
+    implementation must gather back to exactly these arrays."""
+    out_k = [np.concatenate([np.asarray(ctx_k[b]), np.asarray(k_new[b])], axis=0) for b in range(len(ctx_k))]
+    out_v = [np.concatenate([np.asarray(ctx_v[b]), np.asarray(v_new[b])], axis=0) for b in range(len(ctx_v))]
+    return out_k, out_v, [k.shape[0] for k in out_k]
 
 
 def round_bf16(x) -> np.ndarray:

@@ -168,3 +168,23 @@ def test_block_tau_host_validation(lib, ptrs, batch, S):
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
     assert f(ptrs[0], batch, S, ptrs[1], None) == 1   # TT_ERR_INVALID_ARGUMENT
+
+
+def test_kv_append_host_validation(lib):
+    a = B.KvAppendArgs()
+    a.batch, a.block_size, a.num_kv_heads, a.head_dim, a.dtype = 2, 16, 2, 128, B.TT_BF16
+    for name in ("k_new", "v_new", "k_ctx", "v_ctx", "page_table", "ctx_lens", "free_pages", "free_count"):
+        setattr(a, name, 0x1000)
+    a.page_size, a.max_pages_per_seq, a.num_pages = 256, 8, 16
+    ws = ctypes.c_void_p(0x2000)
+    assert lib.tt_kv_append_workspace_bytes(ctypes.byref(a)) == 256
+    a.free_count = None
+    assert lib.tt_kv_append(ctypes.byref(a), ws, 256, None) == B.TT_ERR_INVALID_ARGUMENT
+    a.free_count = 0x1000
+    a.head_dim = 4                                   # 8 bytes per row: not a whole 16-byte vector
+    assert lib.tt_kv_append(ctypes.byref(a), ws, 256, None) == B.TT_ERR_UNSUPPORTED
+    a.head_dim = 128
+    a.k_ctx = 0x1008                                 # misaligned pool
+    assert lib.tt_kv_append(ctypes.byref(a), ws, 256, None) == B.TT_ERR_UNSUPPORTED
+    a.k_ctx = 0x1000
+    assert lib.tt_kv_append(ctypes.byref(a), ws, 64, None) == B.TT_ERR_WORKSPACE_TOO_SMALL

@@ -468,3 +468,43 @@ def test_round_bf16_matches_torch():
     assert diff.sum() <= 2
     m, e = np.frexp(r)
     assert np.all(np.rint(m * 256) == m * 256)
+
+
+# ---------------------------------------------------------------- block commit (Algorithm 1 line 8)
+def test_append_block_is_concatenation():
+    rs = np.random.default_rng(11)
+    lens = [0, 5, 17]
+    ctx_k = [rs.standard_normal((L, 2, 8)) for L in lens]
+    ctx_v = [rs.standard_normal((L, 2, 8)) for L in lens]
+    kn, vn = rs.standard_normal((3, 4, 2, 8)), rs.standard_normal((3, 4, 2, 8))
+    out_k, out_v, new_lens = O.append_block(ctx_k, ctx_v, kn, vn)
+    assert new_lens == [L + 4 for L in lens]
+    for b, L in enumerate(lens):
+        np.testing.assert_array_equal(out_k[b][:L], ctx_k[b])      # the old context is untouched
+        np.testing.assert_array_equal(out_k[b][L:], kn[b])         # the block follows it
+        np.testing.assert_array_equal(out_v[b][L:], vn[b])
+
+
+def test_append_then_attend_sees_the_committed_block():
+    # after the commit, the next block's queries attend to context + committed block + own block:
+    # the same as one softmax over the three key sets written out directly
+    rs = np.random.default_rng(12)
+    B, S, Hq, Hkv, d, L = 2, 3, 4, 2, 8, 5
+    ctx_k, ctx_v = rs.standard_normal((B, L, Hkv, d)), rs.standard_normal((B, L, Hkv, d))
+    kc, vc = rs.standard_normal((B, S, Hkv, d)), rs.standard_normal((B, S, Hkv, d))   # committed block
+    q, kb, vb = rs.standard_normal((B, S, Hq, d)), rs.standard_normal((B, S, Hkv, d)), rs.standard_normal((B, S, Hkv, d))
+    nk, nv, lens = O.append_block(list(ctx_k), list(ctx_v), kc, vc)
+    stride = max(lens)
+    k_slab = np.zeros((B, stride, Hkv, d)); v_slab = np.zeros((B, stride, Hkv, d))
+    for b in range(B):
+        k_slab[b, :lens[b]], v_slab[b, :lens[b]] = nk[b], nv[b]
+    got = O.denoise_attention(q, kb, vb, k_slab, v_slab, lens)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            keys = np.concatenate([ctx_k[b, :, h // G], kc[b, :, h // G], kb[b, :, h // G]])
+            vals = np.concatenate([ctx_v[b, :, h // G], vc[b, :, h // G], vb[b, :, h // G]])
+            x = q[b, :, h] @ keys.T
+            p = np.exp(x - x.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            np.testing.assert_allclose(got[b, :, h], p @ vals, rtol=0, atol=1e-12)
