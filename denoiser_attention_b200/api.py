@@ -9,6 +9,7 @@ kernels. Workspaces are cached per (device, size) and zero-filled once, as the A
     adaln_norm_modulate  modulated RMSNorm prologue                      (tt_adaln_modulate)
     adaln_gated_residual h + gate * f                                    (tt_adaln_modulate)
     unmask_step          ConfidenceSample, Algorithm 2 line 5            (tt_unmask_step)
+                         or the predict-and-noise sampler (keep_masked)
     RefinementStep       the whole step a2..a7 (three concurrent branches), device buffers
     HostStep             the same step from pinned host buffers (copies included)
     block_tau            tau_b = masked fraction of sequence b, on the device  (tt_block_tau)
@@ -102,8 +103,11 @@ def adaln_gated_residual(h, f, mod, out=None, ws_tag: str = "adaln"):
 def unmask_step(logits, tokens, is_masked, *, gamma: float, inv_temperature: float = 1.0, mask_token_id: int = 3,
                 exclude_mask_token: bool = False, remaining_steps: int = 0, want_conf: bool = True,
                 ws_tag: str = "unmask", n_committed: Optional[torch.Tensor] = None,
-                n_masked: Optional[torch.Tensor] = None):
-    """Updates tokens / is_masked in place; returns (n_committed, n_masked, conf, argmax)."""
+                n_masked: Optional[torch.Tensor] = None, keep_masked: Optional[int] = None):
+    """Updates tokens / is_masked in place; returns (n_committed, n_masked, conf, argmax).
+    keep_masked=None runs the confidence-threshold sampler; an int runs the predict-and-noise
+    sampler, which commits all but keep_masked of the masked positions (the least confident stay
+    masked; see linear_schedule_keep)."""
     Bn, S, V = logits.shape
     dev = logits.device
     if n_committed is None:
@@ -115,10 +119,16 @@ def unmask_step(logits, tokens, is_masked, *, gamma: float, inv_temperature: flo
     args = B.unmask_args(logits, tokens, is_masked, n_committed, n_masked, gamma=gamma,
                          inv_temperature=inv_temperature, mask_token_id=mask_token_id,
                          exclude_mask_token=exclude_mask_token, remaining_steps=remaining_steps, conf=conf,
-                         argmax=argmax)
+                         argmax=argmax, keep_masked=keep_masked)
     ws = workspace(max(256, B.tt_unmask_workspace_bytes(args)), dev, ws_tag, (tuple(logits.shape), logits.dtype))
     B.tt_unmask_step(args, ws)
     return n_committed, n_masked, conf, argmax
+
+
+def linear_schedule_keep(block_size: int, steps: int, r: int) -> int:
+    """Positions left masked after step r (1..T) under the linear schedule alpha_t = 1 - t:
+    the masked fraction after the step is t = (T - r) / T, i.e. floor(S (T - r) / T)."""
+    return (block_size * (steps - r)) // steps
 
 
 @dataclasses.dataclass

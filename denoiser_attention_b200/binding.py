@@ -27,6 +27,9 @@ TT_ERR_DEVICE_TIMEOUT = 6
 TT_F32 = 0
 TT_BF16 = 1
 
+TT_SAMPLER_CONFIDENCE = 0
+TT_SAMPLER_PREDICT_NOISE = 1
+
 TT_ADALN_COND = 0
 TT_ADALN_NORM_MODULATE = 1
 TT_ADALN_GATED_RESIDUAL = 2
@@ -70,7 +73,7 @@ class UnmaskArgs(ctypes.Structure):
         ("batch", _i32), ("block_size", _i32), ("vocab", _i32), ("dtype", _i32), ("logits", _vp),
         ("gamma", _f32), ("inv_temperature", _f32), ("mask_token_id", _i32), ("exclude_mask_token", _i32),
         ("remaining_steps", _i32), ("tokens", _vp), ("is_masked", _vp), ("conf", _vp), ("argmax", _vp),
-        ("n_committed", _vp), ("n_masked", _vp),
+        ("n_committed", _vp), ("n_masked", _vp), ("sampler", _i32), ("keep_masked", _i32),
     ]
 
 
@@ -220,7 +223,9 @@ def tt_adaln_modulate(args: AdalnArgs, workspace: torch.Tensor, stream=None) -> 
 # ------------------------------------------------------------------------------------------ unmask
 def unmask_args(logits, tokens, is_masked, n_committed, n_masked, *, gamma: float, inv_temperature: float = 1.0,
                 mask_token_id: int = 3, exclude_mask_token: bool = False, remaining_steps: int = 0,
-                conf=None, argmax=None) -> UnmaskArgs:
+                conf=None, argmax=None, keep_masked: Optional[int] = None) -> UnmaskArgs:
+    """keep_masked=None: the confidence-threshold sampler; an int: the predict-and-noise sampler
+    keeping that many positions masked."""
     B, S, V = logits.shape
     a = UnmaskArgs()
     a.batch, a.block_size, a.vocab, a.dtype = B, S, V, _dtype_code(logits.dtype)
@@ -230,6 +235,10 @@ def unmask_args(logits, tokens, is_masked, n_committed, n_masked, *, gamma: floa
     a.tokens, a.is_masked = _ptr(tokens), _ptr(is_masked)
     a.conf, a.argmax = _ptr(conf), _ptr(argmax)
     a.n_committed, a.n_masked = _ptr(n_committed), _ptr(n_masked)
+    if keep_masked is None:
+        a.sampler, a.keep_masked = TT_SAMPLER_CONFIDENCE, 0
+    else:
+        a.sampler, a.keep_masked = TT_SAMPLER_PREDICT_NOISE, int(keep_masked)
     return a
 
 

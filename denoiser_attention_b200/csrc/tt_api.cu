@@ -48,6 +48,8 @@ static int validate_unmask(const tt_unmask_args_t* a) {
   if (a->block_size > 1024) return TT_ERR_UNSUPPORTED;
   const int W = (a->dtype == TT_BF16) ? 8 : 4;
   if (a->vocab % W != 0 || !aligned16(a->logits)) return TT_ERR_UNSUPPORTED;
+  if (a->sampler != TT_SAMPLER_CONFIDENCE && a->sampler != TT_SAMPLER_PREDICT_NOISE) return TT_ERR_INVALID_ARGUMENT;
+  if (a->sampler == TT_SAMPLER_PREDICT_NOISE && a->keep_masked < 0) return TT_ERR_INVALID_ARGUMENT;
   return TT_OK;
 }
 

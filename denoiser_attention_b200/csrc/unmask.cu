@@ -86,6 +86,8 @@ struct UnmaskParams {
   int32_t mask_token_id;
   int32_t exclude_mask_token;
   int32_t remaining_steps;
+  int32_t sampler;           // tt_sampler_t
+  int32_t keep_masked;
   int32_t* tokens;
   uint8_t* is_masked;
   float* conf_out;
@@ -128,9 +130,15 @@ __device__ void commit_sequence(const UnmaskParams& p, int b, const float* conf_
   __syncthreads();
   const int n_masked = s_counts[0];
   const int n_ge = s_counts[1];
-  int need = 0;
-  if (n_masked > 0) need = (p.remaining_steps > 0) ? (n_masked + p.remaining_steps - 1) / p.remaining_steps : 1;
-  const int K = max(need, n_ge);
+  int K;
+  if (p.sampler == TT_SAMPLER_PREDICT_NOISE) {
+    // predict-and-noise: all but keep_masked of the masked positions are committed
+    K = max(0, n_masked - p.keep_masked);
+  } else {
+    int need = 0;
+    if (n_masked > 0) need = (p.remaining_steps > 0) ? (n_masked + p.remaining_steps - 1) / p.remaining_steps : 1;
+    K = max(need, n_ge);
+  }
   // a masked position commits iff its rank among masked positions (confidence descending,
   // position ascending) is below K; every position >= gamma ranks below n_ge <= K.
   for (int l = tid; l < S; l += blockDim.x) {
@@ -324,6 +332,8 @@ int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cud
   p.mask_token_id = a->mask_token_id;
   p.exclude_mask_token = a->exclude_mask_token;
   p.remaining_steps = a->remaining_steps;
+  p.sampler = a->sampler;
+  p.keep_masked = a->keep_masked;
   p.tokens = a->tokens;
   p.is_masked = a->is_masked;
   p.conf_out = a->conf;

@@ -170,6 +170,11 @@ size_t tt_adaln_workspace_bytes(const tt_adaln_args_t* args);
 int tt_adaln_modulate(const tt_adaln_args_t* args, void* workspace, size_t workspace_bytes,
                       tt_stream_t stream);
 
+typedef enum {
+  TT_SAMPLER_CONFIDENCE = 0,     /* commit every prediction with confidence >= gamma */
+  TT_SAMPLER_PREDICT_NOISE = 1   /* commit all but keep_masked, the least confident re-masked */
+} tt_sampler_t;
+
 /* ---------------------------------------------------------------------------------------------
  * ConfidenceSample, the paper §2.2 "Sampling" and Algorithm 2 line 5: the denoiser predicts
  * every masked position in parallel; predictions whose confidence reaches gamma are committed,
@@ -182,6 +187,13 @@ int tt_adaln_modulate(const tt_adaln_args_t* args, void* workspace, size_t works
  *   remaining_steps > 0 (the T - r + 1 of Algorithm 2), at least ceil(n_masked/remaining_steps)
  *   of the most confident masked positions are committed, so a block finishes within T steps.
  *   Positions already committed are never changed.
+ * sampler = TT_SAMPLER_PREDICT_NOISE selects the predict-and-noise sampler instead (the paper
+ *   §2.2 "Sampling", the standard sampler of block diffusion): every masked position is
+ *   predicted and the least confident ones are re-masked following the noise schedule, i.e. the
+ *   (n_masked - keep_masked) most confident masked positions are committed (confidence
+ *   descending, position ascending) and min(n_masked, keep_masked) stay masked; gamma and
+ *   remaining_steps are ignored. For the linear schedule alpha_t = 1 - t over T steps,
+ *   keep_masked after step r is floor(S * (T - r) / T).
  * Layouts: logits [B][S][V] E; tokens [B][S] int32 (in/out); is_masked [B][S] uint8 (in/out,
  *   0/1); conf [B][S] float and argmax [B][S] int32 (optional outputs, may be NULL);
  *   n_committed, n_masked [B] int32 outputs. exclude_mask_token != 0 removes the logit of
@@ -205,6 +217,8 @@ typedef struct {
   int32_t* argmax;           /* optional */
   int32_t* n_committed;
   int32_t* n_masked;
+  int32_t sampler;           /* tt_sampler_t; 0 (TT_SAMPLER_CONFIDENCE) when zero-initialised */
+  int32_t keep_masked;       /* TT_SAMPLER_PREDICT_NOISE: masked positions to keep, >= 0 */
 } tt_unmask_args_t;
 
 size_t tt_unmask_workspace_bytes(const tt_unmask_args_t* args);

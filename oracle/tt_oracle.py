@@ -17,6 +17,7 @@ Source: "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Conte
   confidence_argmax,
   confidence_commit      the paper §2.2 "Sampling" and Algorithm 2 (ConfidenceSample)
   refine_block           the paper Algorithm 2 (single-block confidence unmasking loop)
+  predict_noise_step     the predict-and-noise sampler (§2.2 "Sampling"), linear schedule
   append_block           the paper Algorithm 1 line 8 (the committed block joins the context)
 
 Readings of points the paper leaves open (each is also listed in the design notes):
@@ -235,6 +236,33 @@ def unmask_step(tokens, is_masked, logits, gamma: float, inv_temperature: float 
     conf, arg = confidence_argmax(logits, inv_temperature, exclude_token)
     t, m, nc, nm = confidence_commit(tokens, is_masked, conf, arg, gamma, remaining_steps)
     return t, m, nc, nm, conf, arg
+
+
+def predict_noise_step(tokens, is_masked, logits, keep_masked: int, inv_temperature: float = 1.0):
+    """The predict-and-noise sampler of block diffusion (the paper §2.2 "Sampling"): predict every
+    masked position (argmax, confidence as in confidence_argmax), then re-mask the least
+    confident ones so that min(n_masked, keep_masked) stay masked; i.e. commit the
+    (n_masked - keep_masked) most confident masked positions, confidence descending and position
+    ascending on ties. Committed positions are never changed."""
+    conf, arg = confidence_argmax(logits, inv_temperature)
+    tokens = np.array(tokens, dtype=np.int64, copy=True)
+    is_masked = np.array(is_masked, dtype=bool, copy=True)
+    n_committed = np.zeros(tokens.shape[0], dtype=np.int64)
+    for b in range(tokens.shape[0]):
+        masked = [l for l in range(tokens.shape[1]) if is_masked[b, l]]
+        k = max(0, len(masked) - keep_masked)
+        # stable sort by confidence, descending: equal confidences keep position order
+        order = sorted(masked, key=lambda l: -conf[b, l])
+        for l in order[:k]:
+            tokens[b, l] = arg[b, l]
+            is_masked[b, l] = False
+        n_committed[b] = k
+    return tokens, is_masked, n_committed, is_masked.sum(axis=1), conf, arg
+
+
+def linear_schedule_keep(block_size: int, steps: int, r: int) -> int:
+    """Masked positions left after step r of T under alpha_t = 1 - t (masked fraction t = (T-r)/T)."""
+    return (block_size * (steps - r)) // steps
 
 
 def refine_block(batch: int, block_size: int, steps: int, gamma: float,

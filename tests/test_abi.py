@@ -188,3 +188,19 @@ def test_kv_append_host_validation(lib):
     assert lib.tt_kv_append(ctypes.byref(a), ws, 256, None) == B.TT_ERR_UNSUPPORTED
     a.k_ctx = 0x1000
     assert lib.tt_kv_append(ctypes.byref(a), ws, 64, None) == B.TT_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_unmask_sampler_fields_validated(lib):
+    from denoiser_attention_b200 import binding as Bd
+    a = Bd.UnmaskArgs()
+    a.batch, a.block_size, a.vocab, a.dtype = 2, 16, 1024, Bd.TT_F32
+    for name in ("logits", "tokens", "is_masked", "n_committed", "n_masked"):
+        setattr(a, name, 0x1000)
+    a.gamma, a.inv_temperature = 0.8, 1.0
+    assert lib.tt_unmask_workspace_bytes(ctypes.byref(a)) > 0          # default: confidence sampler
+    a.sampler = 7
+    assert lib.tt_unmask_workspace_bytes(ctypes.byref(a)) == 0
+    a.sampler, a.keep_masked = Bd.TT_SAMPLER_PREDICT_NOISE, -1
+    assert lib.tt_unmask_workspace_bytes(ctypes.byref(a)) == 0
+    a.keep_masked = 4
+    assert lib.tt_unmask_workspace_bytes(ctypes.byref(a)) > 0

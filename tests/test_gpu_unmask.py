@@ -117,3 +117,47 @@ def test_block_loop_tiny_closes_in_T_steps(cuda_lib):
     t_or, m_or, _ = O.refine_block(1, S, T, w.gamma, lambda r, tau: synth.logits_normal(
         r, 1, S, w.vocab, w.logits_std, torch.float32).double().numpy())
     np.testing.assert_array_equal(tokens.cpu().numpy(), t_or)
+
+
+@pytest.mark.parametrize("B,S,V,dtype,keep", [
+    (4, 16, 131072, torch.bfloat16, 10),
+    (2, 64, 32000, torch.bfloat16, 0),
+    (3, 8, 1000, torch.float32, 3),
+    (2, 16, 1024, torch.float32, 16),     # keep >= masked: nothing commits
+])
+def test_predict_noise_matches_oracle(cuda_lib, B, S, V, dtype, keep):
+    from oracle import tt_oracle as O
+    logits = synth.logits_normal(V + S + keep, B, S, V, 3.0, dtype)
+    tokens, masked = _state(B, S, seed=V + keep, frac_masked=0.8)
+    dev = "cuda"
+    t, m = tokens.to(dev), masked.to(dev)
+    nc, nm, conf, arg = api.unmask_step(logits.to(dev), t, m, gamma=0.8, keep_masked=keep)
+    torch.cuda.synchronize()
+    t_or, m_or, nc_or, nm_or, conf_or, arg_or = O.predict_noise_step(tokens.numpy(), masked.numpy().astype(bool),
+                                                                     np64(logits), keep)
+    np.testing.assert_array_equal(arg.cpu().numpy(), arg_or)
+    assert np.abs(conf.cpu().double().numpy() - conf_or).max() <= 1e-5
+    np.testing.assert_array_equal(nc.cpu().numpy(), nc_or)
+    np.testing.assert_array_equal(nm.cpu().numpy(), nm_or)
+    np.testing.assert_array_equal(t.cpu().numpy(), t_or)
+    np.testing.assert_array_equal(m.cpu().numpy().astype(bool), m_or)
+
+
+def test_predict_noise_schedule_loop(cuda_lib):
+    # T steps of the linear schedule on the device: the trajectory (masked count per step, tokens)
+    # equals the oracle's, and the block is complete at step T
+    from oracle import tt_oracle as O
+    B, S, T, V = 2, 16, 5, 4096
+    dev = "cuda"
+    t = torch.full((B, S), 3, dtype=torch.int32, device=dev)
+    m = torch.ones((B, S), dtype=torch.uint8, device=dev)
+    t_or, m_or = np.full((B, S), 3), np.ones((B, S), bool)
+    for r in range(1, T + 1):
+        logits = synth.logits_normal(100 + r, B, S, V, 3.0, torch.bfloat16)
+        keep = api.linear_schedule_keep(S, T, r)
+        api.unmask_step(logits.to(dev), t, m, gamma=0.8, keep_masked=keep)
+        t_or, m_or, _, _, _, _ = O.predict_noise_step(t_or, m_or, np64(logits), O.linear_schedule_keep(S, T, r))
+        torch.cuda.synchronize()
+        assert int(m.sum()) == B * keep
+        np.testing.assert_array_equal(t.cpu().numpy(), t_or)
+    assert int(m.sum()) == 0

@@ -508,3 +508,47 @@ def test_append_then_attend_sees_the_committed_block():
             p = np.exp(x - x.max(axis=1, keepdims=True))
             p /= p.sum(axis=1, keepdims=True)
             np.testing.assert_allclose(got[b, :, h], p @ vals, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- predict-and-noise sampler
+def test_predict_noise_commits_top_k_by_brute_force():
+    rs = np.random.default_rng(21)
+    B, S, V = 3, 10, 17
+    logits = rs.standard_normal((B, S, V)) * 2
+    masked = rs.random((B, S)) < 0.7
+    tokens = np.where(masked, 3, rs.integers(0, V, (B, S)))
+    conf, arg = O.confidence_argmax(logits)
+    for keep in (0, 2, 5, 100):
+        t, m, nc, nm, _, _ = O.predict_noise_step(tokens, masked, logits, keep)
+        for b in range(B):
+            cand = [l for l in range(S) if masked[b, l]]
+            k = max(0, len(cand) - keep)
+            # brute force: the k positions whose (confidence, -position) is largest
+            best = sorted(cand, key=lambda l: (conf[b, l], -l), reverse=True)[:k]
+            assert set(np.flatnonzero(masked[b] & ~m[b])) == set(best)
+            assert nc[b] == k and nm[b] == len(cand) - k
+            for l in best:
+                assert t[b, l] == arg[b, l]
+            for l in range(S):
+                if not masked[b, l]:
+                    assert t[b, l] == tokens[b, l] and not m[b, l]   # committed positions untouched
+
+
+def test_predict_noise_ties_go_to_the_lower_position():
+    logits = np.zeros((1, 4, 8))
+    logits[0, :, 1] = 5.0                       # four positions with identical confidence
+    t, m, nc, _, _, _ = O.predict_noise_step(np.full((1, 4), 3), np.ones((1, 4), bool), logits, 2)
+    assert m[0].tolist() == [False, False, True, True] and nc[0] == 2
+
+
+def test_predict_noise_linear_schedule_finishes_at_T():
+    S, T = 16, 6
+    rs = np.random.default_rng(22)
+    tokens, masked = np.full((2, S), 3), np.ones((2, S), bool)
+    left = []
+    for r in range(1, T + 1):
+        keep = O.linear_schedule_keep(S, T, r)
+        tokens, masked, _, _, _, _ = O.predict_noise_step(tokens, masked, rs.standard_normal((2, S, 32)), keep)
+        left.append(int(masked[0].sum()))
+    # the masked fraction after step r is (T - r) / T of the block, rounded down; none left at T
+    assert left == [(S * (T - r)) // T for r in range(1, T + 1)] and left[-1] == 0
