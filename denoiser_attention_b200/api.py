@@ -14,6 +14,7 @@ kernels. Workspaces are cached per (device, size) and zero-filled once, as the A
     HostStep             the same step from pinned host buffers (copies included)
     block_tau            tau_b = masked fraction of sequence b, on the device  (tt_block_tau)
     append_block_kv      block commit: the block's context KV into the paged cache (tt_kv_append)
+    lmhead_unmask_step   the unmask step from hidden states, LM head fused (tt_lmhead_unmask_step)
     RefinementLoop       Algorithm 2: T steps of one block, tau from the mask on the device,
                          capturable as one CUDA graph (no host round trip between steps)
 """
@@ -122,6 +123,28 @@ def unmask_step(logits, tokens, is_masked, *, gamma: float, inv_temperature: flo
                          argmax=argmax, keep_masked=keep_masked)
     ws = workspace(max(256, B.tt_unmask_workspace_bytes(args)), dev, ws_tag, (tuple(logits.shape), logits.dtype))
     B.tt_unmask_step(args, ws)
+    return n_committed, n_masked, conf, argmax
+
+
+def lmhead_unmask_step(x, w, tokens, is_masked, *, gamma: float, inv_temperature: float = 1.0,
+                       mask_token_id: int = 3, exclude_mask_token: bool = False, remaining_steps: int = 0,
+                       want_conf: bool = True, keep_masked: Optional[int] = None, ws_tag: str = "lmhead"):
+    """unmask_step from the final hidden states x [B][S][D] and the LM-head weight w [V][D] (bf16):
+    the logits x w^T are reduced on the fly and never stored. Returns (n_committed, n_masked,
+    conf, argmax) and updates tokens / is_masked in place."""
+    Bn, S, _ = x.shape
+    dev = x.device
+    n_committed = torch.empty(Bn, dtype=torch.int32, device=dev)
+    n_masked = torch.empty(Bn, dtype=torch.int32, device=dev)
+    conf = torch.empty((Bn, S), dtype=torch.float32, device=dev) if want_conf else None
+    argmax = torch.empty((Bn, S), dtype=torch.int32, device=dev) if want_conf else None
+    args = B.lmhead_unmask_args(x, w, tokens, is_masked, n_committed, n_masked, gamma=gamma,
+                                inv_temperature=inv_temperature, mask_token_id=mask_token_id,
+                                exclude_mask_token=exclude_mask_token, remaining_steps=remaining_steps, conf=conf,
+                                argmax=argmax, keep_masked=keep_masked)
+    ws = workspace(max(256, B.tt_lmhead_unmask_workspace_bytes(args)), dev, ws_tag,
+                   (tuple(x.shape), int(w.shape[0])))
+    B.tt_lmhead_unmask_step(args, ws)
     return n_committed, n_masked, conf, argmax
 
 

@@ -40,6 +40,7 @@ EXPORTED = [
     "tt_adaln_workspace_bytes", "tt_adaln_modulate",
     "tt_unmask_workspace_bytes", "tt_unmask_step", "tt_unmask_step_noalloc", "tt_block_tau",
     "tt_kv_append_workspace_bytes", "tt_kv_append",
+    "tt_lmhead_unmask_workspace_bytes", "tt_lmhead_unmask_step",
     "tt_get_device_error",
 ]
 
@@ -86,6 +87,16 @@ class KvAppendArgs(ctypes.Structure):
     ]
 
 
+class LmheadUnmaskArgs(ctypes.Structure):
+    _fields_ = [
+        ("batch", _i32), ("block_size", _i32), ("hidden", _i32), ("vocab", _i32), ("dtype", _i32),
+        ("x", _vp), ("w", _vp), ("gamma", _f32), ("inv_temperature", _f32), ("mask_token_id", _i32),
+        ("exclude_mask_token", _i32), ("remaining_steps", _i32), ("tokens", _vp), ("is_masked", _vp),
+        ("conf", _vp), ("argmax", _vp), ("n_committed", _vp), ("n_masked", _vp), ("sampler", _i32),
+        ("keep_masked", _i32),
+    ]
+
+
 _lib = None
 
 
@@ -113,6 +124,10 @@ def lib() -> ctypes.CDLL:
         L.tt_unmask_step.argtypes = [ctypes.POINTER(UnmaskArgs), _vp, ctypes.c_size_t, _vp]
         L.tt_unmask_step_noalloc.restype = ctypes.c_int
         L.tt_block_tau.restype = ctypes.c_int
+        L.tt_lmhead_unmask_workspace_bytes.restype = ctypes.c_size_t
+        L.tt_lmhead_unmask_workspace_bytes.argtypes = [ctypes.POINTER(LmheadUnmaskArgs)]
+        L.tt_lmhead_unmask_step.restype = ctypes.c_int
+        L.tt_lmhead_unmask_step.argtypes = [ctypes.POINTER(LmheadUnmaskArgs), _vp, ctypes.c_size_t, _vp]
         L.tt_kv_append_workspace_bytes.restype = ctypes.c_size_t
         L.tt_kv_append_workspace_bytes.argtypes = [ctypes.POINTER(KvAppendArgs)]
         L.tt_kv_append.restype = ctypes.c_int
@@ -262,6 +277,36 @@ def tt_block_tau(is_masked: torch.Tensor, tau: torch.Tensor, stream=None) -> Non
         raise ValueError("is_masked must be uint8 and tau float32")
     Bn, S = is_masked.shape
     _check(lib().tt_block_tau(_ptr(is_masked), Bn, S, _ptr(tau), _stream(stream)), "tt_block_tau")
+
+
+# ------------------------------------------------------------------------------- LM head + unmask
+def lmhead_unmask_args(x, w, tokens, is_masked, n_committed, n_masked, *, gamma: float,
+                       inv_temperature: float = 1.0, mask_token_id: int = 3, exclude_mask_token: bool = False,
+                       remaining_steps: int = 0, conf=None, argmax=None,
+                       keep_masked: Optional[int] = None) -> LmheadUnmaskArgs:
+    B, S, D = x.shape
+    a = LmheadUnmaskArgs()
+    a.batch, a.block_size, a.hidden, a.vocab, a.dtype = B, S, D, int(w.shape[0]), _dtype_code(x.dtype)
+    a.x, a.w = _ptr(x), _ptr(w)
+    a.gamma, a.inv_temperature = float(gamma), float(inv_temperature)
+    a.mask_token_id, a.exclude_mask_token, a.remaining_steps = int(mask_token_id), int(bool(exclude_mask_token)), int(remaining_steps)
+    a.tokens, a.is_masked, a.conf, a.argmax = _ptr(tokens), _ptr(is_masked), _ptr(conf), _ptr(argmax)
+    a.n_committed, a.n_masked = _ptr(n_committed), _ptr(n_masked)
+    if keep_masked is None:
+        a.sampler, a.keep_masked = TT_SAMPLER_CONFIDENCE, 0
+    else:
+        a.sampler, a.keep_masked = TT_SAMPLER_PREDICT_NOISE, int(keep_masked)
+    return a
+
+
+def tt_lmhead_unmask_workspace_bytes(args: LmheadUnmaskArgs) -> int:
+    return int(lib().tt_lmhead_unmask_workspace_bytes(ctypes.byref(args)))
+
+
+def tt_lmhead_unmask_step(args: LmheadUnmaskArgs, workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().tt_lmhead_unmask_step(ctypes.byref(args), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tt_lmhead_unmask_step")
 
 
 # ------------------------------------------------------------------------------------ block commit

@@ -83,6 +83,19 @@ static int validate_adaln(const tt_adaln_args_t* a) {
   }
 }
 
+static int validate_lmhead(const tt_lmhead_unmask_args_t* a) {
+  if (!a) return TT_ERR_INVALID_ARGUMENT;
+  if (a->batch < 1 || a->block_size < 1 || a->hidden < 1 || a->vocab < 1) return TT_ERR_INVALID_ARGUMENT;
+  if (!a->x || !a->w || !a->tokens || !a->is_masked || !a->n_committed || !a->n_masked) return TT_ERR_INVALID_ARGUMENT;
+  if (!(a->inv_temperature > 0.f)) return TT_ERR_INVALID_ARGUMENT;
+  if (a->sampler != TT_SAMPLER_CONFIDENCE && a->sampler != TT_SAMPLER_PREDICT_NOISE) return TT_ERR_INVALID_ARGUMENT;
+  if (a->sampler == TT_SAMPLER_PREDICT_NOISE && a->keep_masked < 0) return TT_ERR_INVALID_ARGUMENT;
+  if (a->dtype != TT_BF16) return TT_ERR_UNSUPPORTED;
+  if (a->hidden % 64 != 0 || a->vocab % 128 != 0 || a->block_size > 1024) return TT_ERR_UNSUPPORTED;
+  if (!aligned16(a->x) || !aligned16(a->w)) return TT_ERR_UNSUPPORTED;
+  return TT_OK;
+}
+
 static int validate_kv_append(const tt_kv_append_args_t* a) {
   if (!a) return TT_ERR_INVALID_ARGUMENT;
   if (a->batch < 1 || a->block_size < 1 || a->num_kv_heads < 1 || a->head_dim < 1) return TT_ERR_INVALID_ARGUMENT;
@@ -177,6 +190,18 @@ int tt_unmask_step_noalloc(const tt_unmask_args_t* a, tt_stream_t stream) {
 int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, tt_stream_t stream) {
   if (!is_masked || !tau || batch < 1 || block_size < 1) return TT_ERR_INVALID_ARGUMENT;
   return block_tau_launch(is_masked, batch, block_size, tau, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tt_lmhead_unmask_workspace_bytes(const tt_lmhead_unmask_args_t* a) {
+  return validate_lmhead(a) == TT_OK ? lmhead_workspace_bytes(a, device_sm_count()) : 0;
+}
+
+int tt_lmhead_unmask_step(const tt_lmhead_unmask_args_t* a, void* ws, size_t ws_bytes, tt_stream_t stream) {
+  const int st = validate_lmhead(a);
+  if (st != TT_OK) return st;
+  if (!ws) return TT_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < lmhead_workspace_bytes(a, device_sm_count())) return TT_ERR_WORKSPACE_TOO_SMALL;
+  return lmhead_unmask_launch(a, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t tt_kv_append_workspace_bytes(const tt_kv_append_args_t* a) {

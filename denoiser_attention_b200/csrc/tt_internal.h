@@ -21,6 +21,9 @@ UnmaskPlan unmask_plan(const tt_unmask_args_t* a, int num_sms);
 int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& plan, void* ws, cudaStream_t stream);
 // Same launch with the module's static scratch (no allocation, no caller workspace).
 int unmask_launch_static(const tt_unmask_args_t* a, cudaStream_t stream);
+// The unmask step from hidden states through the LM head (logits never stored).
+size_t lmhead_workspace_bytes(const tt_lmhead_unmask_args_t* a, int num_sms);
+int lmhead_unmask_launch(const tt_lmhead_unmask_args_t* a, void* ws, cudaStream_t stream);
 // tau[b] = masked positions of sequence b / S.
 int block_tau_launch(const uint8_t* is_masked, int B, int S, float* tau, cudaStream_t stream);
 

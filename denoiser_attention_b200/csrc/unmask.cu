@@ -18,6 +18,8 @@
 #include <cstdio>
 #include <algorithm>
 #include <mutex>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "tt_common.cuh"
 #include "tt_internal.h"
@@ -351,6 +353,362 @@ int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cud
   else
     launch_pdl(unmask_kernel<float>, dim3(pl.grid), dim3(kUnmaskThreads), 0, stream, p);
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- fused LM head + unmask
+// The same step from the hidden states instead of the logits: logits = x W^T (x [B*S][D] the
+// final hidden states, W [V][D] the LM-head weight) are formed tile by tile on the tensor cores
+// and reduced to (max, sum exp, argmax) in the epilogue, so the [B*S][V] logits never reach
+// memory. A CTA owns one 128-row tile of x (M tile) and a contiguous range of 128-column
+// vocabulary tiles; per vocabulary tile it runs the K loop over D in 64-wide stages (both
+// operands K-major, 128B-swizzled, brought in by TMA without multicast) into one of two TMEM
+// accumulators, while its epilogue warps reduce the other. The per-range partial states of a row
+// are merged by the last CTA of the M tile to finish (ticket), which then applies the commit rule
+// (either sampler) to every sequence whose rows are all merged.
+namespace {
+
+constexpr int kLmThreads = 192;                       // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kLmStages = 6;
+constexpr uint32_t kLmBox = 128 * 128;                // 128 rows x 64 bf16 = 16 KB
+constexpr uint32_t kLmStageBytes = 2 * kLmBox;        // x box + W box
+constexpr uint32_t kLmTiles = kLmStages * kLmStageBytes;   // 192 KB
+constexpr uint32_t kLmSmem = kLmTiles + 2048 + 1024;  // barriers / lists + alignment slack
+constexpr uint32_t kLmTmemCols = 256;                 // two 128-column accumulators
+constexpr uint32_t kLmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+struct LmParams {
+  CUtensorMap tm_x, tm_w;
+  UnmaskParams u;                 // commit rule, outputs, workspace offsets of conf / argmax / sequence tickets
+  int32_t M, D, V, nvr, vtiles;
+  size_t off_parts, off_mt_cnt;
+};
+
+struct LmSmem {
+  uint64_t full[kLmStages], empty[kLmStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int last_flag;
+  int n_commit;
+  int commit_list[128];
+};
+
+__device__ __forceinline__ uint64_t lm_sdesc(uint32_t saddr) {
+  // K-major, 128B swizzle: 8-row groups 1024 bytes apart
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) |
+         ((uint64_t)2 << 61);
+}
+
+__global__ void __launch_bounds__(kLmThreads, 1) lmhead_unmask_kernel(const __grid_constant__ LmParams p) {
+  extern __shared__ __align__(1024) uint8_t lm_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lm_raw) + 1023) & ~uintptr_t(1023));
+  LmSmem& sm = *reinterpret_cast<LmSmem*>(tiles + kLmTiles);
+  const UnmaskParams& u = p.u;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(u.ws);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mt = blockIdx.x / p.nvr, vr = blockIdx.x % p.nvr;
+  const int t0 = (int)((long long)vr * p.vtiles / p.nvr), t1 = (int)((long long)(vr + 1) * p.vtiles / p.nvr);
+  const int ntile = t1 - t0, nk = p.D / 64;
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kLmStages; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.acc_full[i], 1);
+      mbar_init(&sm.acc_empty[i], 128);
+    }
+    mbar_init(&sm.drain, 1);
+    fence_barrier_init();
+    prefetch_tmap(&p.tm_x);
+    prefetch_tmap(&p.tm_w);
+    sm.abort_flag = 0;
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kLmTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  pdl_trigger();
+  pdl_wait();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  auto fail = [&](uint32_t detail) {
+    report_error(hdr, TT_ERR_DEVICE_TIMEOUT, detail);
+    *abort_flag = 1;
+  };
+  const uint32_t tiles_s = smem_u32(tiles);
+
+  if (warp == 0) {
+    // ======================= TMA producer: (x box, W box) per 64-wide K step
+    if (lane == 0) {
+      long long it = 0;
+      bool ok = true;
+      for (int n = 0; n < ntile && ok; ++n) {
+        for (int ks = 0; ks < nk; ++ks, ++it) {
+          const int stage = (int)(it % kLmStages);
+          const uint32_t round = (uint32_t)(it / kLmStages);
+          if (round > 0 && !mbar_wait_bounded(&sm.empty[stage], (round - 1) & 1, abort_flag)) {
+            fail(kDetailWaitKvEmpty);
+            ok = false;
+            break;
+          }
+          uint8_t* dst = tiles + stage * kLmStageBytes;
+          mbar_arrive_expect_tx(&sm.full[stage], kLmStageBytes);
+          tma_load_3d(dst, &p.tm_x, &sm.full[stage], ks * 64, 0, mt * 128);
+          tma_load_3d(dst + kLmBox, &p.tm_w, &sm.full[stage], ks * 64, 0, (t0 + n) * 128);
+        }
+      }
+      for (long long j = (it > kLmStages ? it - kLmStages : 0); j < it; ++j) {
+        const uint64_t tw = globaltimer_ns();
+        while (!mbar_try_wait(&sm.full[j % kLmStages], (uint32_t)((j / kLmStages) & 1)) &&
+               globaltimer_ns() - tw < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer: acc[n % 2] = x_tile W_tile^T over D
+    if (lane == 0) {
+      long long it = 0;
+      bool ok = true;
+      for (int n = 0; n < ntile && ok; ++n) {
+        const int acc = n & 1;
+        if (n >= 2 && !mbar_wait_bounded(&sm.acc_empty[acc], (uint32_t)(((n - 2) >> 1) & 1), abort_flag)) {
+          fail(kDetailWaitPvDone);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tm = tmem + 128u * (uint32_t)acc;
+        for (int ks = 0; ks < nk; ++ks, ++it) {
+          const int stage = (int)(it % kLmStages);
+          if (!mbar_wait_bounded(&sm.full[stage], (uint32_t)((it / kLmStages) & 1), abort_flag)) {
+            fail(kDetailWaitKvFull);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = lm_sdesc(tiles_s + stage * kLmStageBytes);
+          const uint64_t db = lm_sdesc(tiles_s + stage * kLmStageBytes + kLmBox);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(d_tm, da + (uint64_t)((kk * 32) >> 4), db + (uint64_t)((kk * 32) >> 4), kLmIdesc,
+                   (ks > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&sm.empty[stage]);
+        }
+        if (ok) tc_commit(&sm.acc_full[acc]);
+      }
+    }
+  } else {
+    // ======================= epilogue: thread = row (TMEM lane), running (max, sum exp, argmax)
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float c = u.c;
+    float m = -INFINITY, s = 0.f;
+    int32_t idx = 0x7fffffff;
+    for (int n = 0; n < ntile; ++n) {
+      const int acc = n & 1;
+      if (!mbar_wait_bounded(&sm.acc_full[acc], (uint32_t)((n >> 1) & 1), abort_flag)) {
+        fail(kDetailWaitSFull);
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      uint32_t v[128];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tmem_ld32(tmem + lane_off + 128u * (uint32_t)acc + 32u * (uint32_t)q, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&sm.acc_empty[acc]);   // the accumulator can take tile n + 2
+      const int vbase = (t0 + n) * 128;
+      if (u.exclude_mask_token) {
+        const int e = u.mask_token_id - vbase;
+#pragma unroll
+        for (int j = 0; j < 128; ++j)   // static indices keep v[] in registers
+          if (j == e) v[j] = __float_as_uint(-INFINITY);
+      }
+      float tmax = __uint_as_float(v[0]);
+      int targ = 0;
+#pragma unroll
+      for (int j = 1; j < 128; ++j) {
+        if (__uint_as_float(v[j]) > tmax) {
+          tmax = __uint_as_float(v[j]);
+          targ = j;
+        }
+      }
+      const float nm = fmaxf(m, tmax);
+      float ts = 0.f;
+#pragma unroll
+      for (int j = 0; j < 128; ++j) ts += ex2(c * (__uint_as_float(v[j]) - nm));
+      s = ((m == -INFINITY) ? 0.f : s * ex2(c * (m - nm))) + ts;
+      if (tmax > m) idx = vbase + targ;   // strictly larger: an earlier tile keeps ties
+      m = nm;
+    }
+    UnmaskPartial* parts = reinterpret_cast<UnmaskPartial*>(u.ws + p.off_parts);
+    parts[((size_t)mt * p.nvr + vr) * 128 + r] = UnmaskPartial{m, s, idx, 0};
+  }
+
+  // ---- teardown of the tile phase: MMAs drained, TMEM released
+  if (warp == 1 && lane == 0) {
+    tc_commit(&sm.drain);
+    const uint64_t tw = globaltimer_ns();
+    while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - tw < kWaitLimitNs) {
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kLmTmemCols);
+  }
+  if (*abort_flag) return;   // uniform: read after the barrier
+
+  // ---- the last CTA of this M tile merges its rows' partial states and commits finished sequences
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    int* mt_cnt = reinterpret_cast<int*>(u.ws + p.off_mt_cnt);
+    const int old = atomicAdd(mt_cnt + mt, 1);
+    sm.last_flag = (old == p.nvr - 1) ? 1 : 0;
+    if (sm.last_flag) mt_cnt[mt] = 0;
+    sm.n_commit = 0;
+  }
+  __syncthreads();
+  if (!sm.last_flag) return;
+  __threadfence();
+  float* conf_ws = reinterpret_cast<float*>(u.ws + u.off_conf);
+  int32_t* arg_ws = reinterpret_cast<int32_t*>(u.ws + u.off_argmax);
+  int* seq_cnt = reinterpret_cast<int*>(u.ws + u.off_seq_cnt);
+  const float4* pp = reinterpret_cast<const float4*>(u.ws + p.off_parts);
+  if (tid < 128) {
+    const int row = mt * 128 + tid;
+    if (row < p.M) {
+      float4 q = __ldcg(pp + (size_t)mt * p.nvr * 128 + tid);
+      RedState st{q.x, q.y, __float_as_int(q.z)};
+      for (int k = 1; k < p.nvr; ++k) {
+        q = __ldcg(pp + ((size_t)mt * p.nvr + k) * 128 + tid);
+        st = red_combine(st, RedState{q.x, q.y, __float_as_int(q.z)}, u.c);
+      }
+      const float conf = 1.0f / st.s;
+      conf_ws[row] = conf;
+      arg_ws[row] = st.idx;
+      if (u.conf_out) u.conf_out[row] = conf;
+      if (u.argmax_out) u.argmax_out[row] = st.idx;
+      __threadfence();
+      const int b = row / u.block_size;
+      const int old = atomicAdd(seq_cnt + b, 1);
+      if (old == u.block_size - 1) {
+        seq_cnt[b] = 0;
+        __threadfence();
+        sm.commit_list[atomicAdd(&sm.n_commit, 1)] = b;
+      }
+    }
+  }
+  __syncthreads();
+  const int nc = sm.n_commit;
+  for (int i = 0; i < nc; ++i) {
+    commit_sequence(u, sm.commit_list[i], conf_ws, arg_ws);
+    __syncthreads();   // commit_sequence reuses its shared counters
+  }
+}
+
+// 3-D bf16 map (D [contiguous], 1, rows), box (64, 1, 128), 128B swizzle.
+bool lm_make_map(CUtensorMap* m, const void* base, int D, long long rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  const cuuint64_t dims[3] = {(cuuint64_t)D, 1, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct LmLayout {
+  int n_mt, nvr;
+  size_t parts, mt_cnt, seq_cnt, conf, argmax, total;
+};
+
+LmLayout lm_layout(const tt_lmhead_unmask_args_t* a, int num_sms) {
+  LmLayout L{};
+  const int M = a->batch * a->block_size;
+  L.n_mt = (M + 127) / 128;
+  L.nvr = std::max(1, std::min(a->vocab / 128, std::max(1, num_sms) / L.n_mt));
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return o;
+  };
+  L.parts = take(sizeof(UnmaskPartial) * (size_t)L.n_mt * L.nvr * 128);
+  L.mt_cnt = take(sizeof(int) * (size_t)L.n_mt);
+  L.seq_cnt = take(sizeof(int) * (size_t)a->batch);
+  L.conf = take(sizeof(float) * (size_t)M);
+  L.argmax = take(sizeof(int32_t) * (size_t)M);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+size_t lmhead_workspace_bytes(const tt_lmhead_unmask_args_t* a, int num_sms) { return lm_layout(a, num_sms).total; }
+
+int lmhead_unmask_launch(const tt_lmhead_unmask_args_t* a, void* ws, cudaStream_t stream) {
+  const LmLayout L = lm_layout(a, device_sm_count());
+  LmParams p{};
+  const int M = a->batch * a->block_size;
+  if (!lm_make_map(&p.tm_x, a->x, a->hidden, M)) return TT_ERR_CUDA;
+  if (!lm_make_map(&p.tm_w, a->w, a->hidden, a->vocab)) return TT_ERR_CUDA;
+  UnmaskParams& u = p.u;
+  u.block_size = a->block_size;
+  u.rows = M;
+  u.c = a->inv_temperature * 1.4426950408889634f;
+  u.gamma = a->gamma;
+  u.mask_token_id = a->mask_token_id;
+  u.exclude_mask_token = a->exclude_mask_token;
+  u.remaining_steps = a->remaining_steps;
+  u.sampler = a->sampler;
+  u.keep_masked = a->keep_masked;
+  u.tokens = a->tokens;
+  u.is_masked = a->is_masked;
+  u.conf_out = a->conf;
+  u.argmax_out = a->argmax;
+  u.n_committed = a->n_committed;
+  u.n_masked = a->n_masked;
+  u.ws = static_cast<uint8_t*>(ws);
+  u.off_seq_cnt = L.seq_cnt;
+  u.off_conf = L.conf;
+  u.off_argmax = L.argmax;
+  p.M = M;
+  p.D = a->hidden;
+  p.V = a->vocab;
+  p.nvr = L.nvr;
+  p.vtiles = a->vocab / 128;
+  p.off_parts = L.parts;
+  p.off_mt_cnt = L.mt_cnt;
+  static unsigned long long attr_done = 0;   // bit per device ordinal (< 64)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(lmhead_unmask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLmSmem) !=
+        cudaSuccess)
+      return TT_ERR_CUDA;
+    __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+  }
+  return launch_pdl(lmhead_unmask_kernel, dim3(L.n_mt * L.nvr), dim3(kLmThreads), kLmSmem, stream, p) == cudaSuccess
+             ? TT_OK
+             : TT_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- no-allocation variant

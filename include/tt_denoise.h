@@ -10,6 +10,7 @@
  *   tt_unmask_step     confidence-threshold unmasking, the paper §2.2 "Sampling", Algorithm 2
  *   tt_block_tau       the step's time input from the mask, Algorithm 2 line 3
  *   tt_kv_append       block commit into the paged context cache, Algorithm 1 line 8
+ *   tt_lmhead_unmask_step  the unmask step from hidden states (LM head fused, logits never stored)
  *
  * Conventions shared by every entry point
  *   - Every pointer named in an args struct is a DEVICE pointer (cudaMalloc'd or equivalent)
@@ -247,6 +248,45 @@ int tt_unmask_step(const tt_unmask_args_t* args, void* workspace, size_t workspa
  *   - The kernel sets no device error word; tt_get_device_error does not apply.
  * ------------------------------------------------------------------------------------------- */
 int tt_unmask_step_noalloc(const tt_unmask_args_t* args, tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * tt_lmhead_unmask_step: the unmask step (either sampler, same rule and outputs as
+ * tt_unmask_step) computed from the final hidden states instead of the logits, the paper §2.2:
+ * the denoiser's LM head produces p_theta = softmax(x W^T) for every block position, and here the
+ * logits x W^T are reduced to (confidence, argmax) tile by tile on the tensor cores without ever
+ * being written to memory.
+ *   x   device bf16 [batch][block_size][hidden]   (hidden states after the final norm)
+ *   w   device bf16 [vocab][hidden]                (LM-head weight)
+ *   the remaining fields as in tt_unmask_args_t (logits replaced by x and w; conf / argmax are
+ *   optional outputs). Logits are accumulated in fp32.
+ * Supported: TT_BF16; hidden a multiple of 64; vocab a multiple of 128; block_size <= 1024; x and
+ * w 16-byte aligned (else TT_ERR_UNSUPPORTED). Workspace: tt_lmhead_unmask_workspace_bytes(),
+ * zero-filled before first use; the kernel returns its tickets to zero, so it can be reused by
+ * calls with the same sizes.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct {
+  int32_t batch, block_size, hidden, vocab;
+  int32_t dtype;
+  const void* x;
+  const void* w;
+  float gamma;
+  float inv_temperature;
+  int32_t mask_token_id;
+  int32_t exclude_mask_token;
+  int32_t remaining_steps;
+  int32_t* tokens;
+  uint8_t* is_masked;
+  float* conf;
+  int32_t* argmax;
+  int32_t* n_committed;
+  int32_t* n_masked;
+  int32_t sampler;
+  int32_t keep_masked;
+} tt_lmhead_unmask_args_t;
+
+size_t tt_lmhead_unmask_workspace_bytes(const tt_lmhead_unmask_args_t* args);
+int tt_lmhead_unmask_step(const tt_lmhead_unmask_args_t* args, void* workspace, size_t workspace_bytes,
+                          tt_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * tt_kv_append: block commit into the paged context cache, the paper §2.2 Algorithm 1 line 8

@@ -18,6 +18,7 @@ Source: "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Conte
   confidence_commit      the paper §2.2 "Sampling" and Algorithm 2 (ConfidenceSample)
   refine_block           the paper Algorithm 2 (single-block confidence unmasking loop)
   predict_noise_step     the predict-and-noise sampler (§2.2 "Sampling"), linear schedule
+  lmhead_logits          the denoiser's LM head: logits = x W^T (feeds either sampler)
   append_block           the paper Algorithm 1 line 8 (the committed block joins the context)
 
 Readings of points the paper leaves open (each is also listed in the design notes):
@@ -263,6 +264,14 @@ def predict_noise_step(tokens, is_masked, logits, keep_masked: int, inv_temperat
 def linear_schedule_keep(block_size: int, steps: int, r: int) -> int:
     """Masked positions left after step r of T under alpha_t = 1 - t (masked fraction t = (T-r)/T)."""
     return (block_size * (steps - r)) // steps
+
+
+def lmhead_logits(x, w) -> np.ndarray:
+    """The denoiser's LM head (the paper §2.2: p_theta over the vocabulary for every block
+    position): logits[b][l][v] = sum_d x[b][l][d] w[v][d], in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    return np.einsum("bld,vd->blv", x, w)
 
 
 def refine_block(batch: int, block_size: int, steps: int, gamma: float,

@@ -204,3 +204,23 @@ def test_unmask_sampler_fields_validated(lib):
     assert lib.tt_unmask_workspace_bytes(ctypes.byref(a)) == 0
     a.keep_masked = 4
     assert lib.tt_unmask_workspace_bytes(ctypes.byref(a)) > 0
+
+
+def test_lmhead_host_validation(lib):
+    from denoiser_attention_b200 import binding as Bd
+    a = Bd.LmheadUnmaskArgs()
+    a.batch, a.block_size, a.hidden, a.vocab, a.dtype = 2, 16, 256, 4096, Bd.TT_BF16
+    for name in ("x", "w", "tokens", "is_masked", "n_committed", "n_masked"):
+        setattr(a, name, 0x1000)
+    a.gamma, a.inv_temperature = 0.8, 1.0
+    assert lib.tt_lmhead_unmask_workspace_bytes(ctypes.byref(a)) > 256
+    ws = ctypes.c_void_p(0x2000)
+    for field, bad, status in (("hidden", 100, Bd.TT_ERR_UNSUPPORTED), ("vocab", 1000, Bd.TT_ERR_UNSUPPORTED),
+                               ("dtype", Bd.TT_F32, Bd.TT_ERR_UNSUPPORTED), ("x", None, Bd.TT_ERR_INVALID_ARGUMENT),
+                               ("inv_temperature", 0.0, Bd.TT_ERR_INVALID_ARGUMENT),
+                               ("sampler", 5, Bd.TT_ERR_INVALID_ARGUMENT)):
+        good = getattr(a, field)
+        setattr(a, field, bad)
+        assert lib.tt_lmhead_unmask_step(ctypes.byref(a), ws, 1 << 20, None) == status, field
+        setattr(a, field, good)
+    assert lib.tt_lmhead_unmask_step(ctypes.byref(a), ws, 64, None) == Bd.TT_ERR_WORKSPACE_TOO_SMALL

@@ -552,3 +552,19 @@ def test_predict_noise_linear_schedule_finishes_at_T():
         left.append(int(masked[0].sum()))
     # the masked fraction after step r is (T - r) / T of the block, rounded down; none left at T
     assert left == [(S * (T - r)) // T for r in range(1, T + 1)] and left[-1] == 0
+
+
+# ---------------------------------------------------------------- LM head
+def test_lmhead_logits_pins():
+    rs = np.random.default_rng(31)
+    x, w = rs.standard_normal((2, 3, 8)), rs.standard_normal((5, 8))
+    lg = O.lmhead_logits(x, w)
+    # a matrix product written out as nested sums
+    for b in range(2):
+        for l in range(3):
+            for v in range(5):
+                assert abs(lg[b, l, v] - sum(x[b, l, d] * w[v, d] for d in range(8))) < 1e-12
+    # one-hot hidden state picks a column of W; scaling x scales the logits
+    e = np.zeros((1, 1, 8)); e[0, 0, 3] = 1.0
+    np.testing.assert_array_equal(O.lmhead_logits(e, w)[0, 0], w[:, 3])
+    np.testing.assert_allclose(O.lmhead_logits(2 * x, w), 2 * lg, rtol=0, atol=1e-12)
