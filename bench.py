@@ -471,8 +471,17 @@ def run_kernel_only(args):
     tau, h, f = ad.tau.to(dev), ad.h.to(dev), ad.f.to(dev)
     out = torch.empty_like(q)
 
+    if args.kernel == "lmhead":
+        # the fused LM head + unmask at the decode shape: hidden states [8][16][2048], W [131072][2048]
+        gen = torch.Generator(device=dev).manual_seed(w.seed)
+        D, Vh = 2048, 131072
+        xh = torch.randn((B, S, D), device=dev, generator=gen).to(torch.bfloat16)
+        wh = (torch.randn((Vh, D), device=dev, generator=gen) * (3.0 / D ** 0.5)).to(torch.bfloat16)
+
     def once():
-        if args.kernel == "attn":
+        if args.kernel == "lmhead":
+            api.lmhead_unmask_step(xh, wh, tokens, masked, gamma=w.gamma, want_conf=False)
+        elif args.kernel == "attn":
             api.denoise_attention(q, kb, vb, kc, vc, lens, page_table=table, page_size=w.attn.page_size,
                                   ctx_stride=inp.ctx_stride, out=out)
         elif args.kernel == "unmask":
@@ -502,7 +511,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--kernel", choices=["attn", "unmask", "adaln"], default=None,
+    ap.add_argument("--kernel", choices=["attn", "unmask", "adaln", "lmhead"], default=None,
                     help="profiling mode: eager launches of one kernel only (not a bench line)")
     ap.add_argument("--workload", default=WORKLOAD, help="workload of the --kernel profiling mode")
     args = ap.parse_args()

@@ -585,11 +585,18 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_unmask_kernel(const __gr
   if (tid < 128) {
     const int row = mt * 128 + tid;
     if (row < p.M) {
-      float4 q = __ldcg(pp + (size_t)mt * p.nvr * 128 + tid);
-      RedState st{q.x, q.y, __float_as_int(q.z)};
-      for (int k = 1; k < p.nvr; ++k) {
-        q = __ldcg(pp + ((size_t)mt * p.nvr + k) * 128 + tid);
-        st = red_combine(st, RedState{q.x, q.y, __float_as_int(q.z)}, u.c);
+      // the row's nvr partial states, loaded 16 at a time (independent loads in flight) and
+      // combined in range order, so ties still resolve to the lowest token id
+      const float4* base = pp + (size_t)mt * p.nvr * 128 + tid;
+      RedState st{-INFINITY, 0.f, 0x7fffffff};
+      for (int k0 = 0; k0 < p.nvr; k0 += 16) {
+        float4 q[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (k0 + j < p.nvr) q[j] = __ldcg(base + (size_t)(k0 + j) * 128);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (k0 + j < p.nvr) st = red_combine(st, RedState{q[j].x, q[j].y, __float_as_int(q[j].z)}, u.c);
       }
       const float conf = 1.0f / st.s;
       conf_ws[row] = conf;
