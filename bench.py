@@ -153,7 +153,7 @@ def host_inputs(w, seed_offset: int = 0):
     from denoiser_attention_b200 import synth
     inp = synth.attention_inputs(w.attn, seed=w.seed + seed_offset)
     B, S = w.attn.batch, w.attn.block_size
-    tau = [1.0] * B   # first refinement step: the whole block is masked (Algorithm 2, line 3)
+    tau = [1.0] * B   # first refinement step: the whole block is masked (Algorithm 2's time input)
     ad = synth.adaln_inputs(B, S, w.hidden, tau, seed=w.seed + 100 + seed_offset, dtype=w.attn.dtype)
     logits = synth.workload_logits(w, seed=w.seed + seed_offset)
     return inp, ad, logits

@@ -8,7 +8,7 @@ kernels. Workspaces are cached per (device, size) and zero-filled once, as the A
     adaln_cond           adaLN-single: tau -> (shift, scale, gate)       (tt_adaln_modulate)
     adaln_norm_modulate  modulated RMSNorm prologue                      (tt_adaln_modulate)
     adaln_gated_residual h + gate * f                                    (tt_adaln_modulate)
-    unmask_step          ConfidenceSample, Algorithm 2 line 5            (tt_unmask_step)
+    unmask_step          ConfidenceSample, Algorithm 2 (its ConfidenceSample step)            (tt_unmask_step)
                          or the predict-and-noise sampler (keep_masked)
     RefinementStep       the whole step a2..a7 (three concurrent branches), device buffers
     HostStep             the same step from pinned host buffers (copies included)
@@ -175,7 +175,7 @@ class StepBuffers:
 class RefinementStep:
     """One denoiser refinement step of TwoTower decoding on one GPU.
 
-    a2  mod = adaLN-single(tau)                 (tau = masked fraction, Algorithm 2 line 3)
+    a2  mod = adaLN-single(tau)                 (tau = masked fraction: the time input of Algorithm 2)
     a3  y = modulated RMSNorm(h)                (prologue; y feeds the out-of-scope QKV projection)
     a4  O = Eq. (1) attention(q, [K_ctx; K_blk], [V_ctx; V_blk])
     a5  h' = h + gate * f                       (f: the mixer output after its out-projection)
@@ -261,7 +261,7 @@ class RefinementStep:
 
 
 def block_tau(is_masked: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """tau[b] = |{l : is_masked[b, l]}| / S on the device (Algorithm 2 line 3)."""
+    """tau[b] = |{l : is_masked[b, l]}| / S on the device (the time input of Algorithm 2)."""
     tau = torch.empty(is_masked.shape[0], dtype=torch.float32, device=is_masked.device) if out is None else out
     B.tt_block_tau(is_masked, tau)
     return tau

@@ -1,5 +1,5 @@
-// Block commit into the paged context cache: Algorithm 1 line 8 of "Nemotron-TwoTower: Diffusion
-// Language Modeling with Pretrained AR Context" (§2.2 "Sampling"): once block b is committed, the
+// Block commit into the paged context cache: the context update of Algorithm 1 in "Nemotron-TwoTower:
+// Diffusion Language Modeling with Pretrained AR Context" (§2.2 "Sampling"): once block b is committed, the
 // context tower's KV of its S tokens joins the prefix cache that the next block's denoiser
 // attention reads. The context tower itself (which produces that KV) is not part of this path;
 // this kernel appends the rows it produced and grows the page tables.

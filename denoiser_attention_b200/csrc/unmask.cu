@@ -1,4 +1,4 @@
-// ConfidenceSample on sm_100a: the paper §2.2 "Sampling" and Algorithm 2 line 5 of
+// ConfidenceSample on sm_100a: the paper §2.2 "Sampling" and Algorithm 2 (its ConfidenceSample step) of
 // "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Context".
 //
 // One pass over the vocabulary logits computes, per block position, the softmax maximum
@@ -769,7 +769,7 @@ int unmask_launch_static(const tt_unmask_args_t* a, cudaStream_t stream) {
   return unmask_launch(a, pl, ws, stream);
 }
 
-// ---------------------------------------------------------------- Algorithm 2 line 3
+// ---------------------------------------------------------------- Algorithm 2: the time input
 // tau_b = |{l : position l of sequence b is masked}| / S, one warp per sequence, so a multi-step
 // refinement loop can feed the next step's time input from the mask on the device.
 constexpr int kTauThreads = 128;

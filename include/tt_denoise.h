@@ -8,8 +8,8 @@
  *   tt_denoise_attn    layer-aligned denoiser attention, the paper §2.1 Eq. (1)
  *   tt_adaln_modulate  adaLN-single time conditioning, the paper §2.1 "Time conditioning"
  *   tt_unmask_step     confidence-threshold unmasking, the paper §2.2 "Sampling", Algorithm 2
- *   tt_block_tau       the step's time input from the mask, Algorithm 2 line 3
- *   tt_kv_append       block commit into the paged context cache, Algorithm 1 line 8
+ *   tt_block_tau       the step's time input from the mask, Algorithm 2 (its time input, the masked fraction)
+ *   tt_kv_append       block commit into the paged context cache, Algorithm 1 (context update)
  *   tt_lmhead_unmask_step  the unmask step from hidden states (LM head fused, logits never stored)
  *
  * Conventions shared by every entry point
@@ -177,7 +177,7 @@ typedef enum {
 } tt_sampler_t;
 
 /* ---------------------------------------------------------------------------------------------
- * ConfidenceSample, the paper §2.2 "Sampling" and Algorithm 2 line 5: the denoiser predicts
+ * ConfidenceSample, the paper §2.2 "Sampling" and Algorithm 2: the denoiser predicts
  * every masked position in parallel; predictions whose confidence reaches gamma are committed,
  * the rest stay masked for later steps.
  *   conf[b][l]   = max_v softmax(inv_temperature * logits[b][l])_v
@@ -289,7 +289,8 @@ int tt_lmhead_unmask_step(const tt_lmhead_unmask_args_t* args, void* workspace, 
                           tt_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
- * tt_kv_append: block commit into the paged context cache, the paper §2.2 Algorithm 1 line 8
+ * tt_kv_append: block commit into the paged context cache, the paper §2.2, Algorithm 1 (the
+ * context update once a block is committed)
  * ("update the AR context" once block b is committed): the context tower's K and V for the S
  * tokens of the committed block are appended after each sequence's current context, taking new
  * pages from a free-page stack as needed. The context tower that produces k_new / v_new is not
@@ -332,7 +333,8 @@ size_t tt_kv_append_workspace_bytes(const tt_kv_append_args_t* args);
 int tt_kv_append(const tt_kv_append_args_t* args, void* workspace, size_t workspace_bytes, tt_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
- * tt_block_tau: the time input of one refinement step, the paper §2.2 Algorithm 2 line 3:
+ * tt_block_tau: the time input of one refinement step, the paper §2.2, Algorithm 2 (the masked
+ * fraction of the block):
  * tau_b = |{l : z_l = [MASK]}| / S, computed on the device from the mask so that a multi-step
  * loop (captured in one CUDA graph) needs no host round trip between steps.
  *   is_masked  device u8 [batch][block_size], 1 = still masked

@@ -19,7 +19,7 @@ Source: "Nemotron-TwoTower: Diffusion Language Modeling with Pretrained AR Conte
   refine_block           the paper Algorithm 2 (single-block confidence unmasking loop)
   predict_noise_step     the predict-and-noise sampler (§2.2 "Sampling"), linear schedule
   lmhead_logits          the denoiser's LM head: logits = x W^T (feeds either sampler)
-  append_block           the paper Algorithm 1 line 8 (the committed block joins the context)
+  append_block           the paper Algorithm 1, context update (the committed block joins the context)
 
 Readings of points the paper leaves open (each is also listed in the design notes):
   * attention mask: every block query sees all L_b context keys and all S block keys; the only
@@ -300,7 +300,7 @@ def refine_block(batch: int, block_size: int, steps: int, gamma: float,
 
 def append_block(ctx_k: Sequence[np.ndarray], ctx_v: Sequence[np.ndarray], k_new: np.ndarray,
                  v_new: np.ndarray):
-    """Algorithm 1 line 8: after block b is committed, the context tower's K/V of its S tokens
+    """The context update of Algorithm 1: after block b is committed, the context tower's K/V of its S tokens
     follow the sequence's existing context. ctx_k[b] / ctx_v[b] are [L_b][Hkv][d] (the logical
     context, e.g. from gather_context); k_new / v_new are [B][S][Hkv][d]. Returns the new
     per-sequence contexts [L_b + S][Hkv][d] and lengths. Storage (pages) is not modelled: a paged

@@ -1,4 +1,4 @@
-"""Block commit into the paged context cache (tt_kv_append, Algorithm 1 line 8) against the
+"""Block commit into the paged context cache (tt_kv_append, the context update of Algorithm 1) against the
 oracle's append_block: the gathered context after the append is bit-exact the old context
 followed by the block; the pages taken are the top of the free stack; the device reports a
 sequence it cannot give pages; attention over the grown cache matches the oracle."""

@@ -433,7 +433,7 @@ def test_commit_brute_force_tiny():
 def test_refinement_loop_closed_behaviour():
     # tiny fp32 workload: logits ~ N(0, 2^2) over 1024 entries give max probability ~0.1 << 0.8,
     # so every step falls back to exactly one commit and the block finishes at r = T = 16 with
-    # tau = 16/16, 15/16, ..., 1/16 (Algorithm 2, line 3).
+    # tau = 16/16, 15/16, ..., 1/16 (Algorithm 2's time input).
     g = json.load(open(os.path.join(GOLDEN, "generation_defaults.json")))
     S, T, mask_id, gamma = g["block_size"], g["steps_per_block"], g["mask_token_id"], g["confidence_threshold"]
     w = synth.workload("tiny_fp32")
@@ -470,7 +470,7 @@ def test_round_bf16_matches_torch():
     assert np.all(np.rint(m * 256) == m * 256)
 
 
-# ---------------------------------------------------------------- block commit (Algorithm 1 line 8)
+# ---------------------------------------------------------------- block commit (Algorithm 1, context update)
 def test_append_block_is_concatenation():
     rs = np.random.default_rng(11)
     lens = [0, 5, 17]
