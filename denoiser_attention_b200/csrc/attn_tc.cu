@@ -6,8 +6,10 @@
 // G query heads of the kv head times the S block positions, packed as rows m = s * G + g and cut
 // into "query tiles" of at most 128 rows (one tcgen05 M=128 MMA). nq = number of query tiles per
 // group. The CTAs are organised in teams of nq; all groups' key tiles are laid end to end and cut
-// into Pe = min(teams, tiles) equal ranges, one per team, computed on the device from ctx_lens
-// (ragged contexts balance to within a tile, with no host knowledge of the lengths). Within a
+// into ranges, one per team, computed on the device from ctx_lens (no host knowledge of the
+// lengths): either Pe = min(teams, tiles) equal ranges (ragged contexts balance to within a tile),
+// or, when that costs at most kSegPenaltyTiles more per team, ranges that never cross a group
+// boundary (each group cut into near-equal chunks), which spares the teams a second segment. Within a
 // team, CTA q handles query tile q of every group its range touches, and the team's CTAs walk the
 // same key tiles at the same time, so each K/V tile comes from HBM once and the other reads of it
 // hit L2. A CTA that holds a whole group writes its rows of the output directly; a group cut
@@ -80,11 +82,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
-// Workspace: header | meta | group_start[groups + 1] | partials | lse
+// Workspace: header | meta | contributors[groups] | partials | lse
 struct AttnMeta {
   long long total_tiles;
   long long p_eff;   // working teams
 };
+
+// A team whose tile range crosses a group boundary runs two segments and pays a second epilogue
+// and pipeline refill, worth about this many tiles of the steady-state loop (measured on the decode
+// workload). The group-aligned partition is taken when its longest range is at most this much
+// above the uniform one's.
+constexpr long long kSegPenaltyTiles = 2;
 
 struct TcParams {
   CUtensorMap tm_q, tm_kc, tm_vc, tm_kb, tm_vb;
@@ -97,7 +105,7 @@ struct TcParams {
   __nv_bfloat16* out;
   float* lse;
   uint8_t* ws;
-  size_t off_meta, off_ustart, off_partials, off_lse;
+  size_t off_meta, off_crange, off_partials, off_lse;
 };
 
 struct Smem {
@@ -176,9 +184,16 @@ struct SegWalk {
   }
 };
 
+// floor(a / b) for 0 <= a, 1 <= b, a + b < 2^53, through one double division (a 64-bit integer
+// division is a long instruction sequence): a and b are exact in double, and a/b = q + r/b lies at
+// least 1/b below q + 1, more than the division's rounding error (q + 1) 2^-53 when (q + 1) b < 2^53.
+__device__ __forceinline__ long long floor_div(long long a, long long b) {
+  return (long long)floor((double)a / (double)b);
+}
+
 // Team owning global tile t when T tiles are cut into P <= T ranges [c*T/P, (c+1)*T/P).
 __device__ __forceinline__ long long owner_team(long long t, long long T, long long P) {
-  return ((t + 1) * P - 1) / T;
+  return floor_div((t + 1) * P - 1, T);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
@@ -223,59 +238,123 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   pdl_trigger();
   pdl_wait();
 
-  // ---- 1. this team's tile range and the group where it starts (warp 0); CTA 0 also records
-  // the partition for the merge kernel
+  // ---- 1. this team's tile range and the group where it starts (warp 0); CTA 0 also records,
+  // per group, the teams that hold its partials (for the merge kernel).
+  // Two partitions of the T tiles (in group order) are considered. Uniform: team c takes
+  // [c*T/P, (c+1)*T/P), which balances tiles but lets ranges cross group boundaries. Group-aligned
+  // (possible when groups <= teams): each group u is cut into ceil(n_u / t) near-equal chunks for
+  // the smallest t with sum_u ceil(n_u / t) <= teams, one chunk per team, so no team runs two
+  // segments. The aligned one is used when t <= ceil(T/P) + kSegPenaltyTiles.
   if (warp == 0) {
+    // 32-bit arithmetic where the values allow it: 64-bit division is a long instruction
+    // sequence, and this warp's chain of them sits before the first load
+    auto wsum = [](uint32_t v) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      return v;
+    };
     long long T = 0;
+    int nmax = 0;
+    int n_first = 0;   // this lane's group in the first 32 (kept: one read of ctx_lens for those)
     for (int base = 0; base < p.groups; base += 32) {
       const int u = base + lane;
       int n = 0;
       if (u < p.groups) n = group_info(p, u, blockIdx.x == 0, hdr).ntiles;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-      T += n;
+      if (base == 0) n_first = n;
+      nmax = max(nmax, n);
+      T += wsum((uint32_t)n);   // a group has fewer than 2^24 tiles (int32 lengths)
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nmax = max(nmax, __shfl_xor_sync(0xffffffffu, nmax, o));
+    auto ntiles_of = [&](int base, int u) -> int {
+      return (u < p.groups) ? (base == 0 ? n_first : group_info(p, u, false, hdr).ntiles) : 0;
+    };
     // with fewer tiles than teams only the first T teams work (one tile each), so every working
     // team owns a non-empty range and the teams of a group are consecutive
-    const long long Pe = T < p.teams ? T : p.teams;
-    const long long rb = team < Pe ? team * T / Pe : T, re = team < Pe ? (team + 1) * T / Pe : T;
-    long long acc = 0;
+    const long long Pu = T < p.teams ? T : p.teams;
+    uint32_t t_al = 0;   // chunk bound of the group-aligned partition; 0 = uniform
+    if (T > 0 && T < (1LL << 31) && p.groups <= p.teams) {
+      const uint32_t T32 = (uint32_t)T, teams32 = (uint32_t)p.teams, Pu32 = (uint32_t)Pu;
+      auto chunks = [&](uint32_t t) -> uint32_t {   // sum over groups of ceil(n_u / t)
+        uint32_t c = 0;
+        for (int base = 0; base < p.groups; base += 32) c += wsum(((uint32_t)ntiles_of(base, base + lane) + t - 1) / t);
+        return c;
+      };
+      uint32_t lo = (T32 - 1) / teams32 + 1;
+      uint32_t hi = (T32 - 1) / Pu32 + 1 + (uint32_t)kSegPenaltyTiles;
+      if (hi > (uint32_t)nmax) hi = (uint32_t)nmax;
+      if (lo <= hi && chunks(hi) <= teams32) {
+        while (lo < hi) {   // chunks(t) does not increase with t
+          const uint32_t mid = (lo + hi) >> 1;
+          if (chunks(mid) <= teams32) hi = mid; else lo = mid + 1;
+        }
+        t_al = lo;
+      }
+    }
+    const bool aligned = t_al > 0;
+    long long rb = T, re = T;
+    if (!aligned && team < Pu) {
+      rb = floor_div(team * T, Pu);
+      re = floor_div((team + 1) * T, Pu);
+    }
+    long long acc = 0, cacc = 0;
     int u0 = -1;
     long long u0s = 0;
-    int32_t* ustart_out = reinterpret_cast<int32_t*>(p.ws + p.off_ustart);
+    int2* crange_out = reinterpret_cast<int2*>(p.ws + p.off_crange);
     const bool record = (blockIdx.x == 0);
     for (int base = 0; base < p.groups && (u0 < 0 || record); base += 32) {
       const int u = base + lane;
-      const int n = (u < p.groups) ? group_info(p, u, false, hdr).ntiles : 0;
-      int incl = n;
+      const int n = ntiles_of(base, u);
+      const int c = aligned ? (int)(((uint32_t)n + t_al - 1) / t_al) : 0;   // chunks (teams) of group u
+      int incl = n, cincl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+        const int z = __shfl_up_sync(0xffffffffu, cincl, o);
+        if (lane >= o) {
+          incl += y;
+          cincl += z;
+        }
       }
-      const long long lo = acc + incl - n, hi = acc + incl;
-      if (record && u < p.groups) ustart_out[u] = (int32_t)lo;
-      const unsigned hit = __ballot_sync(0xffffffffu, u < p.groups && lo <= rb && rb < hi);
+      const long long lo = acc + incl - n, hi = acc + incl;   // tiles of group u
+      const long long c0 = cacc + cincl - c;                  // its first team (aligned)
+      if (record && u < p.groups) {
+        // n >= 1 (the block tile), so hi - 1 >= lo
+        crange_out[u] = aligned ? make_int2((int)c0, (int)(c0 + c - 1))
+                                : make_int2((int)owner_team(lo, T, Pu), (int)owner_team(hi - 1, T, Pu));
+      }
+      const bool mine = u < p.groups && (aligned ? (c0 <= team && team < c0 + c) : (lo <= rb && rb < hi));
+      const unsigned hit = __ballot_sync(0xffffffffu, mine);
       if (hit && u0 < 0) {
         const int src = __ffs(hit) - 1;
         u0 = base + src;
         u0s = __shfl_sync(0xffffffffu, lo, src);
+        const uint32_t nn = (uint32_t)__shfl_sync(0xffffffffu, n, src);
+        const uint32_t cc = (uint32_t)__shfl_sync(0xffffffffu, c, src);
+        const uint32_t j = (uint32_t)(team - __shfl_sync(0xffffffffu, c0, src));
+        if (aligned) {
+          // chunk j covers [j*nn/cc, (j+1)*nn/cc) of the group, from the quotient and remainder
+          // of nn/cc (j*nn may not fit 32 bits; j*r < cc^2 does)
+          const uint32_t q = nn / cc, r = nn - q * cc;
+          rb = u0s + (long long)j * q + (j * r) / cc;
+          re = u0s + (long long)(j + 1) * q + ((j + 1) * r) / cc;
+        }
       }
       acc += __shfl_sync(0xffffffffu, incl, 31);
+      cacc += __shfl_sync(0xffffffffu, cincl, 31);
     }
     if (lane == 0) {
       sm.total_tiles = T;
-      sm.p_eff = Pe;
+      sm.p_eff = aligned ? cacc : Pu;
       sm.range_begin = rb;
       sm.range_end = re;
       sm.u0 = u0;
       sm.u0_start = u0s;
       sm.abort_flag = 0;
       if (record) {
-        ustart_out[p.groups] = (int32_t)T;
         AttnMeta* meta = reinterpret_cast<AttnMeta*>(p.ws + p.off_meta);
         meta->total_tiles = T;
-        meta->p_eff = Pe;
+        meta->p_eff = aligned ? cacc : Pu;
       }
     }
   }
@@ -704,7 +783,7 @@ struct MergeParams {
   __nv_bfloat16* out;
   float* lse;
   const uint8_t* ws;
-  size_t off_meta, off_ustart, off_partials, off_lse;
+  size_t off_meta, off_crange, off_partials, off_lse;
 };
 
 __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
@@ -714,11 +793,11 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.y * kMergeRows + warp;
   const AttnMeta* meta = reinterpret_cast<const AttnMeta*>(p.ws + p.off_meta);
-  const int32_t* ustart = reinterpret_cast<const int32_t*>(p.ws + p.off_ustart);
-  const long long T = meta->total_tiles, Pe = meta->p_eff;
+  // the two reads are independent: issued together, one round trip
+  const long long T = meta->total_tiles;
+  const int2 cr = reinterpret_cast<const int2*>(p.ws + p.off_crange)[u];   // teams holding group u
   if (T <= 0) return;
-  const long long us = ustart[u], ue = ustart[u + 1];
-  const long long c_lo = owner_team(us, T, Pe), c_hi = owner_team(ue - 1, T, Pe);
+  const long long c_lo = cr.x, c_hi = cr.y;
   if (c_lo == c_hi) return;   // a whole group: the attention kernel wrote it
   const int kvh = u % p.Hkv, b = u / p.Hkv;
   const int s_cnt = min(p.s_per_tile, p.S - qt * p.s_per_tile);
@@ -827,7 +906,7 @@ AttnPlan attn_tc_plan(const tt_attn_args_t* a, int num_sms) {
     return o;
   };
   pl.off_meta = take(sizeof(AttnMeta));
-  pl.off_ustart = take(sizeof(int32_t) * ((size_t)pl.units + 1));
+  pl.off_crange = take(sizeof(int32_t) * 2 * (size_t)pl.units);
   pl.off_partials = take(sizeof(float) * pl.slots * kRows * kD);
   pl.off_lse = take(sizeof(float) * pl.slots * kRows);
   pl.total = off;
@@ -868,7 +947,7 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   p.lse = a->lse;
   p.ws = static_cast<uint8_t*>(ws);
   p.off_meta = pl.off_meta;
-  p.off_ustart = pl.off_ustart;
+  p.off_crange = pl.off_crange;
   p.off_partials = pl.off_partials;
   p.off_lse = pl.off_lse;
   // the shared-memory opt-in is per device; set it once so no attribute call happens while a
@@ -897,7 +976,7 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   mp.lse = p.lse;
   mp.ws = p.ws;
   mp.off_meta = pl.off_meta;
-  mp.off_ustart = pl.off_ustart;
+  mp.off_crange = pl.off_crange;
   mp.off_partials = pl.off_partials;
   mp.off_lse = pl.off_lse;
   const int M = G * pl.s_per_tile;

@@ -41,7 +41,7 @@ struct AttnPlan {
   int s_per_tile;      // block positions per query-row tile
   int units;           // batch * kv heads * qtiles
   size_t off_meta;     // total tiles and working CTAs of the partition
-  size_t off_ustart;   // int32 [units + 1]: first global tile of each unit
+  size_t off_crange;   // int32 [units][2]: first and last team holding each unit's partials
   size_t off_partials; // float [slots][rows][d]
   size_t off_lse;      // float [slots][rows]
   size_t slots;
