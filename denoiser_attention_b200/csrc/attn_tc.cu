@@ -275,21 +275,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     uint32_t t_al = 0;   // chunk bound of the group-aligned partition; 0 = uniform
     if (T > 0 && T < (1LL << 31) && p.groups <= p.teams) {
       const uint32_t T32 = (uint32_t)T, teams32 = (uint32_t)p.teams, Pu32 = (uint32_t)Pu;
-      auto chunks = [&](uint32_t t) -> uint32_t {   // sum over groups of ceil(n_u / t)
-        uint32_t c = 0;
-        for (int base = 0; base < p.groups; base += 32) c += wsum(((uint32_t)ntiles_of(base, base + lane) + t - 1) / t);
-        return c;
-      };
-      uint32_t lo = (T32 - 1) / teams32 + 1;
+      // candidates t in [ceil(T/teams), ceil(T/Pu) + kSegPenaltyTiles], at most kSegPenaltyTiles + 1
+      // of them (ceil(T/Pu) = ceil(T/teams) when Pu = teams, and both are 1 when Pu = T < teams):
+      // sum_u ceil(n_u / t) for all of them in one pass, independent divisions side by side
+      const uint32_t lo = (T32 - 1) / teams32 + 1;
       uint32_t hi = (T32 - 1) / Pu32 + 1 + (uint32_t)kSegPenaltyTiles;
       if (hi > (uint32_t)nmax) hi = (uint32_t)nmax;
-      if (lo <= hi && chunks(hi) <= teams32) {
-        while (lo < hi) {   // chunks(t) does not increase with t
-          const uint32_t mid = (lo + hi) >> 1;
-          if (chunks(mid) <= teams32) hi = mid; else lo = mid + 1;
-        }
-        t_al = lo;
+      constexpr int kCand = (int)kSegPenaltyTiles + 1;
+      uint32_t cnt[kCand];
+#pragma unroll
+      for (int k = 0; k < kCand; ++k) cnt[k] = 0;
+      for (int base = 0; base < p.groups; base += 32) {
+        const uint32_t n = (uint32_t)ntiles_of(base, base + lane);
+#pragma unroll
+        for (int k = 0; k < kCand; ++k) cnt[k] += (n + lo + k - 1) / (lo + k);
       }
+#pragma unroll
+      for (int k = 0; k < kCand; ++k) cnt[k] = wsum(cnt[k]);
+      // the smallest feasible candidate (the count does not increase with t)
+#pragma unroll
+      for (int k = kCand - 1; k >= 0; --k)
+        if (lo + k <= hi && cnt[k] <= teams32) t_al = lo + k;
     }
     const bool aligned = t_al > 0;
     long long rb = T, re = T;
