@@ -34,6 +34,13 @@ if ROOT not in sys.path:
 METRIC = "denoise-step attn query-tok/s, KV-read GB/s vs HBM peak; unmask steps/s"
 WORKLOAD = "decode_bf16"
 PER_GPU_BATCH = 8
+# RefinementStep schedules (how the step's three independent branches go on streams)
+SCHEDULE_TEXT = {
+    "branches": "each step three concurrent branches on forked streams",
+    "attn_then_unmask": "each step: attention then unmask on one forked stream, the modulation alongside",
+    "unmask_then_attn": "each step: unmask then attention on one forked stream, the modulation alongside",
+    "serial": "each step on one stream",
+}
 
 
 def shard_range(global_batch: int, world: int, rank: int):
@@ -237,7 +244,7 @@ def run_ours(args):
             tokens=torch.full((B, S), 3, dtype=torch.int32, device=dev),
             is_masked=torch.ones((B, S), dtype=torch.uint8, device=dev)))
     step = api.RefinementStep(weights, gamma=w.gamma, inv_temperature=w.inv_temperature,
-                              ctx_stride=inp.ctx_stride)
+                              ctx_stride=inp.ctx_stride, schedule=args.schedule)
     outs = [torch.empty_like(s.q) for s in sets]
 
     # eager warm-up (sets the kernels' attributes, allocates workspaces), then capture M steps
@@ -341,7 +348,8 @@ def run_ours(args):
             "config": {"workload": workload_desc(w), "global_batch": global_batch,
                        "seq_len": a.ctx_lens[0] + S, "parallelism": f"dp{world} (independent sequences)",
                        "l2": f"{n_sets} rotating input sets of {ws_bytes / 1e6:.1f} MB (> 4x L2)",
-                       "timing": f"CUDA graph of {M} steps replayed (each step three concurrent branches on forked streams); per-kernel events on the streams the kernels run on"},
+                       "schedule": args.schedule,
+                       "timing": f"CUDA graph of {M} steps replayed ({SCHEDULE_TEXT[args.schedule]}); per-kernel events on the streams the kernels run on"},
             "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                          "frac": attn_gbs / peak, "traffic": traffic, "kernel": "attn_tc_kernel",
                          "peak_source": peak_src, "algorithmic_bytes_per_launch": kv_bytes},
@@ -514,6 +522,8 @@ def main():
     ap.add_argument("--kernel", choices=["attn", "unmask", "adaln", "lmhead"], default=None,
                     help="profiling mode: eager launches of one kernel only (not a bench line)")
     ap.add_argument("--workload", default=WORKLOAD, help="workload of the --kernel profiling mode")
+    ap.add_argument("--schedule", choices=list(SCHEDULE_TEXT), default="branches",
+                    help="how the step's three branches are put on streams")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

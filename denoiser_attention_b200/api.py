@@ -183,11 +183,18 @@ class RefinementStep:
     The weights (adaLN MLP, per-layer embedding, norm weight) live on the device.
 
     The step has three independent branches: a2 -> a3 -> a5 (modulation), a4 (attention) and
-    a6/a7 (unmask). With concurrent=True (the default) the attention and the unmask run on two
-    side streams forked from the caller's stream and joined back into it before run() returns,
-    so the three branches overlap on the device (and appear as parallel branches of a CUDA graph
-    captured around run()). Every output is allocated on the caller's stream before the fork.
+    a6/a7 (unmask). schedule says how they are put on streams:
+      "branches"          attention and unmask on two side streams forked from the caller's stream,
+                          the modulation on the caller's stream: all three overlap on the device
+      "attn_then_unmask"  attention, then unmask, on one side stream; the modulation alongside
+      "unmask_then_attn"  the same with the unmask first
+      "serial"            everything on the caller's stream (also concurrent=False)
+    Side streams are joined back into the caller's stream before run() returns, so a CUDA graph
+    captured around run() holds the same branches. Every output is allocated on the caller's
+    stream before the fork. The outputs do not depend on the schedule.
     """
+
+    SCHEDULES = ("branches", "attn_then_unmask", "unmask_then_attn", "serial")
 
     # kernel launches per step: adaLN COND (3 batched GEMVs), RMSNorm prologue, attention +
     # split-KV merge, gated residual, unmask
@@ -195,7 +202,8 @@ class RefinementStep:
 
     def __init__(self, weights: Dict[str, torch.Tensor], *, gamma: float, inv_temperature: float = 1.0,
                  mask_token_id: int = 3, page_size: int = 0, ctx_stride: int = 0, softmax_scale: float = 1.0,
-                 eps: float = 1e-5, remaining_steps: int = 0, concurrent: bool = True):
+                 eps: float = 1e-5, remaining_steps: int = 0, concurrent: bool = True,
+                 schedule: str = "branches"):
         self.w = weights
         self.gamma = gamma
         self.inv_temperature = inv_temperature
@@ -205,7 +213,9 @@ class RefinementStep:
         self.softmax_scale = softmax_scale
         self.eps = eps
         self.remaining_steps = remaining_steps
-        self.concurrent = concurrent
+        if schedule not in self.SCHEDULES:
+            raise ValueError(f"schedule must be one of {self.SCHEDULES}")
+        self.schedule = schedule if concurrent else "serial"
         self._streams = {}
 
     def _side(self, dev):
@@ -225,38 +235,53 @@ class RefinementStep:
         Bn = b.q.shape[0]
         nc = torch.empty(Bn, dtype=torch.int32, device=dev)
         nm = torch.empty(Bn, dtype=torch.int32, device=dev)
-        if self.concurrent:
-            s_attn, s_unm, fork, join_a, join_u = self._side(dev)
+        forked = self.schedule != "serial"
+        if forked:
+            s_a, s_b, fork, join_a, join_u = self._side(dev)
             fork.record(main)
-            s_attn.wait_event(fork)
-            s_unm.wait_event(fork)
+            s_a.wait_event(fork)
+            s_attn = s_a
+            s_unm = s_b if self.schedule == "branches" else s_a
+            if s_unm is not s_attn:
+                s_unm.wait_event(fork)
         else:
             s_attn = s_unm = main
 
-        with torch.cuda.stream(s_attn):
-            if events is not None:
-                events[0].record(s_attn)
-            denoise_attention(b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
-                              page_size=self.page_size, ctx_stride=self.ctx_stride,
-                              softmax_scale=self.softmax_scale, out=out_attn)
-            if events is not None:
-                events[1].record(s_attn)
-        with torch.cuda.stream(s_unm):
-            if events is not None:
-                events[2].record(s_unm)
-            unmask_step(b.logits, b.tokens, b.is_masked, gamma=self.gamma, inv_temperature=self.inv_temperature,
-                        mask_token_id=self.mask_token_id, remaining_steps=self.remaining_steps, want_conf=False,
-                        n_committed=nc, n_masked=nm)
-            if events is not None:
-                events[3].record(s_unm)
+        def attention():
+            with torch.cuda.stream(s_attn):
+                if events is not None:
+                    events[0].record(s_attn)
+                denoise_attention(b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
+                                  page_size=self.page_size, ctx_stride=self.ctx_stride,
+                                  softmax_scale=self.softmax_scale, out=out_attn)
+                if events is not None:
+                    events[1].record(s_attn)
+
+        def unmask():
+            with torch.cuda.stream(s_unm):
+                if events is not None:
+                    events[2].record(s_unm)
+                unmask_step(b.logits, b.tokens, b.is_masked, gamma=self.gamma,
+                            inv_temperature=self.inv_temperature, mask_token_id=self.mask_token_id,
+                            remaining_steps=self.remaining_steps, want_conf=False, n_committed=nc, n_masked=nm)
+                if events is not None:
+                    events[3].record(s_unm)
+
+        if self.schedule == "unmask_then_attn":
+            unmask()
+            attention()
+        else:
+            attention()
+            unmask()
         mod = adaln_cond(b.tau, w["w1"], w["b1"], w["w2"], w["b2"], w["w3"], w["b3"], w["layer_emb"])
         y = adaln_norm_modulate(b.h, w["norm_w"], mod, eps=self.eps)
         h_new = adaln_gated_residual(b.h, b.f, mod)
-        if self.concurrent:
+        if forked:
             join_a.record(s_attn)
-            join_u.record(s_unm)
             main.wait_event(join_a)
-            main.wait_event(join_u)
+            if s_unm is not s_attn:
+                join_u.record(s_unm)
+                main.wait_event(join_u)
         return {"mod": mod, "y": y, "attn": out_attn, "h": h_new, "n_committed": nc, "n_masked": nm}
 
 

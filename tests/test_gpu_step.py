@@ -83,20 +83,20 @@ def test_graph_captured_step_matches_eager(cuda_lib):
 
 
 def test_concurrent_branches_match_sequential(cuda_lib):
-    # the three branches on forked streams give the bits of the one-stream order
+    # every stream schedule of the three branches gives the bits of the one-stream order
     w, inp, ad, logits = _workload_inputs("decode_bf16")
     B, S = w.attn.batch, w.attn.block_size
     dev = "cuda"
     weights = {k: getattr(ad, k).to(dev) for k in ("w1", "b1", "w2", "b2", "w3", "b3", "layer_emb", "norm_w")}
     results = []
-    for concurrent in (False, True, True):
+    for schedule in ("serial", "branches", "branches", "attn_then_unmask", "unmask_then_attn"):
         bufs = api.StepBuffers(tau=ad.tau.to(dev), h=ad.h.to(dev), f=ad.f.to(dev), q=inp.q.to(dev),
                                k_blk=inp.k_blk.to(dev), v_blk=inp.v_blk.to(dev), k_ctx=inp.k_ctx.to(dev),
                                v_ctx=inp.v_ctx.to(dev), ctx_lens=inp.ctx_lens.to(dev), page_table=None,
                                logits=logits.to(dev),
                                tokens=torch.full((B, S), 3, dtype=torch.int32, device=dev),
                                is_masked=torch.ones((B, S), dtype=torch.uint8, device=dev))
-        step = api.RefinementStep(weights, gamma=w.gamma, ctx_stride=inp.ctx_stride, concurrent=concurrent)
+        step = api.RefinementStep(weights, gamma=w.gamma, ctx_stride=inp.ctx_stride, schedule=schedule)
         r = step.run(bufs)
         torch.cuda.synchronize()
         results.append({k: v.cpu() for k, v in r.items()} | {"tokens": bufs.tokens.cpu(),
