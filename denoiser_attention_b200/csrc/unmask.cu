@@ -229,7 +229,19 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
 #pragma unroll
       for (int u = 0; u < kUnmaskUnroll; ++u) consume(raw[u], v + u * kUnmaskThreads);
     }
-    for (; v < ve; v += kUnmaskThreads) consume(__ldcs(vp + v), v);
+    // the rest, fewer than kUnmaskUnroll vectors per thread: their loads in flight together (not
+    // one dependent round trip each), consumed in the same order
+    if (v < ve) {
+      uint4 raw[kUnmaskUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnmaskUnroll; ++u) {
+        const int vv = v + u * kUnmaskThreads;
+        raw[u] = vv < ve ? __ldcs(vp + vv) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnmaskUnroll; ++u)
+        if (v + u * kUnmaskThreads < ve) consume(raw[u], v + u * kUnmaskThreads);
+    }
 
     // ---- CTA reduction (warp shuffles, then across warps), lowest index on ties
     RedState st{m, s, idx};
