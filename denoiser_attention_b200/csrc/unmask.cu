@@ -3,8 +3,10 @@
 //
 // One pass over the vocabulary logits computes, per block position, the softmax maximum
 // probability (confidence) and the argmax token; the CTA that finishes the last position of a
-// sequence then applies the commit rule to that sequence. Logits are read once, with 128-bit
-// streaming loads, 8 in flight per thread.
+// sequence then applies the commit rule to that sequence. Logits are read once: each thread
+// streams its 16-byte vectors through its own ring of 8 shared-memory slots with asynchronous
+// copies (cp.async, L2 only), so 8 loads stay in flight per thread without holding registers and
+// without block barriers.
 //
 // Work split: the logits of all positions are one flat array of 16-byte vectors, cut into equal
 // contiguous ranges, one per CTA (4 CTAs per SM), so every SM streams the same number of bytes
@@ -101,7 +103,7 @@ struct UnmaskParams {
 };
 
 constexpr int kUnmaskThreads = 256;
-constexpr int kUnmaskUnroll = 8;
+constexpr int kUnmaskRing = 8;    // 16-byte vectors in flight per thread (shared-memory ring)
 constexpr int kUnmaskCtasPerSm = 4;
 
 // CTA owning vector v when E vectors are cut into P <= E ranges [c*E/P, (c+1)*E/P).
@@ -164,6 +166,15 @@ __device__ void commit_sequence(const UnmaskParams& p, int b, const float* conf_
   }
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), one commit group per call site
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <typename T>
 __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskParams p) {
   using VT = VecTraits<T>;
@@ -184,6 +195,8 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
   int* seq_cnt = reinterpret_cast<int*>(p.ws + p.off_seq_cnt);
   UnmaskPartial* parts = reinterpret_cast<UnmaskPartial*>(p.ws + p.off_partials);
   __shared__ RedState s_red[kUnmaskThreads / 32];
+  // each thread's own ring of kUnmaskRing vectors (slot-major: consecutive threads, consecutive 16 B)
+  __shared__ __align__(16) uint4 s_ring[kUnmaskRing][kUnmaskThreads];
   __shared__ int s_flag;
   const int warp = tid >> 5, lane = tid & 31;
 
@@ -221,27 +234,23 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
 #pragma unroll
       for (int k = 0; k < N; ++k) s += ex2(fmaf(x[k], c, nmc));
     };
-    int v = vb + tid;
-    for (; v + (kUnmaskUnroll - 1) * kUnmaskThreads < ve; v += kUnmaskUnroll * kUnmaskThreads) {
-      uint4 raw[kUnmaskUnroll];
+    // this thread's vectors vb + tid + i * kUnmaskThreads, i < nv, stream through its ring: the
+    // copy of vector i + kUnmaskRing is issued once vector i has been consumed, so kUnmaskRing
+    // copies stay in flight (one commit group per index, empty past the end, keeps the count)
+    const int nv = (ve - vb > tid) ? (ve - vb - tid + kUnmaskThreads - 1) / kUnmaskThreads : 0;
+    auto issue = [&](int i) {
+      if (i < nv) cp_async16(&s_ring[i % kUnmaskRing][tid], vp + vb + tid + i * kUnmaskThreads);
+      cp_async_commit();
+    };
 #pragma unroll
-      for (int u = 0; u < kUnmaskUnroll; ++u) raw[u] = __ldcs(vp + v + u * kUnmaskThreads);
-#pragma unroll
-      for (int u = 0; u < kUnmaskUnroll; ++u) consume(raw[u], v + u * kUnmaskThreads);
+    for (int i = 0; i < kUnmaskRing; ++i) issue(i);
+    for (int i = 0; i < nv; ++i) {
+      cp_async_wait<kUnmaskRing - 1>();   // the oldest copy (vector i) has landed
+      const uint4 raw = s_ring[i % kUnmaskRing][tid];
+      consume(raw, vb + tid + i * kUnmaskThreads);
+      issue(i + kUnmaskRing);
     }
-    // the rest, fewer than kUnmaskUnroll vectors per thread: their loads in flight together (not
-    // one dependent round trip each), consumed in the same order
-    if (v < ve) {
-      uint4 raw[kUnmaskUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnmaskUnroll; ++u) {
-        const int vv = v + u * kUnmaskThreads;
-        raw[u] = vv < ve ? __ldcs(vp + vv) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnmaskUnroll; ++u)
-        if (v + u * kUnmaskThreads < ve) consume(raw[u], v + u * kUnmaskThreads);
-    }
+    cp_async_wait<0>();
 
     // ---- CTA reduction (warp shuffles, then across warps), lowest index on ties
     RedState st{m, s, idx};
