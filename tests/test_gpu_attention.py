@@ -65,6 +65,9 @@ CASES = [
     (1, 16, 4, 1, 64, [64], torch.float32, 0),
     (3, 7, 8, 2, 128, [0, 90, 300], torch.float32, 0),
     (2, 16, 4, 1, 64, [100, 37], torch.float32, 32),
+    # more than 32 groups with the group-aligned partition (on 148 SMs: 74 teams):
+    (36, 16, 32, 2, 128, [300] * 36, torch.bfloat16, 0),    # 72 groups of 4 tiles, one team each
+    (17, 16, 32, 2, 128, [1024] * 17, torch.bfloat16, 0),   # 34 groups of 9 tiles, chunks of 4 + 5
 ]
 
 
