@@ -39,7 +39,7 @@ struct AttnPlan {
   int grid;            // persistent CTAs
   int qtiles;          // query-row tiles per (sequence, kv head)
   int s_per_tile;      // block positions per query-row tile
-  int units;           // batch * kv heads * qtiles
+  int units;           // groups: batch * kv heads
   size_t off_meta;     // total tiles and working CTAs of the partition
   size_t off_crange;   // int32 [units][2]: first and last team holding each unit's partials
   size_t off_partials; // float [slots][rows][d]
