@@ -239,13 +239,15 @@ def unmask_step(tokens, is_masked, logits, gamma: float, inv_temperature: float 
     return t, m, nc, nm, conf, arg
 
 
-def predict_noise_step(tokens, is_masked, logits, keep_masked: int, inv_temperature: float = 1.0):
+def predict_noise_step(tokens, is_masked, logits, keep_masked: int, inv_temperature: float = 1.0,
+                       exclude_token: Optional[int] = None):
     """The predict-and-noise sampler of block diffusion (the paper §2.2 "Sampling"): predict every
-    masked position (argmax, confidence as in confidence_argmax), then re-mask the least
-    confident ones so that min(n_masked, keep_masked) stay masked; i.e. commit the
-    (n_masked - keep_masked) most confident masked positions, confidence descending and position
-    ascending on ties. Committed positions are never changed."""
-    conf, arg = confidence_argmax(logits, inv_temperature)
+    masked position (argmax, confidence as in confidence_argmax, with the same optional removal
+    of the [MASK] token's own logit), then re-mask the least confident ones so that
+    min(n_masked, keep_masked) stay masked; i.e. commit the (n_masked - keep_masked) most
+    confident masked positions, confidence descending and position ascending on ties. Committed
+    positions are never changed."""
+    conf, arg = confidence_argmax(logits, inv_temperature, exclude_token)
     tokens = np.array(tokens, dtype=np.int64, copy=True)
     is_masked = np.array(is_masked, dtype=bool, copy=True)
     n_committed = np.zeros(tokens.shape[0], dtype=np.int64)

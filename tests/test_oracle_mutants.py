@@ -32,6 +32,10 @@ MUTANTS = [
     ("floor schedule", "need = -(-len(masked) // remaining_steps)", "need = len(masked) // remaining_steps"),
     ("tau from committed count", "tau = is_masked.sum(axis=1) / block_size", "tau = (~is_masked).sum(axis=1) / block_size"),
     ("no fallback", "if len(chosen) < need:", "if False:"),
+    ("predict-noise ignores exclusion",
+     'positions are never changed."""\n    conf, arg = confidence_argmax(logits, inv_temperature, exclude_token)',
+     'positions are never changed."""\n    conf, arg = confidence_argmax(logits, inv_temperature)'),
+    ("schedule rounds up", "return (block_size * (steps - r)) // steps", "return -(-(block_size * (steps - r)) // steps)"),
 ]
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
@@ -44,7 +48,9 @@ def _run_pins():
         params = [m for m in marks if m.name == "parametrize"]
         cases = [()]
         if params:
-            cases = params[0].args[1]
+            names = params[0].args[0]
+            single = isinstance(names, str) and "," not in names
+            cases = [(c,) for c in params[0].args[1]] if single else params[0].args[1]
         for case in cases:
             try:
                 fn(*case)

@@ -541,17 +541,49 @@ def test_predict_noise_ties_go_to_the_lower_position():
     assert m[0].tolist() == [False, False, True, True] and nc[0] == 2
 
 
-def test_predict_noise_linear_schedule_finishes_at_T():
-    S, T = 16, 6
-    rs = np.random.default_rng(22)
+def _schedule_cases():
+    return json.load(open(os.path.join(GOLDEN, "noise_schedule_linear.json")))["cases"]
+
+
+@pytest.mark.parametrize("case", _schedule_cases(), ids=lambda c: f"S{c['S']}T{c['T']}")
+def test_predict_noise_linear_schedule_golden(case):
+    # the hand-derived table (alpha_t = 1 - t, the masked fraction after step r is (T - r) / T):
+    # the schedule and a whole T-step predict-and-noise loop both follow it, ending with none left
+    S, T, want = case["S"], case["T"], case["keep"]
+    assert [O.linear_schedule_keep(S, T, r) for r in range(1, T + 1)] == want
+    rs = np.random.default_rng(22 + S + T)
     tokens, masked = np.full((2, S), 3), np.ones((2, S), bool)
     left = []
     for r in range(1, T + 1):
-        keep = O.linear_schedule_keep(S, T, r)
-        tokens, masked, _, _, _, _ = O.predict_noise_step(tokens, masked, rs.standard_normal((2, S, 32)), keep)
-        left.append(int(masked[0].sum()))
-    # the masked fraction after step r is (T - r) / T of the block, rounded down; none left at T
-    assert left == [(S * (T - r)) // T for r in range(1, T + 1)] and left[-1] == 0
+        tokens, masked, _, _, _, _ = O.predict_noise_step(tokens, masked, rs.standard_normal((2, S, 32)),
+                                                          O.linear_schedule_keep(S, T, r))
+        left.append(masked.sum(axis=1).tolist())
+    assert left == [[k, k] for k in want] and left[-1] == [0, 0]
+
+
+def test_predict_noise_excluded_token():
+    # with the [MASK] id excluded its logit takes part in neither the confidence nor the argmax
+    # (reading R10), so the ranking is the one of the logits with that column removed
+    rs = np.random.default_rng(23)
+    B, S, V, mask_id = 2, 8, 12, 3
+    logits = rs.standard_normal((B, S, V))
+    logits[:, :, mask_id] = 30.0
+    masked = np.ones((B, S), bool)
+    t, m, nc, _, conf, arg = O.predict_noise_step(np.full((B, S), mask_id), masked, logits, 3, exclude_token=mask_id)
+    assert (arg != mask_id).all()
+    kept = np.delete(logits, mask_id, axis=2)
+    p = np.exp(kept - kept.max(axis=2, keepdims=True))
+    np.testing.assert_allclose(conf, (p / p.sum(axis=2, keepdims=True)).max(axis=2), rtol=0, atol=1e-15)
+    want_arg = np.argmax(kept, axis=2)
+    want_arg = want_arg + (want_arg >= mask_id)
+    np.testing.assert_array_equal(arg, want_arg)
+    for b in range(B):
+        top = sorted(range(S), key=lambda l: (conf[b, l], -l), reverse=True)[:S - 3]
+        assert set(np.flatnonzero(~m[b])) == set(top) and nc[b] == S - 3
+        assert (t[b][~m[b]] == arg[b][~m[b]]).all()
+    # without the exclusion every position would predict the [MASK] id with confidence ~1
+    _, _, _, _, conf_in, arg_in = O.predict_noise_step(np.full((B, S), mask_id), masked, logits, 3)
+    assert (arg_in == mask_id).all() and (conf_in > 0.99).all()
 
 
 # ---------------------------------------------------------------- LM head
