@@ -3,13 +3,17 @@
 A step is one pass of the whole hot path over one batch: adaLN-single conditioning, modulated
 RMSNorm prologue, Eq. (1) layer-aligned denoiser attention, gated residual and ConfidenceSample
 over the vocabulary logits (the paper "Nemotron-TwoTower: Diffusion Language Modeling with
-Pretrained AR Context", §2.1-§2.2, Algorithm 2). The workload is the bf16 decode step: per GPU
-8 sequences with 4096 context tokens + a block of S=16, 32 query / 2 kv heads, head dim 128,
-adaLN width 2048, vocabulary 131072, gamma 0.8, seeded synthetic inputs.
+Pretrained AR Context", §2.1-§2.2, Algorithm 2). The headline workload is the bf16 batch-generation
+step: per GPU 64 sequences with 16384 context tokens + a block of S=16 at step t=8 of T=16
+(tau = 9/16), 32 query / 2 kv heads, head dim 128, adaLN width 2048, vocabulary 131072, gamma
+0.8, seeded synthetic inputs. Extra keys report the decode step (8 sequences, 4096 context
+tokens), the attention alone on every workload, and the block-sweep unmask table (committed
+tokens per step for S x temperature x gamma).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-extras]
 
-N > 1 runs under torchrun: every rank processes its own 8 sequences (weak scaling; sequences
+N > 1 runs under torchrun: every rank processes its own 64 sequences (weak scaling; sequences
 are independent, so there is no data-path collective); the elapsed time is the max over ranks.
 `--impl reference` times the CPU fp64 oracle on the host cores instead (the comparison arm).
 Rank 0 prints one JSON line.
@@ -18,7 +22,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import re
 import math
 import os
 import statistics
@@ -32,8 +35,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "denoise-step attn query-tok/s, KV-read GB/s vs HBM peak; unmask steps/s"
-WORKLOAD = "decode_bf16"
-PER_GPU_BATCH = 8
+# the headline: the batch-generation workload, the largest configuration that fits one GPU
+WORKLOAD = "batch_bf16"
 # RefinementStep schedules (how the step's three independent branches go on streams)
 SCHEDULE_TEXT = {
     "branches": "each step three concurrent branches on forked streams",
@@ -156,11 +159,12 @@ def blas_threads() -> int:
 
 
 def host_inputs(w, seed_offset: int = 0):
-    import torch
+    """Seeded host tensors of one step of workload w: attention inputs, adaLN inputs (tau = the
+    workload's fixed time, else 1: the first refinement step, everything masked) and logits."""
     from denoiser_attention_b200 import synth
     inp = synth.attention_inputs(w.attn, seed=w.seed + seed_offset)
     B, S = w.attn.batch, w.attn.block_size
-    tau = [1.0] * B   # first refinement step: the whole block is masked (Algorithm 2's time input)
+    tau = [w.tau if w.tau is not None else 1.0] * B
     ad = synth.adaln_inputs(B, S, w.hidden, tau, seed=w.seed + 100 + seed_offset, dtype=w.attn.dtype)
     logits = synth.workload_logits(w, seed=w.seed + seed_offset)
     return inp, ad, logits
@@ -172,7 +176,7 @@ def run_reference(args):
     if rank != 0:
         return
     from denoiser_attention_b200 import synth
-    w = synth.workload(WORKLOAD)
+    w = synth.workload(args.workload)
     inp, ad, logits = host_inputs(w)
     B, S = w.attn.batch, w.attn.block_size
     # calibrate one token sample, then size each step so that warmup + steps take ~2 minutes
@@ -207,186 +211,62 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------------------------------ our arm
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
-    from denoiser_attention_b200 import api, build, synth
+def kv_bytes_of(a) -> int:
+    """Algorithmic K/V bytes of one attention launch: (context + block) tokens x kv heads x
+    (K + V) x d x 2 bytes (bf16)."""
+    return sum(int(L) + a.block_size for L in a.ctx_lens) * a.num_kv_heads * a.head_dim * 2 * 2
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    build.build()
 
-    w = synth.workload(WORKLOAD)
-    B, S = w.attn.batch, w.attn.block_size
-    global_batch = B * world
-    lo, hi = shard_range(global_batch, world, rank)
-    assert hi - lo == B
-    inp, ad, logits = host_inputs(w, seed_offset=lo)     # this rank's sequences
+def attn_flops_of(a) -> int:
+    """Tensor-core FLOPs of one attention launch: 4 G S d per key and kv head (QK^T and PV)."""
+    G = a.num_q_heads // a.num_kv_heads
+    return sum(int(L) + a.block_size for L in a.ctx_lens) * a.num_kv_heads * 4 * G * a.block_size * a.head_dim
 
-    # ---- rotating input sets on the device (same bytes at distinct addresses): the per-step
-    # working set is smaller than L2, so consecutive steps read different sets
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    ws_bytes = sum(t.numel() * t.element_size() for t in (inp.k_ctx, inp.v_ctx, logits, inp.q, ad.h, ad.f))
-    n_sets = max(2, math.ceil(4 * l2 / ws_bytes))
-    weights = {k: getattr(ad, k).to(dev) for k in ("w1", "b1", "w2", "b2", "w3", "b3", "layer_emb", "norm_w")}
-    sets = []
-    for i in range(n_sets):
-        sets.append(api.StepBuffers(
-            tau=ad.tau.to(dev), h=ad.h.to(dev), f=ad.f.to(dev), q=inp.q.to(dev), k_blk=inp.k_blk.to(dev),
-            v_blk=inp.v_blk.to(dev), k_ctx=inp.k_ctx.to(dev), v_ctx=inp.v_ctx.to(dev),
-            ctx_lens=inp.ctx_lens.to(dev), page_table=None, logits=logits.to(dev),
-            tokens=torch.full((B, S), 3, dtype=torch.int32, device=dev),
-            is_masked=torch.ones((B, S), dtype=torch.uint8, device=dev)))
-    step = api.RefinementStep(weights, gamma=w.gamma, inv_temperature=w.inv_temperature,
-                              ctx_stride=inp.ctx_stride, schedule=args.schedule)
-    outs = [torch.empty_like(s.q) for s in sets]
 
-    # eager warm-up (sets the kernels' attributes, allocates workspaces), then capture M steps
-    for i in range(n_sets):
-        step.run(sets[i], out_attn=outs[i])
-    torch.cuda.synchronize()
-    M = 2 * n_sets
-    # events recorded inside the graph must be "external" to become timestamped graph nodes
-    mk = lambda: torch.cuda.Event(enable_timing=True, external=True)
-    ev = [(mk(), mk(), mk(), mk()) for _ in range(M)]
-    g = torch.cuda.CUDAGraph()
-    cap_stream = torch.cuda.Stream(device=dev)
-    cap_stream.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(cap_stream):
-        with torch.cuda.graph(g, stream=cap_stream):
-            for j in range(M):
-                step.run(sets[j % n_sets], out_attn=outs[j % n_sets], events=ev[j])
-    torch.cuda.current_stream().wait_stream(cap_stream)
-    launches_per_step = api.RefinementStep.LAUNCHES
+class StepRun:
+    """Device buffers of one workload (rotating input sets, more than 4x L2 in total) and its
+    RefinementStep, with a CUDA graph of M steps holding per-branch timing events."""
 
-    # warm-up: at least W steps and about half a second, untimed
-    reps_w = max(1, math.ceil(args.warmup / M))
-    clocks = ClockSampler(local)
-    clocks.start()
-    t_w = time.time()
-    while True:
-        for _ in range(reps_w):
-            g.replay()
+    def __init__(self, w, inp, ad, logits, dev, schedule):
+        import torch
+        from denoiser_attention_b200 import api
+        B, S = w.attn.batch, w.attn.block_size
+        self.w = w
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.set_bytes = sum(t.numel() * t.element_size() for t in (inp.k_ctx, inp.v_ctx, logits, inp.q, ad.h, ad.f))
+        self.n_sets = max(2, math.ceil(4 * l2 / self.set_bytes))
+        weights = {k: getattr(ad, k).to(dev) for k in ("w1", "b1", "w2", "b2", "w3", "b3", "layer_emb", "norm_w")}
+        self.sets = []
+        for _ in range(self.n_sets):
+            self.sets.append(api.StepBuffers(
+                tau=ad.tau.to(dev), h=ad.h.to(dev), f=ad.f.to(dev), q=inp.q.to(dev), k_blk=inp.k_blk.to(dev),
+                v_blk=inp.v_blk.to(dev), k_ctx=inp.k_ctx.to(dev), v_ctx=inp.v_ctx.to(dev),
+                ctx_lens=inp.ctx_lens.to(dev),
+                page_table=None if inp.page_table is None else inp.page_table.to(dev), logits=logits.to(dev),
+                tokens=torch.full((B, S), 3, dtype=torch.int32, device=dev),
+                is_masked=torch.ones((B, S), dtype=torch.uint8, device=dev)))
+        self.step = api.RefinementStep(weights, gamma=w.gamma, inv_temperature=w.inv_temperature,
+                                       page_size=w.attn.page_size, ctx_stride=inp.ctx_stride, schedule=schedule)
+        self.outs = [torch.empty_like(s.q) for s in self.sets]
+        for i in range(self.n_sets):   # eager warm-up: kernel attributes, workspaces
+            self.step.run(self.sets[i], out_attn=self.outs[i])
         torch.cuda.synchronize()
-        if time.time() - t_w > 0.5:
-            break
-    # ---- timed region: exactly K steps (R replays of M steps, then a remainder graph)
-    R, rem = divmod(args.steps, M)
-    g_rem = None
-    if rem:
-        g_rem = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(cap_stream):
-            with torch.cuda.graph(g_rem, stream=cap_stream):
-                for j in range(rem):
-                    step.run(sets[j % n_sets], out_attn=outs[j % n_sets])
-        torch.cuda.current_stream().wait_stream(cap_stream)
+        self.cap_stream = torch.cuda.Stream(device=dev)
+
+    def capture(self, n_steps, with_events):
+        import torch
+        mk = lambda: torch.cuda.Event(enable_timing=True, external=True)
+        ev = [(mk(), mk(), mk(), mk()) for _ in range(n_steps)] if with_events else None
+        g = torch.cuda.CUDAGraph()
+        self.cap_stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.cap_stream):
+            with torch.cuda.graph(g, stream=self.cap_stream):
+                for j in range(n_steps):
+                    k = j % self.n_sets
+                    self.step.run(self.sets[k], out_attn=self.outs[k], events=None if ev is None else ev[j])
+        torch.cuda.current_stream().wait_stream(self.cap_stream)
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_c0 = time.time()
-    start.record()
-    for _ in range(R):
-        g.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    stop.record()
-    torch.cuda.synchronize()
-    t_c1 = time.time()
-    if world > 1:
-        dist.barrier()
-    clocks.stop()
-    ms = start.elapsed_time(stop)
-    ms_max = max_over_ranks(ms, dev)
-    ms_per_step = ms_max / args.steps
-
-    # per-kernel durations from the events of the last replay of the M-step graph
-    if R == 0:
-        for _ in range(1):
-            g.replay()
-        torch.cuda.synchronize()
-    attn_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    unmask_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
-    attn_ms = max_over_ranks(attn_ms, dev)
-    unmask_ms = max_over_ranks(unmask_ms, dev)
-    # the same two kernels alone (own graphs over the same rotating input sets), for context: inside
-    # the step they share the GPU with the other branches
-    attn_iso_ms = max_over_ranks(isolated_ms(lambda b, o: api.denoise_attention(
-        b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens, page_table=b.page_table,
-        page_size=step.page_size, ctx_stride=step.ctx_stride, softmax_scale=step.softmax_scale, out=o),
-        sets, outs, cap_stream), dev)
-    unmask_iso_ms = max_over_ranks(isolated_ms(lambda b, o: api.unmask_step(
-        b.logits, b.tokens, b.is_masked, gamma=step.gamma, inv_temperature=step.inv_temperature,
-        mask_token_id=step.mask_token_id, want_conf=False), sets, outs, cap_stream), dev)
-
-    a = w.attn
-    kv_bytes = B * (a.ctx_lens[0] + S) * a.num_kv_heads * a.head_dim * 2 * 2
-    logit_bytes = B * S * w.vocab * 2
-    peak, peak_src = measured_peaks()
-    attn_gbs = kv_bytes / (attn_ms * 1e-3) / 1e9
-    unmask_gbs = logit_bytes / (unmask_ms * 1e-3) / 1e9
-    traffic = measured_traffic()
-
-    # ---- end to end through the public API with host buffers (pinned), copies timed
-    e2e = run_e2e(step, inp, ad, logits, w, dev, args, world)
-
-    result = None
-    if rank == 0:
-        value = global_batch * S / (ms_max * 1e-3 / args.steps)
-        cpu = cpu_baseline(w, inp, ad, logits) if world == 1 else None
-        result = {
-            "metric": METRIC, "value": value, "unit": "query-tok/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_desc(w), "global_batch": global_batch,
-                       "seq_len": a.ctx_lens[0] + S, "parallelism": f"dp{world} (independent sequences)",
-                       "l2": f"{n_sets} rotating input sets of {ws_bytes / 1e6:.1f} MB (> 4x L2)",
-                       "schedule": args.schedule,
-                       "timing": f"CUDA graph of {M} steps replayed ({SCHEDULE_TEXT[args.schedule]}); per-kernel events on the streams the kernels run on"},
-            "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": attn_gbs / peak, "traffic": traffic, "kernel": "attn_tc_kernel",
-                         "peak_source": peak_src, "algorithmic_bytes_per_launch": kv_bytes},
-            "attn_us": attn_ms * 1e3, "attn_kv_gbs": attn_gbs, "attn_query_tok_s": B * S / (attn_ms * 1e-3),
-            "attn_isolated_us": attn_iso_ms * 1e3, "attn_isolated_kv_gbs": kv_bytes / (attn_iso_ms * 1e-3) / 1e9,
-            "attn_isolated_frac": kv_bytes / (attn_iso_ms * 1e-3) / 1e9 / peak,
-            "unmask_isolated_us": unmask_iso_ms * 1e3,
-            "unmask_us": unmask_ms * 1e3, "unmask_steps_per_s": 1.0 / (unmask_ms * 1e-3),
-            "unmask_logits_gbs": unmask_gbs, "unmask_frac": unmask_gbs / peak,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks.summary(t_c0 - 0.3, t_c1 + 0.1),
-        }
-        print(json.dumps(result))
-    if world > 1:
-        dist.barrier()
-        del g
-        dist.destroy_process_group()
-    return result
-
-
-def measured_traffic():
-    """DRAM bytes (read + write) per attention launch from the committed ncu summary of the decode
-    workload, or None when that summary is absent or was taken on another version of the kernel
-    source (its recorded sha256 differs from the current attn_tc.cu)."""
-    import hashlib
-    p = os.path.join(ROOT, "profiles", "attn_tc_kernel_decode_bf16.md")
-    src = os.path.join(ROOT, "denoiser_attention_b200", "csrc", "attn_tc.cu")
-    if not os.path.exists(p):
-        return None
-    text = open(p).read()
-    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
-    if not (m_bytes and m_sha):
-        return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
-        return None
-    return int(m_bytes.group(1))
+        return g, ev
 
 
 def isolated_ms(op, sets, outs, cap_stream, reps: int = 20):
@@ -414,6 +294,257 @@ def isolated_ms(op, sets, outs, cap_stream, reps: int = 20):
     return ms
 
 
+def attn_op(step):
+    from denoiser_attention_b200 import api
+    return lambda b, o: api.denoise_attention(b.q, b.k_blk, b.v_blk, b.k_ctx, b.v_ctx, b.ctx_lens,
+                                              page_table=b.page_table, page_size=step.page_size,
+                                              ctx_stride=step.ctx_stride, softmax_scale=step.softmax_scale, out=o)
+
+
+def unmask_op(step):
+    from denoiser_attention_b200 import api
+    return lambda b, o: api.unmask_step(b.logits, b.tokens, b.is_masked, gamma=step.gamma,
+                                        inv_temperature=step.inv_temperature, mask_token_id=step.mask_token_id,
+                                        want_conf=False)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from denoiser_attention_b200 import api, build, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    build.build()
+
+    w = synth.workload(args.workload)
+    B, S = w.attn.batch, w.attn.block_size
+    global_batch = B * world
+    lo, hi = shard_range(global_batch, world, rank)
+    assert hi - lo == B
+    inp, ad, logits = host_inputs(w, seed_offset=lo)     # this rank's sequences
+    run = StepRun(w, inp, ad, logits, dev, args.schedule)
+    M = 2 * run.n_sets
+    g, ev = run.capture(M, with_events=True)
+
+    # warm-up: at least W steps and about half a second, untimed
+    reps_w = max(1, math.ceil(args.warmup / M))
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_w = time.time()
+    while True:
+        for _ in range(reps_w):
+            g.replay()
+        torch.cuda.synchronize()
+        if time.time() - t_w > 0.5:
+            break
+    # ---- timed region: exactly K steps (R replays of M steps, then a remainder graph)
+    R, rem = divmod(args.steps, M)
+    g_rem = run.capture(rem, with_events=False)[0] if rem else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_c0 = time.time()
+    start.record()
+    for _ in range(R):
+        g.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    t_c1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    ms = start.elapsed_time(stop)
+    ms_max = max_over_ranks(ms, dev)
+    ms_per_step = ms_max / args.steps
+
+    # per-kernel durations from the events of the last replay of the M-step graph
+    if R == 0:
+        g.replay()
+        torch.cuda.synchronize()
+    attn_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev), dev)
+    unmask_ms = max_over_ranks(statistics.mean(e[2].elapsed_time(e[3]) for e in ev), dev)
+    del g, g_rem
+    # the same two kernels alone (own graphs over the same rotating input sets), for context: inside
+    # the step they share the GPU with the other branches
+    attn_iso_ms = max_over_ranks(isolated_ms(attn_op(run.step), run.sets, run.outs, run.cap_stream), dev)
+    unmask_iso_ms = max_over_ranks(isolated_ms(unmask_op(run.step), run.sets, run.outs, run.cap_stream), dev)
+
+    a = w.attn
+    kv_bytes = kv_bytes_of(a)
+    logit_bytes = B * S * w.vocab * 2
+    peak, peak_src = measured_peaks()
+    attn_gbs = kv_bytes / (attn_ms * 1e-3) / 1e9
+    unmask_gbs = logit_bytes / (unmask_ms * 1e-3) / 1e9
+    traffic = measured_traffic(args.workload)
+    launches_per_step = api.RefinementStep.LAUNCHES
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    e2e = run_e2e(run.step, inp, ad, logits, w, dev, args, world)
+    del run
+    torch.cuda.empty_cache()
+
+    extras = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        extras = run_extras(args, dev, peak)
+
+    result = None
+    if rank == 0:
+        value = global_batch * S / (ms_max * 1e-3 / args.steps)
+        cpu = cpu_baseline(w, inp, ad, logits) if world == 1 else None
+        result = {
+            "metric": METRIC, "value": value, "unit": "query-tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_desc(w), "global_batch": global_batch,
+                       "seq_len": a.ctx_lens[0] + S, "parallelism": f"dp{world} (independent sequences)",
+                       "l2": f"{M // 2} rotating input sets of {run_set_mb(inp, ad, logits):.1f} MB (> 4x L2 together)",
+                       "schedule": args.schedule,
+                       "timing": f"CUDA graph of {M} steps replayed ({SCHEDULE_TEXT[args.schedule]}); per-kernel events on the streams the kernels run on"},
+            "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": attn_gbs / peak, "traffic": traffic, "kernel": "attn_tc_kernel",
+                         "peak_source": peak_src, "algorithmic_bytes_per_launch": kv_bytes},
+            "attn_us": attn_ms * 1e3, "attn_kv_gbs": attn_gbs, "attn_query_tok_s": B * S / (attn_ms * 1e-3),
+            "attn_tflops": attn_flops_of(a) / (attn_ms * 1e-3) / 1e12,
+            "attn_isolated_us": attn_iso_ms * 1e3, "attn_isolated_kv_gbs": kv_bytes / (attn_iso_ms * 1e-3) / 1e9,
+            "attn_isolated_frac": kv_bytes / (attn_iso_ms * 1e-3) / 1e9 / peak,
+            "unmask_isolated_us": unmask_iso_ms * 1e3,
+            "unmask_us": unmask_ms * 1e3, "unmask_steps_per_s": 1.0 / (unmask_ms * 1e-3),
+            "unmask_logits_gbs": unmask_gbs, "unmask_frac": unmask_gbs / peak,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(t_c0 - 0.3, t_c1 + 0.1),
+        }
+        if extras is not None:
+            result.update(extras)
+        print(json.dumps(result))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_set_mb(inp, ad, logits) -> float:
+    return sum(t.numel() * t.element_size() for t in (inp.k_ctx, inp.v_ctx, logits, inp.q, ad.h, ad.f)) / 1e6
+
+
+def run_extras(args, dev, peak):
+    """Numbers beyond the headline, each from CUDA events over graphs of rotating input sets: the
+    decode step, the attention alone on every workload, and the block-sweep unmask table."""
+    import torch
+    from denoiser_attention_b200 import api, synth
+    out = {}
+    # ---- the decode step (8 sequences, ctx 4096): whole step and its kernels
+    w = synth.workload("decode_bf16")
+    inp, ad, logits = host_inputs(w)
+    run = StepRun(w, inp, ad, logits, dev, args.schedule)
+    M = 2 * run.n_sets
+    g, ev = run.capture(M, with_events=True)
+    for _ in range(5):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, math.ceil(2000 / M))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * M)
+    attn_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    unmask_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    del g
+    kvb = kv_bytes_of(w.attn)
+    out["decode_step"] = {
+        "workload": workload_desc(w), "value": w.attn.batch * w.attn.block_size / (ms * 1e-3),
+        "unit": "query-tok/s", "ms_per_step": ms, "steps": reps * M, "attn_us": attn_ms * 1e3,
+        "attn_frac": kvb / (attn_ms * 1e-3) / 1e9 / peak, "unmask_us": unmask_ms * 1e3}
+    del run
+    # ---- the attention alone on every workload
+    attn = {}
+    for name, S in (("decode_bf16", None), ("batch_bf16", None), ("ragged_paged", None),
+                    ("sweep_bf16", 4), ("sweep_bf16", 8), ("sweep_bf16", 16), ("sweep_bf16", 32), ("sweep_bf16", 64)):
+        w = synth.workload(name, block_size=S)
+        a = synth.attention_inputs(w.attn, seed=w.seed)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        nbytes = (a.k_ctx.numel() + a.v_ctx.numel()) * 2
+        n_sets = max(2, math.ceil(4 * l2 / nbytes))
+        sets = []
+        for _ in range(n_sets):
+            sets.append(api.StepBuffers(
+                tau=None, h=None, f=None, q=a.q.to(dev), k_blk=a.k_blk.to(dev), v_blk=a.v_blk.to(dev),
+                k_ctx=a.k_ctx.to(dev), v_ctx=a.v_ctx.to(dev), ctx_lens=a.ctx_lens.to(dev),
+                page_table=None if a.page_table is None else a.page_table.to(dev), logits=None, tokens=None,
+                is_masked=None))
+        outs = [torch.empty_like(s.q) for s in sets]
+        step = api.RefinementStep({}, gamma=0.8, page_size=w.attn.page_size, ctx_stride=a.ctx_stride)
+        for b, o in zip(sets, outs):
+            attn_op(step)(b, o)
+        torch.cuda.synchronize()
+        ms = isolated_ms(attn_op(step), sets, outs, torch.cuda.Stream(device=dev), reps=max(3, 200 // n_sets))
+        kvb = kv_bytes_of(w.attn)
+        key = name if S is None else f"{name}_S{S}"
+        attn[key] = {"us": ms * 1e3, "kv_gbs": kvb / (ms * 1e-3) / 1e9, "frac": kvb / (ms * 1e-3) / 1e9 / peak,
+                     "tflops": attn_flops_of(w.attn) / (ms * 1e-3) / 1e12, "kv_bytes": kvb}
+        del sets, outs, a
+        torch.cuda.empty_cache()
+    out["attention"] = attn
+    # ---- the block-sweep unmask table: per S the unmask step time, and per (S, temperature,
+    # gamma) the mean number of positions committed in the first refinement step (all masked)
+    table = []
+    times = {}
+    for S in (4, 8, 16, 32, 64):
+        w = synth.workload("sweep_bf16", block_size=S)
+        B = w.attn.batch
+        lg = synth.workload_logits(w).to(dev)
+        t = torch.full((B, S), 3, dtype=torch.int32, device=dev)
+        m = torch.ones((B, S), dtype=torch.uint8, device=dev)
+        for inv_temp in (2.0, 1.0, 0.5):
+            for gamma in (0.5, 0.7, 0.8, 0.9, 0.95):
+                t.fill_(3)
+                m.fill_(1)
+                nc, _, conf, _ = api.unmask_step(lg, t, m, gamma=gamma, inv_temperature=inv_temp)
+                torch.cuda.synchronize()
+                table.append({"S": S, "temperature": 1.0 / inv_temp, "gamma": gamma,
+                              "committed_per_step": float(nc.float().mean()),
+                              "frac_above_gamma": float((conf >= gamma).float().mean())})
+        b = api.StepBuffers(tau=None, h=None, f=None, q=None, k_blk=None, v_blk=None, k_ctx=None, v_ctx=None,
+                            ctx_lens=None, page_table=None, logits=lg, tokens=t, is_masked=m)
+        st = api.RefinementStep({}, gamma=0.8)
+        times[S] = isolated_ms(unmask_op(st), [b], [None], torch.cuda.Stream(device=dev), reps=50) * 1e3
+        del lg
+        torch.cuda.empty_cache()
+    out["sweep_unmask"] = {"unmask_us_by_S": times, "cells": table,
+                           "note": "committed tokens per step: mean over the 32 sequences of the first step "
+                                   "(every position masked), confidence sampler"}
+    return out
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes (read + write) per attention launch on `workload` from the ncu capture recorded
+    in profiles/attn_tc_kernel_traffic.json, or None when there is none for this workload or it
+    was taken on another version of the kernel source (its sha256 differs from attn_tc.cu)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "attn_tc_kernel_traffic.json")
+    src = os.path.join(ROOT, "denoiser_attention_b200", "csrc", "attn_tc.cu")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(workload)
+    if not rec:
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec.get("source_sha256"):
+        return None
+    return int(rec["dram_bytes_per_launch"])
+
+
 def run_e2e(step, inp, ad, logits, w, dev, args, world):
     """Same metric through the public host-buffer API: every step copies its inputs from pinned
     host memory to the device, runs the step and copies the results back."""
@@ -429,7 +560,7 @@ def run_e2e(step, inp, ad, logits, w, dev, args, world):
     runner = api.HostStep(step, host, dev)
     h2d = runner.h2d_bytes
     d2h = runner.d2h_bytes
-    steps = max(3, min(args.steps, 50))
+    steps = max(3, min(args.steps, 20))
     for _ in range(3):
         runner.run()
     torch.cuda.synchronize()
@@ -459,77 +590,22 @@ def cpu_baseline(w, inp, ad, logits):
             "sample": f"{k} query tokens of the workload (all heads, adaLN, unmask of that position), {el:.1f} s"}
 
 
-def run_kernel_only(args):
-    """Eager launches of one kernel of the step on the workload (for ncu captures): warmup + steps
-    launches, one input set, no graph; prints the mean launch time from CUDA events."""
-    import torch
-    from denoiser_attention_b200 import api, build, synth
-    build.build()
-    dev = torch.device("cuda", 0)
-    w = synth.workload(args.workload)
-    inp, ad, logits = host_inputs(w)
-    B, S = w.attn.batch, w.attn.block_size
-    q, kb, vb = inp.q.to(dev), inp.k_blk.to(dev), inp.v_blk.to(dev)
-    kc, vc, lens = inp.k_ctx.to(dev), inp.v_ctx.to(dev), inp.ctx_lens.to(dev)
-    table = None if inp.page_table is None else inp.page_table.to(dev)
-    lg = logits.to(dev)
-    tokens = torch.full((B, S), 3, dtype=torch.int32, device=dev)
-    masked = torch.ones((B, S), dtype=torch.uint8, device=dev)
-    weights = {k: getattr(ad, k).to(dev) for k in ("w1", "b1", "w2", "b2", "w3", "b3", "layer_emb", "norm_w")}
-    tau, h, f = ad.tau.to(dev), ad.h.to(dev), ad.f.to(dev)
-    out = torch.empty_like(q)
-
-    if args.kernel == "lmhead":
-        # the fused LM head + unmask at the decode shape: hidden states [8][16][2048], W [131072][2048]
-        gen = torch.Generator(device=dev).manual_seed(w.seed)
-        D, Vh = 2048, 131072
-        xh = torch.randn((B, S, D), device=dev, generator=gen).to(torch.bfloat16)
-        wh = (torch.randn((Vh, D), device=dev, generator=gen) * (3.0 / D ** 0.5)).to(torch.bfloat16)
-
-    def once():
-        if args.kernel == "lmhead":
-            api.lmhead_unmask_step(xh, wh, tokens, masked, gamma=w.gamma, want_conf=False)
-        elif args.kernel == "attn":
-            api.denoise_attention(q, kb, vb, kc, vc, lens, page_table=table, page_size=w.attn.page_size,
-                                  ctx_stride=inp.ctx_stride, out=out)
-        elif args.kernel == "unmask":
-            api.unmask_step(lg, tokens, masked, gamma=w.gamma, want_conf=False)
-        else:
-            mod = api.adaln_cond(tau, weights["w1"], weights["b1"], weights["w2"], weights["b2"], weights["w3"],
-                                 weights["b3"], weights["layer_emb"])
-            api.adaln_norm_modulate(h, weights["norm_w"], mod)
-            api.adaln_gated_residual(h, f, mod)
-
-    for _ in range(args.warmup):
-        once()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        once()
-    e1.record()
-    torch.cuda.synchronize()
-    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "launches": args.steps,
-                      "mean_us_incl_host_gaps": 1e3 * e0.elapsed_time(e1) / args.steps}))
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--kernel", choices=["attn", "unmask", "adaln", "lmhead"], default=None,
-                    help="profiling mode: eager launches of one kernel only (not a bench line)")
-    ap.add_argument("--workload", default=WORKLOAD, help="workload of the --kernel profiling mode")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="the step's workload (default: the batch-generation workload, the headline)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the extra keys (decode step, attention per workload, block-sweep unmask table)")
     ap.add_argument("--schedule", choices=list(SCHEDULE_TEXT), default="branches",
                     help="how the step's three branches are put on streams")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.kernel:
-        run_kernel_only(args)
-    elif args.impl == "reference":
+    if args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -41,8 +41,11 @@ EXPORTED = [
     "tt_unmask_workspace_bytes", "tt_unmask_step", "tt_unmask_step_noalloc", "tt_block_tau",
     "tt_kv_append_workspace_bytes", "tt_kv_append",
     "tt_lmhead_unmask_workspace_bytes", "tt_lmhead_unmask_step",
+    "tt_linear_schedule_keep", "tt_probe_bounded_wait",
     "tt_get_device_error",
 ]
+
+TT_DETAIL_WAIT_PROBE = 0x1FF
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -56,7 +59,7 @@ class AttnArgs(ctypes.Structure):
         ("q", _vp), ("k_blk", _vp), ("v_blk", _vp), ("k_ctx", _vp), ("v_ctx", _vp),
         ("ctx_lens", _vp), ("page_table", _vp),
         ("page_size", _i32), ("max_pages_per_seq", _i32), ("num_pages", _i32), ("ctx_stride", _i32),
-        ("out", _vp), ("lse", _vp),
+        ("out", _vp), ("lse", _vp), ("skip_if", _vp),
     ]
 
 
@@ -66,6 +69,7 @@ class AdalnArgs(ctypes.Structure):
         ("mlp_width", _i32), ("dtype", _i32), ("eps", _f32),
         ("tau", _vp), ("w1", _vp), ("b1", _vp), ("w2", _vp), ("b2", _vp), ("w3", _vp), ("b3", _vp),
         ("layer_emb", _vp), ("mod", _vp), ("h", _vp), ("norm_w", _vp), ("f", _vp), ("out", _vp),
+        ("skip_if", _vp),
     ]
 
 
@@ -75,6 +79,7 @@ class UnmaskArgs(ctypes.Structure):
         ("gamma", _f32), ("inv_temperature", _f32), ("mask_token_id", _i32), ("exclude_mask_token", _i32),
         ("remaining_steps", _i32), ("tokens", _vp), ("is_masked", _vp), ("conf", _vp), ("argmax", _vp),
         ("n_committed", _vp), ("n_masked", _vp), ("sampler", _i32), ("keep_masked", _i32),
+        ("noise_steps", _i32), ("noise_step", _i32), ("skip_if", _vp), ("all_done", _vp),
     ]
 
 
@@ -93,7 +98,7 @@ class LmheadUnmaskArgs(ctypes.Structure):
         ("x", _vp), ("w", _vp), ("gamma", _f32), ("inv_temperature", _f32), ("mask_token_id", _i32),
         ("exclude_mask_token", _i32), ("remaining_steps", _i32), ("tokens", _vp), ("is_masked", _vp),
         ("conf", _vp), ("argmax", _vp), ("n_committed", _vp), ("n_masked", _vp), ("sampler", _i32),
-        ("keep_masked", _i32),
+        ("keep_masked", _i32), ("noise_steps", _i32), ("noise_step", _i32), ("skip_if", _vp), ("all_done", _vp),
     ]
 
 
@@ -132,8 +137,12 @@ def lib() -> ctypes.CDLL:
         L.tt_kv_append_workspace_bytes.argtypes = [ctypes.POINTER(KvAppendArgs)]
         L.tt_kv_append.restype = ctypes.c_int
         L.tt_kv_append.argtypes = [ctypes.POINTER(KvAppendArgs), _vp, ctypes.c_size_t, _vp]
-        L.tt_block_tau.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp]
+        L.tt_block_tau.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp]
         L.tt_unmask_step_noalloc.argtypes = [ctypes.POINTER(UnmaskArgs), _vp]
+        L.tt_linear_schedule_keep.restype = ctypes.c_int32
+        L.tt_linear_schedule_keep.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+        L.tt_probe_bounded_wait.restype = ctypes.c_int
+        L.tt_probe_bounded_wait.argtypes = [_vp, ctypes.c_uint32, _vp]
         L.tt_get_device_error.restype = ctypes.c_int
         L.tt_get_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
@@ -180,7 +189,7 @@ def status_string(status: int) -> str:
 
 # ------------------------------------------------------------------------------------------ attn
 def attn_args(q, k_blk, v_blk, k_ctx, v_ctx, ctx_lens, out, page_table=None, page_size=0,
-              ctx_stride=0, softmax_scale=1.0, lse=None) -> AttnArgs:
+              ctx_stride=0, softmax_scale=1.0, lse=None, skip_if=None) -> AttnArgs:
     B, S, Hq, d = q.shape
     Hkv = k_blk.shape[2]
     a = AttnArgs()
@@ -199,6 +208,7 @@ def attn_args(q, k_blk, v_blk, k_ctx, v_ctx, ctx_lens, out, page_table=None, pag
         a.ctx_stride = int(ctx_stride) if ctx_stride else int(k_ctx.shape[1])
     a.out = _ptr(out)
     a.lse = _ptr(lse)
+    a.skip_if = _ptr(skip_if)
     return a
 
 
@@ -215,13 +225,14 @@ def tt_denoise_attn(args: AttnArgs, workspace: torch.Tensor, stream=None) -> Non
 def adaln_args(op: int, *, batch: int, hidden: int, block_size: int = 0, freq_dim: int = 256,
                mlp_width: int = 256, dtype=torch.float32, eps: float = 1e-5, tau=None, w1=None, b1=None,
                w2=None, b2=None, w3=None, b3=None, layer_emb=None, mod=None, h=None, norm_w=None, f=None,
-               out=None) -> AdalnArgs:
+               out=None, skip_if=None) -> AdalnArgs:
     a = AdalnArgs()
     a.op, a.batch, a.block_size, a.hidden = op, batch, block_size, hidden
     a.freq_dim, a.mlp_width, a.dtype, a.eps = freq_dim, mlp_width, _dtype_code(dtype), float(eps)
     a.tau, a.w1, a.b1, a.w2, a.b2 = _ptr(tau), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)
     a.w3, a.b3, a.layer_emb, a.mod = _ptr(w3), _ptr(b3), _ptr(layer_emb), _ptr(mod)
     a.h, a.norm_w, a.f, a.out = _ptr(h), _ptr(norm_w), _ptr(f), _ptr(out)
+    a.skip_if = _ptr(skip_if)
     return a
 
 
@@ -238,9 +249,11 @@ def tt_adaln_modulate(args: AdalnArgs, workspace: torch.Tensor, stream=None) -> 
 # ------------------------------------------------------------------------------------------ unmask
 def unmask_args(logits, tokens, is_masked, n_committed, n_masked, *, gamma: float, inv_temperature: float = 1.0,
                 mask_token_id: int = 3, exclude_mask_token: bool = False, remaining_steps: int = 0,
-                conf=None, argmax=None, keep_masked: Optional[int] = None) -> UnmaskArgs:
-    """keep_masked=None: the confidence-threshold sampler; an int: the predict-and-noise sampler
-    keeping that many positions masked."""
+                conf=None, argmax=None, keep_masked: Optional[int] = None,
+                noise_schedule: Optional[tuple] = None, skip_if=None, all_done=None) -> UnmaskArgs:
+    """keep_masked=None and noise_schedule=None: the confidence-threshold sampler; keep_masked=k:
+    the predict-and-noise sampler keeping k positions masked; noise_schedule=(T, r): the
+    predict-and-noise sampler at step r of T of the linear schedule (the library derives k)."""
     B, S, V = logits.shape
     a = UnmaskArgs()
     a.batch, a.block_size, a.vocab, a.dtype = B, S, V, _dtype_code(logits.dtype)
@@ -250,11 +263,30 @@ def unmask_args(logits, tokens, is_masked, n_committed, n_masked, *, gamma: floa
     a.tokens, a.is_masked = _ptr(tokens), _ptr(is_masked)
     a.conf, a.argmax = _ptr(conf), _ptr(argmax)
     a.n_committed, a.n_masked = _ptr(n_committed), _ptr(n_masked)
-    if keep_masked is None:
-        a.sampler, a.keep_masked = TT_SAMPLER_CONFIDENCE, 0
-    else:
-        a.sampler, a.keep_masked = TT_SAMPLER_PREDICT_NOISE, int(keep_masked)
+    _set_sampler(a, keep_masked, noise_schedule)
+    a.skip_if, a.all_done = _ptr(skip_if), _ptr(all_done)
     return a
+
+
+def _set_sampler(a, keep_masked, noise_schedule):
+    if keep_masked is not None and noise_schedule is not None:
+        raise ValueError("give keep_masked or noise_schedule, not both")
+    a.sampler, a.keep_masked, a.noise_steps, a.noise_step = TT_SAMPLER_CONFIDENCE, 0, 0, 0
+    if keep_masked is not None:
+        a.sampler, a.keep_masked = TT_SAMPLER_PREDICT_NOISE, int(keep_masked)
+    elif noise_schedule is not None:
+        a.sampler = TT_SAMPLER_PREDICT_NOISE
+        a.noise_steps, a.noise_step = int(noise_schedule[0]), int(noise_schedule[1])
+
+
+def tt_linear_schedule_keep(block_size: int, steps: int, step: int) -> int:
+    """Positions left masked after step `step` of `steps` (linear schedule); -1 if invalid."""
+    return int(lib().tt_linear_schedule_keep(int(block_size), int(steps), int(step)))
+
+
+def tt_probe_bounded_wait(workspace: torch.Tensor, limit_us: int, stream=None) -> None:
+    """Runs the library's bounded device wait on a barrier nothing arrives on (diagnostic)."""
+    _check(lib().tt_probe_bounded_wait(_ptr(workspace), int(limit_us), _stream(stream)), "tt_probe_bounded_wait")
 
 
 def tt_unmask_workspace_bytes(args: UnmaskArgs) -> int:
@@ -271,19 +303,20 @@ def tt_unmask_step_noalloc(args: UnmaskArgs, stream=None) -> None:
     _check(lib().tt_unmask_step_noalloc(ctypes.byref(args), _stream(stream)), "tt_unmask_step_noalloc")
 
 
-def tt_block_tau(is_masked: torch.Tensor, tau: torch.Tensor, stream=None) -> None:
-    """tau[b] = masked positions of sequence b / S, on the device."""
+def tt_block_tau(is_masked: torch.Tensor, tau: torch.Tensor, stream=None, skip_if=None) -> None:
+    """tau[b] = masked positions of sequence b / S, on the device (nothing when *skip_if != 0)."""
     if is_masked.dtype != torch.uint8 or tau.dtype != torch.float32:
         raise ValueError("is_masked must be uint8 and tau float32")
     Bn, S = is_masked.shape
-    _check(lib().tt_block_tau(_ptr(is_masked), Bn, S, _ptr(tau), _stream(stream)), "tt_block_tau")
+    _check(lib().tt_block_tau(_ptr(is_masked), Bn, S, _ptr(tau), _ptr(skip_if), _stream(stream)), "tt_block_tau")
 
 
 # ------------------------------------------------------------------------------- LM head + unmask
 def lmhead_unmask_args(x, w, tokens, is_masked, n_committed, n_masked, *, gamma: float,
                        inv_temperature: float = 1.0, mask_token_id: int = 3, exclude_mask_token: bool = False,
                        remaining_steps: int = 0, conf=None, argmax=None,
-                       keep_masked: Optional[int] = None) -> LmheadUnmaskArgs:
+                       keep_masked: Optional[int] = None, noise_schedule: Optional[tuple] = None,
+                       skip_if=None, all_done=None) -> LmheadUnmaskArgs:
     B, S, D = x.shape
     a = LmheadUnmaskArgs()
     a.batch, a.block_size, a.hidden, a.vocab, a.dtype = B, S, D, int(w.shape[0]), _dtype_code(x.dtype)
@@ -292,10 +325,8 @@ def lmhead_unmask_args(x, w, tokens, is_masked, n_committed, n_masked, *, gamma:
     a.mask_token_id, a.exclude_mask_token, a.remaining_steps = int(mask_token_id), int(bool(exclude_mask_token)), int(remaining_steps)
     a.tokens, a.is_masked, a.conf, a.argmax = _ptr(tokens), _ptr(is_masked), _ptr(conf), _ptr(argmax)
     a.n_committed, a.n_masked = _ptr(n_committed), _ptr(n_masked)
-    if keep_masked is None:
-        a.sampler, a.keep_masked = TT_SAMPLER_CONFIDENCE, 0
-    else:
-        a.sampler, a.keep_masked = TT_SAMPLER_PREDICT_NOISE, int(keep_masked)
+    _set_sampler(a, keep_masked, noise_schedule)
+    a.skip_if, a.all_done = _ptr(skip_if), _ptr(all_done)
     return a
 
 

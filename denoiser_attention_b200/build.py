@@ -20,7 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtt_denoise.so")
-SOURCES = ["tt_api.cu", "unmask.cu", "adaln.cu", "attn_simt.cu", "attn_tc.cu", "kv_append.cu"]
+SOURCES = ["tt_api.cu", "unmask.cu", "adaln.cu", "attn_tf32.cu", "attn_tc.cu", "kv_append.cu"]
 HEADERS = ["tt_common.cuh", "tt_internal.h", os.path.join("..", "..", "include", "tt_denoise.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

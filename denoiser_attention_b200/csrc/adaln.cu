@@ -3,12 +3,14 @@
 // PixArt-alpha: one global MLP from the diffusion time to shared shift/scale/gate, plus a learned
 // per-layer embedding).
 //
-//   COND             tau -> mod[B][3][D]   three batched-GEMV launches (F->W, W->W, W->3D), each
-//                                          reading its weight rows once for every sequence
+//   COND             tau -> mod[B][3][D]   two launches: per sequence the sinusoid and the two
+//                                          W-wide layers; then the W->3D layer tiled over 32-row
+//                                          slices of W3, each read once for the whole batch
 //   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one CTA per token row
 //   GATED_RESIDUAL   h + gate * f: a vectorised elementwise pass
 // All arithmetic is fp32 (the timestep sinusoid in fp64); bf16 tensors are widened on load and
 // rounded to nearest on store.
+#include <algorithm>
 #include <cmath>
 
 #include "tt_common.cuh"
@@ -25,14 +27,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-
-// Batched GEMV for the three layers of the conditioning MLP:
-//   y[b][o] = act(sum_i W[o][i] x[b][i] + bias[o]) (+ extra[o])
-// Each warp holds R rows of W in registers (float4 per lane, KW of them per row) and applies them
-// to every batch row; batch rows are staged in shared memory in chunks. kPhi: x is the timestep
-// sinusoid phi(tau_b), computed in the kernel (IN = F); otherwise x is read from global memory.
-constexpr int kGemvBatchChunk = 8;
-constexpr int kGemvMaxIn = 1024;
 
 // phi(tau) = [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)). The angle (up to
 // 1000 rad) is formed and reduced modulo 2 pi in double, so the single-precision sincos only sees
@@ -52,90 +46,120 @@ __device__ __forceinline__ void phi_row(float tau, int F, float* dst, int tid, i
   }
 }
 
-template <int KW, int R, bool kPhi, bool kSilu>
-__global__ void __launch_bounds__(kAdalnThreads) adaln_gemv_kernel(const float* __restrict__ Wt,
-                                                                   const float* __restrict__ bias,
-                                                                   const float* __restrict__ extra,
-                                                                   const float* __restrict__ x, int B, int IN,
-                                                                   int OUT, float* __restrict__ y) {
-  __shared__ __align__(16) float s_x[kGemvBatchChunk * kGemvMaxIn];
-  pdl_trigger();
-  pdl_wait();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int o0 = (blockIdx.x * (kAdalnThreads / 32) + warp) * R;
-  float4 w[R][KW];
-  float bo[R];
+constexpr int kMaxWidth = 1024;   // F and W bound (host-validated)
+
+// y[o] = act(W[o, :] . x + bias[o]) for o < OUT, x in shared memory; each warp takes four rows at
+// a time (four independent dot products and reductions in flight), lanes stride the row in float4.
+template <bool kSilu>
+__device__ __forceinline__ void cta_gemv(const float* __restrict__ Wt, const float* __restrict__ bias,
+                                         const float* x, int IN, int OUT, float* y) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int o0 = warp * 4; o0 < OUT; o0 += nwarps * 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = lane * 4; i < IN; i += 128) {
+      const float4 xv = *reinterpret_cast<const float4*>(x + i);
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int o = o0 + r;
-    bo[r] = 0.f;
-    if (o < OUT) bo[r] = bias[o] + (extra ? extra[o] : 0.f);
-#pragma unroll
-    for (int k = 0; k < KW; ++k) {
-      const int i = (lane + 32 * k) * 4;
-      w[r][k] = (o < OUT && i < IN) ? *reinterpret_cast<const float4*>(Wt + (size_t)o * IN + i)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  }
-  for (int b0 = 0; b0 < B; b0 += kGemvBatchChunk) {
-    const int nb = min(kGemvBatchChunk, B - b0);
-    __syncthreads();
-    if (kPhi) {
-      for (int bb = 0; bb < nb; ++bb) phi_row(x[b0 + bb], IN, s_x + bb * IN, threadIdx.x, blockDim.x);
-    } else {
-      for (int i = threadIdx.x; i < nb * IN; i += blockDim.x) s_x[i] = x[(size_t)b0 * IN + i];
-    }
-    __syncthreads();
-    for (int bb = 0; bb < nb; ++bb) {
-      float acc[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) acc[r] = 0.f;
-#pragma unroll
-      for (int k = 0; k < KW; ++k) {
-        const int i = (lane + 32 * k) * 4;
-        if (i < IN) {
-          const float4 xv = *reinterpret_cast<const float4*>(s_x + bb * IN + i);
-#pragma unroll
-          for (int r = 0; r < R; ++r)
-            acc[r] = fmaf(w[r][k].x, xv.x, fmaf(w[r][k].y, xv.y, fmaf(w[r][k].z, xv.z, fmaf(w[r][k].w, xv.w, acc[r]))));
+      for (int r = 0; r < 4; ++r) {
+        if (o0 + r < OUT) {
+          const float4 wv = *reinterpret_cast<const float4*>(Wt + (size_t)(o0 + r) * IN + i);
+          acc[r] = fmaf(wv.x, xv.x, fmaf(wv.y, xv.y, fmaf(wv.z, xv.z, fmaf(wv.w, xv.w, acc[r]))));
         }
       }
+    }
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float v = warp_sum(acc[r]) + bo[r];
-        if (lane == 0 && o0 + r < OUT) y[(size_t)(b0 + bb) * OUT + o0 + r] = kSilu ? silu_f(v) : v;
-      }
+    for (int r = 0; r < 4; ++r) acc[r] = warp_sum(acc[r]);
+    if (lane < 4 && o0 + lane < OUT) {
+      const float v = (lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3]) + bias[o0 + lane];
+      y[o0 + lane] = kSilu ? silu_f(v) : v;
     }
   }
 }
 
-template <bool kPhi, bool kSilu>
-static void launch_gemv(const float* Wt, const float* bias, const float* extra, const float* x, int B, int IN, int OUT,
-                        float* y, cudaStream_t stream) {
-  const int kw = (IN + 127) / 128;   // float4 per lane per row
-  const int warps = kAdalnThreads / 32;
-  // small layers: one row per warp (more CTAs); wide ones: four rows per warp
-  const bool wide = OUT > 2048;
-  if (kw <= 1) {
-    if (wide)
-      launch_pdl(adaln_gemv_kernel<1, 4, kPhi, kSilu>, dim3((OUT + warps * 4 - 1) / (warps * 4)), dim3(kAdalnThreads),
-                 0, stream, Wt, bias, extra, x, B, IN, OUT, y);
-    else
-      launch_pdl(adaln_gemv_kernel<1, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0,
-                 stream, Wt, bias, extra, x, B, IN, OUT, y);
-  } else if (kw <= 2) {
-    if (wide)
-      launch_pdl(adaln_gemv_kernel<2, 4, kPhi, kSilu>, dim3((OUT + warps * 4 - 1) / (warps * 4)), dim3(kAdalnThreads),
-                 0, stream, Wt, bias, extra, x, B, IN, OUT, y);
-    else
-      launch_pdl(adaln_gemv_kernel<2, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0,
-                 stream, Wt, bias, extra, x, B, IN, OUT, y);
-  } else if (kw <= 4) {
-    launch_pdl(adaln_gemv_kernel<4, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0, stream,
-               Wt, bias, extra, x, B, IN, OUT, y);
-  } else {
-    launch_pdl(adaln_gemv_kernel<8, 1, kPhi, kSilu>, dim3((OUT + warps - 1) / warps), dim3(kAdalnThreads), 0, stream,
-               Wt, bias, extra, x, B, IN, OUT, y);
+// COND, first launch: one CTA per sequence b computes a2[b] = SiLU(W2 SiLU(W1 phi(tau_b) + b1) + b2).
+__global__ void __launch_bounds__(kAdalnThreads) adaln_hidden_kernel(const float* __restrict__ tau,
+                                                                     const float* __restrict__ w1,
+                                                                     const float* __restrict__ b1,
+                                                                     const float* __restrict__ w2,
+                                                                     const float* __restrict__ b2, int F, int W,
+                                                                     float* __restrict__ a2,
+                                                                     const int32_t* skip_if) {
+  __shared__ __align__(16) float s_phi[kMaxWidth];
+  __shared__ __align__(16) float s_a1[kMaxWidth];
+  pdl_trigger();
+  pdl_wait();
+  if (skip_requested(skip_if)) return;
+  const int b = blockIdx.x;
+  phi_row(tau[b], F, s_phi, threadIdx.x, blockDim.x);
+  __syncthreads();
+  cta_gemv<true>(w1, b1, s_phi, F, W, s_a1);
+  __syncthreads();
+  cta_gemv<true>(w2, b2, s_a1, W, W, a2 + (size_t)b * W);
+}
+
+// COND, second launch: mod[b][o] = W3[o, :] . a2[b] + b3[o] + layer_emb[o] for o < 3D. A CTA
+// owns 32 rows of W3 (in shared memory, rows padded by 4 floats so that the quarter-warp float4
+// reads of 8 rows hit distinct banks) and every sequence: lane = row, warp = a group of sequences
+// whose a2 rows are read as broadcasts; chunks of up to 64 sequences at a time (fewer for wide W,
+// so that the chunk and the W3 slice fit in shared memory).
+constexpr int kOutRows = 32;
+constexpr int kOutSeqChunk = 64;
+inline int out_seq_chunk(int W) { return W <= 256 ? 64 : (W <= 512 ? 32 : 16); }
+inline size_t out_smem_bytes(int W) {
+  return sizeof(float) * ((size_t)kOutRows * (W + 4) + (size_t)out_seq_chunk(W) * W);
+}
+
+__global__ void __launch_bounds__(kAdalnThreads) adaln_out_kernel(const float* __restrict__ w3,
+                                                                  const float* __restrict__ b3,
+                                                                  const float* __restrict__ emb,
+                                                                  const float* __restrict__ a2, int B, int W,
+                                                                  int OUT, int chunk, float* __restrict__ mod,
+                                                                  const int32_t* skip_if) {
+  extern __shared__ __align__(16) float s_dyn[];
+  const int WP = W + 4;
+  float* s_w = s_dyn;                          // [32][W + 4]
+  float* s_a = s_dyn + kOutRows * WP;          // [chunk][W]
+  pdl_trigger();
+  pdl_wait();
+  if (skip_requested(skip_if)) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int o0 = blockIdx.x * kOutRows;
+  const int nrow = min(kOutRows, OUT - o0);
+  const int wv = W / 4;
+  for (int i = threadIdx.x; i < kOutRows * wv; i += blockDim.x) {
+    const int r = i / wv, c = i - r * wv;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < nrow) v = reinterpret_cast<const float4*>(w3 + (size_t)(o0 + r) * W)[c];
+    *reinterpret_cast<float4*>(s_w + r * WP + 4 * c) = v;
+  }
+  const int o = o0 + lane;
+  const float add = (lane < nrow) ? b3[o] + emb[o] : 0.f;
+  for (int c0 = 0; c0 < B; c0 += chunk) {
+    const int nb = min(chunk, B - c0);
+    __syncthreads();   // the previous chunk is consumed (and, the first time, s_w is written)
+    for (int i = threadIdx.x; i < nb * wv; i += blockDim.x)
+      reinterpret_cast<float4*>(s_a)[i] = reinterpret_cast<const float4*>(a2 + (size_t)c0 * W)[i];
+    __syncthreads();
+    float acc[kOutSeqChunk / 8];
+#pragma unroll
+    for (int i = 0; i < kOutSeqChunk / 8; ++i) acc[i] = 0.f;
+    for (int k = 0; k < W; k += 4) {
+      const float4 w = *reinterpret_cast<const float4*>(s_w + lane * WP + k);
+#pragma unroll
+      for (int i = 0; i < kOutSeqChunk / 8; ++i) {
+        const int bb = warp + 8 * i;
+        if (bb < nb) {
+          const float4 x = *reinterpret_cast<const float4*>(s_a + bb * W + k);
+          acc[i] = fmaf(w.x, x.x, fmaf(w.y, x.y, fmaf(w.z, x.z, fmaf(w.w, x.w, acc[i]))));
+        }
+      }
+    }
+    if (lane < nrow) {
+#pragma unroll
+      for (int i = 0; i < kOutSeqChunk / 8; ++i) {
+        const int bb = warp + 8 * i;
+        if (bb < nb) mod[(size_t)(c0 + bb) * OUT + o] = acc[i] + add;
+      }
+    }
   }
 }
 
@@ -180,10 +204,12 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_norm_modulate_kernel(cons
                                                                             const float* __restrict__ norm_w,
                                                                             const float* __restrict__ mod,
                                                                             int S, int D, float eps,
-                                                                            void* __restrict__ out) {
+                                                                            void* __restrict__ out,
+                                                                            const int32_t* skip_if) {
   constexpr int N = Io<T>::kN;
   pdl_trigger();
   pdl_wait();
+  if (skip_requested(skip_if)) return;
   const int row = blockIdx.x;
   const int b = row / S;
   const int nv = D / N;
@@ -223,10 +249,11 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_gated_residual_kernel(con
                                                                              const void* __restrict__ f,
                                                                              const float* __restrict__ mod,
                                                                              int S, int D, size_t nvec,
-                                                                             void* out) {
+                                                                             void* out, const int32_t* skip_if) {
   constexpr int N = Io<T>::kN;
   pdl_trigger();
   pdl_wait();
+  if (skip_requested(skip_if)) return;
   const int nv_row = D / N;
   for (size_t v = blockIdx.x * (size_t)blockDim.x + threadIdx.x; v < nvec; v += (size_t)gridDim.x * blockDim.x) {
     const size_t row = v / nv_row;
@@ -243,27 +270,40 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_gated_residual_kernel(con
 }
 
 size_t adaln_workspace_bytes(const tt_adaln_args_t* a) {
-  if (a->op == TT_ADALN_COND) return kHeaderBytes + 2 * sizeof(float) * (size_t)a->batch * a->mlp_width;
+  if (a->op == TT_ADALN_COND) return kHeaderBytes + sizeof(float) * (size_t)a->batch * a->mlp_width;
   return kHeaderBytes;
 }
 
 int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
   const int B = a->batch, D = a->hidden;
   if (a->op == TT_ADALN_COND) {
-    float* a1 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
-    float* a2 = a1 + (size_t)B * a->mlp_width;
-    const int F = a->freq_dim, W = a->mlp_width;
-    launch_gemv<true, true>(a->w1, a->b1, nullptr, a->tau, B, F, W, a1, stream);
-    launch_gemv<false, true>(a->w2, a->b2, nullptr, a1, B, W, W, a2, stream);
-    launch_gemv<false, false>(a->w3, a->b3, a->layer_emb, a2, B, W, 3 * D, a->mod, stream);
+    float* a2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+    const int F = a->freq_dim, W = a->mlp_width, OUT = 3 * D;
+    launch_pdl(adaln_hidden_kernel, dim3(B), dim3(kAdalnThreads), 0, stream, a->tau, a->w1, a->b1, a->w2, a->b2, F,
+               W, a2, a->skip_if);
+    const size_t smem = out_smem_bytes(W);
+    static unsigned long long attr_done = 0;   // bit per device ordinal (< 64): the opt-in for W up to 1024
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+      size_t max_smem = 0;
+      for (int w = 256; w <= kMaxWidth; w *= 2) max_smem = std::max(max_smem, out_smem_bytes(w));
+      if (cudaFuncSetAttribute(adaln_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem) !=
+          cudaSuccess)
+        return TT_ERR_CUDA;
+      __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
+    }
+    launch_pdl(adaln_out_kernel, dim3((OUT + kOutRows - 1) / kOutRows), dim3(kAdalnThreads), smem, stream, a->w3,
+               a->b3, a->layer_emb, a2, B, W, OUT, out_seq_chunk(W), a->mod, a->skip_if);
   } else if (a->op == TT_ADALN_NORM_MODULATE) {
     const int rows = B * a->block_size;
     if (a->dtype == TT_BF16)
       launch_pdl(adaln_norm_modulate_kernel<__nv_bfloat16>, dim3(rows), dim3(kAdalnThreads), 0, stream, a->h,
-                 a->norm_w, (const float*)a->mod, a->block_size, D, a->eps, a->out);
+                 a->norm_w, (const float*)a->mod, a->block_size, D, a->eps, a->out, a->skip_if);
     else
       launch_pdl(adaln_norm_modulate_kernel<float>, dim3(rows), dim3(kAdalnThreads), 0, stream, a->h, a->norm_w,
-                 (const float*)a->mod, a->block_size, D, a->eps, a->out);
+                 (const float*)a->mod, a->block_size, D, a->eps, a->out, a->skip_if);
   } else {
     const int N = (a->dtype == TT_BF16) ? 8 : 4;
     const size_t nvec = (size_t)B * a->block_size * D / N;
@@ -273,10 +313,10 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
     if (grid == 0) grid = 1;
     if (a->dtype == TT_BF16)
       launch_pdl(adaln_gated_residual_kernel<__nv_bfloat16>, dim3((unsigned)grid), dim3(kAdalnThreads), 0, stream,
-                 a->h, a->f, (const float*)a->mod, a->block_size, D, nvec, a->out);
+                 a->h, a->f, (const float*)a->mod, a->block_size, D, nvec, a->out, a->skip_if);
     else
       launch_pdl(adaln_gated_residual_kernel<float>, dim3((unsigned)grid), dim3(kAdalnThreads), 0, stream, a->h,
-                 a->f, (const float*)a->mod, a->block_size, D, nvec, a->out);
+                 a->f, (const float*)a->mod, a->block_size, D, nvec, a->out, a->skip_if);
   }
   return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }

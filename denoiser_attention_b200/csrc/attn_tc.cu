@@ -5,33 +5,35 @@
 // tiles of 128 tokens followed by one tile holding the S block tokens. Its query rows are the
 // G query heads of the kv head times the S block positions, packed as rows m = s * G + g and cut
 // into "query tiles" of at most 128 rows (one tcgen05 M=128 MMA). nq = number of query tiles per
-// group. The CTAs are organised in teams of nq; all groups' key tiles are laid end to end and cut
-// into ranges, one per team, computed on the device from ctx_lens (no host knowledge of the
-// lengths): either Pe = min(teams, tiles) equal ranges (ragged contexts balance to within a tile),
-// or, when that costs at most kSegPenaltyTiles more per team, ranges that never cross a group
-// boundary (each group cut into near-equal chunks), which spares the teams a second segment. Within a
-// team, CTA q handles query tile q of every group its range touches, and the team's CTAs walk the
-// same key tiles at the same time, so each K/V tile comes from HBM once and the other reads of it
-// hit L2. A CTA that holds a whole group writes its rows of the output directly; a group cut
-// between teams leaves a normalised partial (O_j / l_j and the log2-sum-exp) per CTA, and a second,
-// wide kernel merges them (flash-decoding combine), launched as a programmatic dependent.
+// group. A CTA holds two query tiles of a group (one for odd nq's last CTA), so the CTAs form
+// teams of ceil(nq / 2); all groups' key tiles are laid end to end and cut into ranges, one per
+// team, computed on the device from ctx_lens (no host knowledge of the lengths): either
+// Pe = min(teams, tiles) equal ranges (ragged contexts balance to within a tile), or, when that
+// costs at most kSegPenaltyTiles more per team, ranges that never cross a group boundary (each
+// group cut into near-equal chunks), which spares the teams a second segment. For the common
+// G * S = 256 one CTA holds the whole group: every K/V tile is staged once per group. A CTA that
+// holds a whole group writes its rows of the output directly; a group cut between teams leaves a
+// normalised partial (O_j / l_j and the log2-sum-exp) per query tile, and a second, wide kernel
+// merges them (flash-decoding combine), launched as a programmatic dependent.
 //
-// Inside a CTA (320 threads):
-//   warp 0     TMA producer: the Q tile of the group, then K and V tiles of 128 tokens into a
-//              2-stage ring with separate K and V barriers (128B-swizzled boxes; no multicast)
-//   warp 1     MMA issuer (one thread): S[f%2] = Q K^T (M=128, N=128, K=128, both operands from
-//              shared memory) for tile f+1 is issued before O += P V for tile f (A = P from TMEM,
-//              B = V), so the tensor pipe computes the next scores while the softmax runs
-//   warps 2-9  softmax + epilogue: a thread owns query row = its TMEM lane (lane quadrant =
-//              warp % 4) and one half of the 128 key columns (warps 2-5 keys 0-63, warps 6-9
-//              keys 64-127); the two threads of a row exchange their partial maxima and sums
-//              through shared memory (bounded mbarrier handshakes)
-// TMEM (512 columns allocated): O [0,128), S/P double buffer [128,256), [256,384); each thread
-// writes its 64 P values (bf16) over the first 32 columns of its own S columns, and the PV
-// product reads P from TMEM.
+// Inside a CTA (384 threads: warpgroup 0 load and MMA, warpgroups 1-2 softmax), two independent
+// softmax streams, one per query tile:
+//   warps 0, 2 TMA producers: warp 0 the CTA's query tiles of the group and the K tiles of 128
+//              tokens (3-stage ring), warp 2 the V tiles (2-stage ring), so that neither ring
+//              waits for the other (128B-swizzled boxes; no multicast)
+//   warp 1     MMA issuer (one thread): for stream j, S_j = Q_j K^T (M=128, N=128, K=128, both
+//              operands from shared memory) and O_j += P_j V (A = P_j from TMEM, B = V). Per key
+//              tile it issues PV_0(f), QK_0(f+1), PV_1(f), QK_1(f+1): while stream 0 runs its
+//              softmax on tile f+1 the tensor pipe works for stream 1, and the other way round
+//   warps 4-7  softmax + epilogue of stream 0, warps 8-11 of stream 1: a thread owns one query
+//              row (its TMEM lane; lane quadrant = warp % 4) and all 128 key columns of a tile,
+//              so the row maximum and sum need no exchange between threads
+// TMEM (512 columns): O_0 [0,128), O_1 [128,256), S_0 [256,384), S_1 [384,512); a thread writes
+// its row's 128 P values (bf16 pairs) over the first 64 columns of its S, which the PV product
+// reads as its A operand.
 // The softmax works in the exp2 domain with the scale folded in and computes P against the
-// running maximum; only when a tile's maximum exceeds it by more than 8 (P > 256) is the tile
-// redone against the new maximum and O rescaled (exact: numerator and denominator share the
+// running maximum; only when a tile's maximum exceeds it by more than 8 (P > 256) does the
+// base move to the tile maximum, with O rescaled (exact: numerator and denominator share the
 // stale maximum).
 #include <cstdio>
 #include <cuda.h>
@@ -46,20 +48,30 @@ namespace {
 
 constexpr int kD = 128;           // head dim handled by this kernel
 constexpr int kTile = 128;        // keys per tile
-constexpr int kStages = 2;        // K/V ring depth
-constexpr int kRows = 128;        // query rows per CTA (one M=128 MMA)
-constexpr int kThreads = 320;     // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int kKStages = 3;       // K ring depth
+constexpr int kVStages = 2;       // V ring depth
+constexpr bool kSplitProducers = true;   // V loads from their own thread (warp 2), K and Q from warp 0
+constexpr int kRows = 128;        // query rows per query tile (one M=128 MMA)
+constexpr int kStreams = 2;       // query tiles (softmax streams) per CTA
+// warpgroup 0: warp 0 TMA, warp 1 MMA (warps 2-3 idle); warpgroups 1-2: one softmax stream each
+constexpr int kThreads = 128 + kStreams * kRows;
+// Registers are handed out per warpgroup: the block launches with kLaunchRegs per thread, then the
+// producer warpgroup gives registers back and the two softmax warpgroups take them (the sum stays
+// within the launch pool: 128 * 88 + 256 * 208 = 384 * 168).
+constexpr int kLaunchRegs = 168, kProducerRegs = 88, kSoftmaxRegs = 208;
+static_assert(128 * kProducerRegs + 2 * 128 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS = 256;  // S_j at column kTmemS + 128 j, O_j at 128 j
 
 constexpr uint32_t kQBytesPerDh = kRows * 128;                 // 128 rows x 128 B = 16 KB
-constexpr uint32_t kQBytes = 2 * kQBytesPerDh;                 // 32 KB
+constexpr uint32_t kQBytes = 2 * kQBytesPerDh;                 // 32 KB per query tile
 constexpr uint32_t kKVBoxBytes = kTile * 128;                  // 128 rows x 128 B = 16 KB
 constexpr uint32_t kKBytesPerStage = 2 * kKVBoxBytes;          // 32 KB (two 64-dim boxes)
 constexpr uint32_t kSmemQ = 0;
-constexpr uint32_t kSmemK = kQBytes;
-constexpr uint32_t kSmemV = kSmemK + kStages * kKBytesPerStage;
-constexpr uint32_t kSmemBar = kSmemV + kStages * kKBytesPerStage;
-constexpr uint32_t kSmemBytes = kSmemBar + 4096 + 1024;        // barriers/scratch + alignment slack
+constexpr uint32_t kSmemK = kStreams * kQBytes;
+constexpr uint32_t kSmemV = kSmemK + kKStages * kKBytesPerStage;
+constexpr uint32_t kSmemBar = kSmemV + kVStages * kKBytesPerStage;
+constexpr uint32_t kSmemBytes = kSmemBar + 1024 + 1024;        // barriers + alignment slack
 
 constexpr int kMergeRows = 8;     // rows per merge CTA (one per warp)
 
@@ -99,29 +111,30 @@ struct TcParams {
   const int32_t* ctx_lens;
   const int32_t* page_table;
   int32_t B, S, Hq, Hkv, G;
-  int32_t nq, s_per_tile, groups, teams;
+  int32_t nq, nq2, s_per_tile, groups, teams;   // nq2 = CTAs per team = ceil(nq / 2)
   int32_t page_size, max_pages, num_pages, ctx_stride, paged;
   float scale_log2;   // softmax_scale * log2(e)
   __nv_bfloat16* out;
   float* lse;
   uint8_t* ws;
   size_t off_meta, off_crange, off_partials, off_lse;
+  const int32_t* skip_if;
 };
 
 struct Smem {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], pv_done;
-  uint64_t x_bar, l_bar;   // row-max and row-sum exchange between the two column halves
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[kStreams];   // S_j = Q_j K^T of the current tile is in TMEM
+  uint64_t p_full[kStreams];   // P_j of the current tile is in TMEM (and O_j rescaled)
+  uint64_t o_full[kStreams];   // O_j of the segment is complete
   uint64_t drain;
-  float xmax[2][2][kRows];  // [tile parity][column half][row]
-  float xsum[2][kRows];
   uint32_t tmem_base;
   int abort_flag;
   long long range_begin, range_end, total_tiles, p_eff;
   int u0;
   long long u0_start;
 };
+static_assert(sizeof(Smem) <= 1024, "barrier block");
 
 struct GroupInfo {
   int b, kvh, L, nctx, ntiles;
@@ -202,26 +215,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   Smem& sm = *reinterpret_cast<Smem*>(smem + kSmemBar);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int team = blockIdx.x / p.nq, qt = blockIdx.x % p.nq;
+  const int team = blockIdx.x / p.nq2;
+  const int qt0 = 2 * (blockIdx.x % p.nq2);              // this CTA's first query tile
+  const int nstreams = (qt0 + 1 < p.nq) ? 2 : 1;         // query tiles it holds
 
   // ---- 0. prologue that touches no input: barriers, TMEM, tensor-map prefetch. With a
   // programmatic launch it overlaps the previous kernel; inputs are read after pdl_wait().
   if (warp == 0 && lane == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&sm.k_full[i], 1);
       mbar_init(&sm.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.p_full[b], 2 * kRows);
+    for (int j = 0; j < kStreams; ++j) {
+      mbar_init(&sm.s_full[j], 1);
+      mbar_init(&sm.p_full[j], kRows);
+      mbar_init(&sm.o_full[j], 1);
     }
-    mbar_init(&sm.pv_done, 1);
-    mbar_init(&sm.x_bar, 2 * kRows);
-    mbar_init(&sm.l_bar, 2 * kRows);
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
     prefetch_tmap(&p.tm_q);
@@ -237,6 +252,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
   pdl_trigger();
   pdl_wait();
+  if (skip_requested(p.skip_if)) {
+    // early exit of a multi-step loop: nothing to do; release TMEM and leave
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(sm.tmem_base, kTmemCols);
+    }
+    return;
+  }
 
   // ---- 1. this team's tile range and the group where it starts (warp 0); CTA 0 also records,
   // per group, the teams that hold its partials (for the merge kernel).
@@ -378,37 +402,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const uint32_t sQ = smem_u32(smem + kSmemQ);
   const uint32_t sK = smem_u32(smem + kSmemK);
   const uint32_t sV = smem_u32(smem + kSmemV);
-  const int s_cnt = min(p.s_per_tile, p.S - qt * p.s_per_tile);   // block positions of this query tile
-  const int nrows = p.G * s_cnt;                                   // valid query rows (<= 128)
 
+  if (warp < 4) {
+    setmaxnreg_dec<kProducerRegs>();
   if (!has_work) {
     // nothing to do (more teams than tiles, or a CTA beyond the last full team)
-  } else if (warp == 0) {
-    // ======================= TMA producer
+  } else if (warp == 0 || (kSplitProducers && warp == 2)) {
+    // ======================= TMA producers: warp 0 loads the query tiles and the K ring, warp 2
+    // the V ring (warp 0 both when kSplitProducers is off), so that neither ring waits for the other
     if (lane == 0) {
+      const bool do_kq = (warp == 0);
+      const bool do_v = (warp == 2) || !kSplitProducers;
       SegWalk w;
       w.init(p, sm, hdr);
       long long f = 0;
       int qn = 0;
       bool ok = true;
-      const uint32_t q_bytes = 2u * 128u * (uint32_t)p.G * (uint32_t)p.s_per_tile;
+      const uint32_t q_bytes = 2u * 128u * (uint32_t)p.G * (uint32_t)p.s_per_tile;   // one query tile
       while (ok && !w.done()) {
         int kb, ke;
         w.segment(kb, ke);
         const GroupInfo& gi = w.gi;
-        if (qn > 0 && !mbar_wait_bounded(&sm.q_empty, (qn - 1) & 1, abort_flag)) {
-          fail(kDetailWaitQEmpty);
-          ok = false;
-          break;
+        if (do_kq) {
+          if (qn > 0 && !mbar_wait_bounded(&sm.q_empty, (qn - 1) & 1, abort_flag)) {
+            fail(kDetailWaitQEmpty);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.q_full, q_bytes * (uint32_t)nstreams);
+          for (int j = 0; j < nstreams; ++j) {
+            const int qrow = gi.b * p.S + (qt0 + j) * p.s_per_tile;
+            uint8_t* qdst = smem + kSmemQ + j * kQBytes;
+            tma_load_3d(qdst, &p.tm_q, &sm.q_full, 0, gi.kvh * p.G, qrow);
+            tma_load_3d(qdst + kQBytesPerDh, &p.tm_q, &sm.q_full, 64, gi.kvh * p.G, qrow);
+          }
+          ++qn;
         }
-        mbar_arrive_expect_tx(&sm.q_full, q_bytes);
-        const int qrow = gi.b * p.S + qt * p.s_per_tile;
-        tma_load_3d(smem + kSmemQ, &p.tm_q, &sm.q_full, 0, gi.kvh * p.G, qrow);
-        tma_load_3d(smem + kSmemQ + kQBytesPerDh, &p.tm_q, &sm.q_full, 64, gi.kvh * p.G, qrow);
-        ++qn;
         for (int k = kb; k < ke; ++k, ++f) {
-          const int stage = (int)(f % kStages);
-          const uint32_t round = (uint32_t)(f / kStages);
           const CUtensorMap* mk;
           const CUtensorMap* mv;
           int row;
@@ -431,44 +461,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             mk = &p.tm_kb;
             mv = &p.tm_vb;
           }
-          // K of a stage is free once its QK^T has run, V once its PV has run
-          if (round > 0 && !mbar_wait_bounded(&sm.k_empty[stage], (round - 1) & 1, abort_flag)) {
-            fail(kDetailWaitKvEmpty);
-            ok = false;
-            break;
+          if (do_kq) {
+            // K of a stage is free once both streams' QK^T have read it
+            const int ks = (int)(f % kKStages);
+            const uint32_t kround = (uint32_t)(f / kKStages);
+            if (kround > 0 && !mbar_wait_bounded(&sm.k_empty[ks], (kround - 1) & 1, abort_flag)) {
+              fail(kDetailWaitKvEmpty);
+              ok = false;
+              break;
+            }
+            uint8_t* kdst = smem + kSmemK + ks * kKBytesPerStage;
+            mbar_arrive_expect_tx(&sm.k_full[ks], kKBytesPerStage);
+            tma_load_3d(kdst, mk, &sm.k_full[ks], 0, gi.kvh, row);
+            tma_load_3d(kdst + kKVBoxBytes, mk, &sm.k_full[ks], 64, gi.kvh, row);
           }
-          uint8_t* kdst = smem + kSmemK + stage * kKBytesPerStage;
-          mbar_arrive_expect_tx(&sm.k_full[stage], kKBytesPerStage);
-          tma_load_3d(kdst, mk, &sm.k_full[stage], 0, gi.kvh, row);
-          tma_load_3d(kdst + kKVBoxBytes, mk, &sm.k_full[stage], 64, gi.kvh, row);
-          if (round > 0 && !mbar_wait_bounded(&sm.v_empty[stage], (round - 1) & 1, abort_flag)) {
-            fail(kDetailWaitKvEmpty);
-            ok = false;
-            break;
+          if (do_v) {
+            // V of a stage is free once both streams' PV have read it
+            const int vs = (int)(f % kVStages);
+            const uint32_t vround = (uint32_t)(f / kVStages);
+            if (vround > 0 && !mbar_wait_bounded(&sm.v_empty[vs], (vround - 1) & 1, abort_flag)) {
+              fail(kDetailWaitKvEmpty);
+              ok = false;
+              break;
+            }
+            uint8_t* vdst = smem + kSmemV + vs * kKBytesPerStage;
+            mbar_arrive_expect_tx(&sm.v_full[vs], kKBytesPerStage);
+            tma_load_3d(vdst, mv, &sm.v_full[vs], 0, gi.kvh, row);
+            tma_load_3d(vdst + kKVBoxBytes, mv, &sm.v_full[vs], 64, gi.kvh, row);
           }
-          uint8_t* vdst = smem + kSmemV + stage * kKBytesPerStage;
-          mbar_arrive_expect_tx(&sm.v_full[stage], kKBytesPerStage);
-          tma_load_3d(vdst, mv, &sm.v_full[stage], 0, gi.kvh, row);
-          tma_load_3d(vdst + kKVBoxBytes, mv, &sm.v_full[stage], 64, gi.kvh, row);
         }
         if (!ok) break;
         w.advance(p, hdr);
       }
-      // make sure every copy this CTA issued has landed before the CTA can exit
+      // make sure every copy this thread issued has landed before the CTA can exit
       const long long nf = f;
-      for (long long j = (nf > kStages ? nf - kStages : 0); j < nf; ++j) {
-        const int stage = (int)(j % kStages);
-        const uint32_t par = (uint32_t)((j / kStages) & 1);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&sm.k_full[stage], par) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
-        while (!mbar_try_wait(&sm.v_full[stage], par) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
+      const uint64_t t0 = globaltimer_ns();
+      if (do_kq) {
+        for (long long jj = (nf > kKStages ? nf - kKStages : 0); jj < nf; ++jj)
+          while (!mbar_try_wait(&sm.k_full[jj % kKStages], (uint32_t)((jj / kKStages) & 1)) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        if (qn > 0)
+          while (!mbar_try_wait(&sm.q_full, (uint32_t)((qn - 1) & 1)) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
       }
-      if (qn > 0) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&sm.q_full, (uint32_t)((qn - 1) & 1)) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
+      if (do_v) {
+        for (long long jj = (nf > kVStages ? nf - kVStages : 0); jj < nf; ++jj)
+          while (!mbar_try_wait(&sm.v_full[jj % kVStages], (uint32_t)((jj / kVStages) & 1)) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
       }
     }
   } else if (warp == 1) {
@@ -484,284 +525,280 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       long long f = 0;
       int seg = 0;
       bool ok = true;
-      bool have_prev = false;
-      bool prev_first = false;
-      // O (+)= P V for tile pf; P is in TMEM over S[pf % 2]
-      auto pv = [&](long long pf, bool first) -> bool {
-        const int stage = (int)(pf % kStages);
-        if (!mbar_wait_bounded(&sm.v_full[stage], (uint32_t)((pf / kStages) & 1), abort_flag)) {
-          fail(kDetailWaitKvFull);
-          return false;
-        }
-        if (!mbar_wait_bounded(&sm.p_full[pf & 1], (uint32_t)((pf >> 1) & 1), abort_flag)) {
-          fail(kDetailWaitPFull);
-          return false;
-        }
-        tc_fence_after();
-        const uint32_t p_tm = tmem + 128u + 128u * (uint32_t)(pf & 1);
-        const uint64_t vd = dv0 + (uint64_t)((stage * kKBytesPerStage) >> 4);
-        // keys 0-63: P columns 0-31; keys 64-127: P columns 64-95 (one block per column half)
-        mma_ts(tmem, p_tm, vd, kIdescPV, first ? 0u : 1u);
-#pragma unroll
-        for (int kk = 1; kk < kTile / 16; ++kk)
-          mma_ts(tmem, p_tm + 8u * (kk & 3) + 64u * (kk >> 2), vd + (uint64_t)((kk * 2048) >> 4), kIdescPV, 1u);
-        tc_commit(&sm.pv_done);
-        tc_commit(&sm.v_empty[stage]);
-        return true;
-      };
-      // S[ff % 2] = Q K^T for tile ff
-      auto qk = [&](long long ff) {
-        const int stage = (int)(ff % kStages);
-        const uint32_t d_tm = tmem + 128u + 128u * (uint32_t)(ff & 1);
+      // S_j = Q_j K^T for tile ff
+      auto qk = [&](int j, long long ff) {
+        const int stage = (int)(ff % kKStages);
+        const uint32_t d_tm = tmem + kTmemS + 128u * (uint32_t)j;
         const uint64_t kd = dk0 + (uint64_t)((stage * kKBytesPerStage) >> 4);
+        const uint64_t qd = dq0 + (uint64_t)((j * kQBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off_q = ((kk >> 2) * kQBytesPerDh + (kk & 3) * 32) >> 4;
           const uint32_t off_k = ((kk >> 2) * kKVBoxBytes + (kk & 3) * 32) >> 4;
-          mma_ss(d_tm, dq0 + off_q, kd + off_k, kIdescQK, kk > 0 ? 1u : 0u);
+          mma_ss(d_tm, qd + off_q, kd + off_k, kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&sm.s_full[ff & 1]);
-        tc_commit(&sm.k_empty[stage]);
+        tc_commit(&sm.s_full[j]);
+      };
+      // O_j (+)= P_j V for tile pf; P_j is in TMEM over the first 64 columns of S_j (keys 2c, 2c+1
+      // in column c)
+      auto pv = [&](int j, long long pf, bool first) {
+        const int stage = (int)(pf % kVStages);
+        const uint32_t p_tm = tmem + kTmemS + 128u * (uint32_t)j;
+        const uint32_t o_tm = tmem + 128u * (uint32_t)j;
+        const uint64_t vd = dv0 + (uint64_t)((stage * kKBytesPerStage) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(o_tm, p_tm + 8u * (uint32_t)kk, vd + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+                 (first && kk == 0) ? 0u : 1u);
       };
       while (ok && !w.done()) {
         int kb, ke;
         w.segment(kb, ke);
-        for (int k = kb; k < ke; ++k, ++f) {
-          const int stage = (int)(f % kStages);
-          if (k == kb && !mbar_wait_bounded(&sm.q_full, (uint32_t)(seg & 1), abort_flag)) {
-            fail(kDetailWaitQFull);
-            ok = false;
-            break;
-          }
-          if (!mbar_wait_bounded(&sm.k_full[stage], (uint32_t)((f / kStages) & 1), abort_flag)) {
+        if (!mbar_wait_bounded(&sm.q_full, (uint32_t)(seg & 1), abort_flag)) {
+          fail(kDetailWaitQFull);
+          break;
+        }
+        // the segment's first tile: both streams' scores
+        if (!mbar_wait_bounded(&sm.k_full[f % kKStages], (uint32_t)((f / kKStages) & 1), abort_flag)) {
+          fail(kDetailWaitKvFull);
+          break;
+        }
+        tc_fence_after();
+        for (int j = 0; j < nstreams; ++j) qk(j, f);
+        tc_commit(&sm.k_empty[f % kKStages]);
+        if (ke - kb == 1) tc_commit(&sm.q_empty);
+        for (int k = kb; k < ke && ok; ++k, ++f) {
+          const bool first = (k == kb), last = (k == ke - 1);
+          const int stage = (int)(f % kVStages);
+          if (!mbar_wait_bounded(&sm.v_full[stage], (uint32_t)((f / kVStages) & 1), abort_flag)) {
             fail(kDetailWaitKvFull);
             ok = false;
             break;
           }
-          tc_fence_after();
-          // S[f % 2] was last read as P of tile f-2, whose PV was issued before this QK^T
-          qk(f);
-          if (k == ke - 1) tc_commit(&sm.q_empty);
-          if (have_prev && !pv(f - 1, prev_first)) {
-            ok = false;
-            break;
+          for (int j = 0; j < nstreams; ++j) {
+            // P_j of tile f written (and O_j rescaled) by stream j's softmax
+            if (!mbar_wait_bounded(&sm.p_full[j], (uint32_t)(f & 1), abort_flag)) {
+              fail(kDetailWaitPFull);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            pv(j, f, first);
+            if (last) {
+              tc_commit(&sm.o_full[j]);
+            } else {
+              // S_j is free again: P_j(f) is read by the PV just issued, which runs first
+              const int nstage = (int)((f + 1) % kKStages);
+              if (j == 0) {
+                if (!mbar_wait_bounded(&sm.k_full[nstage], (uint32_t)(((f + 1) / kKStages) & 1), abort_flag)) {
+                  fail(kDetailWaitKvFull);
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+              }
+              qk(j, f + 1);
+              if (j == nstreams - 1) {
+                tc_commit(&sm.k_empty[nstage]);
+                if (k + 1 == ke - 1) tc_commit(&sm.q_empty);
+              }
+            }
           }
-          have_prev = true;
-          prev_first = (k == kb);
+          if (!ok) break;
+          tc_commit(&sm.v_empty[stage]);
         }
         if (!ok) break;
         ++seg;
         w.advance(p, hdr);
       }
-      if (ok && have_prev) pv(f - 1, prev_first);
     }
+  }
   } else {
-    // ======================= softmax + epilogue (warps 2-9)
-    const int t = 32 * (warp & 3) + lane;   // TMEM lane quadrant warp % 4 -> query row t
-    const int ch = (warp - 2) >> 2;         // column half: keys [64 ch, 64 ch + 64)
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t o_tm = tmem + lane_off + 64u * (uint32_t)ch;   // this thread's 64 output dims
-    const float sc = p.scale_log2;
-    float* partials = reinterpret_cast<float*>(p.ws + p.off_partials);
-    float* plse = reinterpret_cast<float*>(p.ws + p.off_lse);
-    SegWalk w;
-    w.init(p, sm, hdr);
-    long long f = 0;
-    int nseg = 0;
-    bool ok = true;
-    // partial row maximum of this thread's 64 raw scores -> exchanged maximum of the row (scaled)
-    auto exchange_max = [&](float mine, long long ff, float& row_max) -> bool {
-      sm.xmax[ff & 1][ch][t] = mine;
-      mbar_arrive(&sm.x_bar);
-      if (!mbar_wait_bounded(&sm.x_bar, (uint32_t)(ff & 1), abort_flag)) {
-        fail(kDetailWaitTicket);
-        return false;
-      }
-      __syncwarp();
-      row_max = fmaxf(mine, sm.xmax[ff & 1][ch ^ 1][t]);
-      return true;
-    };
-    while (ok && !w.done()) {
-      int kb, ke;
-      w.segment(kb, ke);
-      const GroupInfo gi = w.gi;
-      float m_used = -INFINITY, l = 0.f;
-      for (int k = kb; k < ke; ++k, ++f) {
-        const int valid = (k < gi.nctx) ? min(kTile, gi.L - k * kTile) : p.S;
-        const int lim = valid - 64 * ch;    // valid columns among this thread's 64
-        const uint32_t s_tm = tmem + lane_off + 128u + 128u * (uint32_t)(f & 1) + 64u * (uint32_t)ch;
-        if (!mbar_wait_bounded(&sm.s_full[f & 1], (uint32_t)((f >> 1) & 1), abort_flag)) {
-          fail(kDetailWaitSFull);
-          ok = false;
-          break;
-        }
-        __syncwarp();   // lanes leave the wait one by one; the tcgen05 accesses are warp-collective
-        tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(s_tm, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(s_tm + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_wait_ld();
-        // The row's tile maximum (both column halves, exchanged through shared memory) decides the
-        // exponent base: a segment's first tile uses it; later tiles keep the running maximum
-        // m_used unless the tile exceeds it by more than 8 (P would exceed 256), in which case the
-        // base moves to the tile maximum and O is rescaled. Then one pass writes
-        // P = 2^(s*scale - base) in bf16 over this thread's S columns and sums P in fp32.
-        const bool first = (k == kb);
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (lim >= 64) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sr[j]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            if (j >= lim) sr[j] = __float_as_uint(-INFINITY);
-            mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sr[j]));
-          }
-        }
-        float rm;
-        if (!exchange_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), f, rm)) {
-          ok = false;
-          break;
-        }
-        const float mt = rm * sc;
-        float m_new = m_used;
-        bool resc = false;
-        if (first) {
-          m_new = mt;
-        } else if (mt > m_used + 8.0f) {
-          m_new = mt;
-          resc = true;
-        }
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int j = 16 * q + jj;
-            const float p0 = ex2(fmaf(__uint_as_float(sr[2 * j]), sc, -m_new));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[2 * j + 1]), sc, -m_new));
-            ps[j & 3] += p0 + p1;
-            pk[jj] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(s_tm + 16u * q, pk);
-        }
-        const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-        const float factor = resc ? ex2(m_used - m_new) : 1.0f;
-        l = l * factor + psum;
-        tmem_wait_st();
-        if (!first) {
-          // O holds the sum up to tile f-1: its PV product must be complete before O is rescaled
-          // and before P of this tile is handed over (so the pv_done phases stay one step apart)
-          if (!mbar_wait_bounded(&sm.pv_done, (uint32_t)((f - 1) & 1), abort_flag)) {
-            fail(kDetailWaitPvDone);
+    setmaxnreg_inc<kSoftmaxRegs>();
+    // ======================= softmax + epilogue (stream j = warps 4-7 / 8-11)
+    const int j = (warp - 4) >> 2;
+    if (has_work && j < nstreams) {
+      const int t = 32 * (warp & 3) + lane;   // TMEM lane quadrant warp % 4 -> query row t
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t s_tm = tmem + lane_off + kTmemS + 128u * (uint32_t)j;
+      const uint32_t o_tm = tmem + lane_off + 128u * (uint32_t)j;
+      const int qt = qt0 + j;
+      const int s_cnt = min(p.s_per_tile, p.S - qt * p.s_per_tile);   // block positions of this query tile
+      const int nrows = p.G * s_cnt;                                   // valid query rows (<= 128)
+      const float sc = p.scale_log2;
+      float* partials = reinterpret_cast<float*>(p.ws + p.off_partials);
+      float* plse = reinterpret_cast<float*>(p.ws + p.off_lse);
+      SegWalk w;
+      w.init(p, sm, hdr);
+      long long f = 0;
+      int nseg = 0;
+      bool ok = true;
+      while (ok && !w.done()) {
+        int kb, ke;
+        w.segment(kb, ke);
+        const GroupInfo gi = w.gi;
+        float m_used = -INFINITY, l = 0.f;
+        for (int k = kb; k < ke; ++k, ++f) {
+          const int valid = (k < gi.nctx) ? min(kTile, gi.L - k * kTile) : p.S;
+          if (!mbar_wait_bounded(&sm.s_full[j], (uint32_t)(f & 1), abort_flag)) {
+            fail(kDetailWaitSFull);
             ok = false;
             break;
           }
-          __syncwarp();
+          // The commit behind s_full also covers every earlier MMA of the issuing thread, so the
+          // PV of the previous tile has completed: O_j may be read and rescaled below.
+          __syncwarp();   // lanes leave the wait one by one; the tcgen05 accesses are warp-collective
           tc_fence_after();
-          // rows decide separately; the O accesses are warp-collective, so the warp rescales when
-          // any of its rows needs it (factor is 1 for the others)
-          if (__any_sync(0xffffffffu, resc)) {
+          uint32_t sr[128];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tmem_ld32(s_tm + 32u * (uint32_t)q, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * q]));
+          tmem_wait_ld();
+          if (valid < kTile) {
+#pragma unroll
+            for (int c = 0; c < kTile; ++c)
+              if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+          }
+          // the row's tile maximum decides the exponent base: a segment's first tile uses it;
+          // later tiles keep the running maximum m_used unless the tile exceeds it by more than 8
+          // (P would exceed 256), in which case the base moves and O is rescaled
+          float mx[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mx[q] = __uint_as_float(sr[q]);
+#pragma unroll
+          for (int c = 4; c + 8 <= kTile; c += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) mx[q] = fmax3(mx[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + 4 + q]));
+          }
+          mx[0] = fmax3(mx[0], __uint_as_float(sr[kTile - 4]), __uint_as_float(sr[kTile - 3]));
+          mx[1] = fmax3(mx[1], __uint_as_float(sr[kTile - 2]), __uint_as_float(sr[kTile - 1]));
+          const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc;
+          const bool first = (k == kb);
+          float m_new = m_used;
+          bool resc = false;
+          if (first) {
+            m_new = mt;
+          } else if (mt > m_used + 8.0f) {
+            m_new = mt;
+            resc = true;
+          }
+          // P = 2^(s * scale - base), written as bf16 pairs over the first 64 columns of S_j,
+          // summed in fp32
+          const uint64_t sc2 = pack_f32x2(sc, sc);
+          const uint64_t nb2 = pack_f32x2(-m_new, -m_new);
+          uint64_t acc2[2] = {pack_f32x2(0.f, 0.f), pack_f32x2(0.f, 0.f)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int c = 32 * q + 2 * jj;
+              const uint64_t x2 = ffma_f32x2(pack_u32x2(sr[c], sr[c + 1]), sc2, nb2);
+              const float p0 = ex2(lo_f32(x2)), p1 = ex2(hi_f32(x2));
+              const uint64_t p2 = pack_f32x2(p0, p1);
+              acc2[jj & 1] = fadd_f32x2(acc2[jj & 1], p2);
+              pk[jj] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(s_tm + 16u * (uint32_t)q, pk);
+          }
+          const uint64_t acc = fadd_f32x2(acc2[0], acc2[1]);
+          const float psum = lo_f32(acc) + hi_f32(acc);
+          const float factor = resc ? ex2(m_used - m_new) : 1.0f;
+          l = l * factor + psum;
+          tmem_wait_st();
+          if (!first && __any_sync(0xffffffffu, resc)) {
+            // rows decide separately; the O accesses are warp-collective, so the warp rescales when
+            // any of its rows needs it (factor is 1 for the others)
 #pragma unroll 1
-            for (int cb = 0; cb < 2; ++cb) {
+            for (int cb = 0; cb < 4; ++cb) {
               uint32_t orr[32];
-              tmem_ld32(o_tm + 32u * cb, orr);
+              tmem_ld32(o_tm + 32u * (uint32_t)cb, orr);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * factor);
-              tmem_st32(o_tm + 32u * cb, orr);
+              for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * factor);
+              tmem_st32(o_tm + 32u * (uint32_t)cb, orr);
             }
             tmem_wait_st();
           }
-        }
-        if (ch == 0 && k < gi.nctx && valid < kTile) {
-          // Rows past the end of the context hold whatever the caller's slab or page holds
-          // there; P is 0 for them, but 0 * NaN would still poison O, so zero those V rows
-          // before the PV product reads them. The V tile must have landed first.
-          const int stage = (int)(f % kStages);
-          if (!mbar_wait_bounded(&sm.v_full[stage], (uint32_t)((f / kStages) & 1), abort_flag)) {
-            fail(kDetailWaitKvFull);
-            ok = false;
-            break;
+          if (j == 0 && k < gi.nctx && valid < kTile) {
+            // Rows past the end of the context hold whatever the caller's slab or page holds
+            // there; P is 0 for them, but 0 * NaN would still poison O, so zero those V rows
+            // before the PV products (stream 0's runs first) read them. The V tile must have
+            // landed first.
+            const int stage = (int)(f % kVStages);
+            if (!mbar_wait_bounded(&sm.v_full[stage], (uint32_t)((f / kVStages) & 1), abort_flag)) {
+              fail(kDetailWaitKvFull);
+              ok = false;
+              break;
+            }
+            uint8_t* vbase = smem + kSmemV + stage * kKBytesPerStage;
+            const int chunks_per_box = (kTile - valid) * 8;   // 16-byte chunks
+            for (int i = t; i < 2 * chunks_per_box; i += kRows) {
+              const int box = i / chunks_per_box, r = i - box * chunks_per_box;
+              *reinterpret_cast<uint4*>(vbase + box * kKVBoxBytes + (valid + r / 8) * 128 + (r % 8) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           }
-          uint8_t* vbase = smem + kSmemV + stage * kKBytesPerStage;
-          const int chunks_per_box = (kTile - valid) * 8;   // 16-byte chunks
-          for (int i = t; i < 2 * chunks_per_box; i += kRows) {
-            const int box = i / chunks_per_box, r = i - box * chunks_per_box;
-            *reinterpret_cast<uint4*>(vbase + box * kKVBoxBytes + (valid + r / 8) * 128 + (r % 8) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          m_used = m_new;
+          tc_fence_before();
+          mbar_arrive(&sm.p_full[j]);
         }
-        m_used = m_new;
-        tc_fence_before();
-        mbar_arrive(&sm.p_full[f & 1]);
-      }
-      if (!ok) break;
-      // ---- epilogue of the segment: wait for the last PV product, combine the two column
-      // halves' sums, then O / l for this thread's 64 dims of its row
-      const long long lf = f - 1;
-      if (!mbar_wait_bounded(&sm.pv_done, (uint32_t)(lf & 1), abort_flag)) {
-        fail(kDetailWaitPvDone);
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      sm.xsum[ch][t] = l;
-      mbar_arrive(&sm.l_bar);
-      if (!mbar_wait_bounded(&sm.l_bar, (uint32_t)(nseg & 1), abort_flag)) {
-        fail(kDetailWaitTicket);
-        ok = false;
-        break;
-      }
-      __syncwarp();
-      l += sm.xsum[ch ^ 1][t];
-      ++nseg;
-      const bool whole = (kb == 0) && (ke == gi.ntiles);
-      const bool row_valid = t < nrows;
-      const int s_idx = qt * p.s_per_tile + t / p.G;
-      const int hq = gi.kvh * p.G + t % p.G;
-      const float inv_l = 1.0f / l;
-      const float lse2 = m_used + log2f(l);
-      // partial slot unique per (group, team, query tile)
-      const size_t slot = ((size_t)w.u + (size_t)team) * (size_t)p.nq + (size_t)qt;
-      __nv_bfloat16* orow = p.out + (((size_t)gi.b * p.S + s_idx) * p.Hq + hq) * kD + 64 * ch;
-      float* prow = partials + (slot * kRows + t) * kD + 64 * ch;
+        if (!ok) break;
+        // ---- epilogue of the segment: wait for the last PV product, then O / l for the row
+        if (!mbar_wait_bounded(&sm.o_full[j], (uint32_t)(nseg & 1), abort_flag)) {
+          fail(kDetailWaitPvDone);
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        ++nseg;
+        const bool whole = (kb == 0) && (ke == gi.ntiles);
+        const bool row_valid = t < nrows;
+        const int s_idx = qt * p.s_per_tile + t / p.G;
+        const int hq = gi.kvh * p.G + t % p.G;
+        const float inv_l = 1.0f / l;
+        const float lse2 = m_used + log2f(l);
+        // partial slot unique per (group, team, query tile)
+        const size_t slot = ((size_t)w.u + (size_t)team) * (size_t)p.nq + (size_t)qt;
+        __nv_bfloat16* orow = p.out + (((size_t)gi.b * p.S + s_idx) * p.Hq + hq) * kD;
+        float* prow = partials + (slot * kRows + t) * kD;
 #pragma unroll 1
-      for (int cb = 0; cb < 2; ++cb) {
-        uint32_t orr[32];
-        tmem_ld32(o_tm + 32u * cb, orr);
-        tmem_wait_ld();
+        for (int cb = 0; cb < 4; ++cb) {
+          uint32_t orr[32];
+          tmem_ld32(o_tm + 32u * (uint32_t)cb, orr);
+          tmem_wait_ld();
+          if (row_valid) {
+            if (whole) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(orr[8 * q4 + 0]) * inv_l, __uint_as_float(orr[8 * q4 + 1]) * inv_l);
+                v.y = pack_bf16x2(__uint_as_float(orr[8 * q4 + 2]) * inv_l, __uint_as_float(orr[8 * q4 + 3]) * inv_l);
+                v.z = pack_bf16x2(__uint_as_float(orr[8 * q4 + 4]) * inv_l, __uint_as_float(orr[8 * q4 + 5]) * inv_l);
+                v.w = pack_bf16x2(__uint_as_float(orr[8 * q4 + 6]) * inv_l, __uint_as_float(orr[8 * q4 + 7]) * inv_l);
+                dst[q4] = v;
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(prow + cb * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                dst[q4] = make_float4(__uint_as_float(orr[4 * q4 + 0]) * inv_l, __uint_as_float(orr[4 * q4 + 1]) * inv_l,
+                                      __uint_as_float(orr[4 * q4 + 2]) * inv_l, __uint_as_float(orr[4 * q4 + 3]) * inv_l);
+            }
+          }
+        }
         if (row_valid) {
           if (whole) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(orr[8 * q4 + 0]) * inv_l, __uint_as_float(orr[8 * q4 + 1]) * inv_l);
-              v.y = pack_bf16x2(__uint_as_float(orr[8 * q4 + 2]) * inv_l, __uint_as_float(orr[8 * q4 + 3]) * inv_l);
-              v.z = pack_bf16x2(__uint_as_float(orr[8 * q4 + 4]) * inv_l, __uint_as_float(orr[8 * q4 + 5]) * inv_l);
-              v.w = pack_bf16x2(__uint_as_float(orr[8 * q4 + 6]) * inv_l, __uint_as_float(orr[8 * q4 + 7]) * inv_l);
-              dst[q4] = v;
-            }
+            if (p.lse) p.lse[((size_t)gi.b * p.Hq + hq) * p.S + s_idx] = lse2 * 0.69314718055994531f;
           } else {
-            float4* dst = reinterpret_cast<float4*>(prow + cb * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              dst[q4] = make_float4(__uint_as_float(orr[4 * q4 + 0]) * inv_l, __uint_as_float(orr[4 * q4 + 1]) * inv_l,
-                                    __uint_as_float(orr[4 * q4 + 2]) * inv_l, __uint_as_float(orr[4 * q4 + 3]) * inv_l);
+            plse[slot * kRows + t] = lse2;
           }
         }
+        w.advance(p, hdr);
       }
-      if (row_valid && ch == 0) {
-        if (whole) {
-          if (p.lse) p.lse[((size_t)gi.b * p.Hq + hq) * p.S + s_idx] = lse2 * 0.69314718055994531f;
-        } else {
-          plse[slot * kRows + t] = lse2;
-        }
-      }
-      w.advance(p, hdr);
     }
   }
 
@@ -790,10 +827,12 @@ struct MergeParams {
   float* lse;
   const uint8_t* ws;
   size_t off_meta, off_crange, off_partials, off_lse;
+  const int32_t* skip_if;
 };
 
 __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   pdl_wait();
+  if (skip_requested(p.skip_if)) return;
   const int u = blockIdx.x;             // group
   const int qt = blockIdx.z;            // query tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -899,11 +938,12 @@ AttnPlan attn_tc_plan(const tt_attn_args_t* a, int num_sms) {
   const int G = a->num_q_heads / a->num_kv_heads;
   const int S = a->block_size;
   pl.s_per_tile = std::min(S, kRows / G);
-  pl.qtiles = (S + pl.s_per_tile - 1) / pl.s_per_tile;        // nq, CTAs per team
+  pl.qtiles = (S + pl.s_per_tile - 1) / pl.s_per_tile;        // nq
+  pl.team_size = (pl.qtiles + 1) / 2;                           // CTAs per team, two query tiles each
   pl.units = a->batch * a->num_kv_heads;                        // groups
   const int sms = std::max(1, num_sms);
-  const int teams = std::max(1, sms / pl.qtiles);
-  pl.grid = teams * pl.qtiles;
+  const int teams = std::max(1, sms / pl.team_size);
+  pl.grid = teams * pl.team_size;
   pl.slots = ((size_t)pl.units + (size_t)teams) * (size_t)pl.qtiles;
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
@@ -940,9 +980,10 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   p.Hkv = a->num_kv_heads;
   p.G = G;
   p.nq = pl.qtiles;
+  p.nq2 = pl.team_size;
   p.s_per_tile = pl.s_per_tile;
   p.groups = pl.units;
-  p.teams = pl.grid / pl.qtiles;
+  p.teams = pl.grid / pl.team_size;
   p.page_size = a->page_size;
   p.max_pages = a->max_pages_per_seq;
   p.num_pages = a->num_pages;
@@ -956,6 +997,7 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   p.off_crange = pl.off_crange;
   p.off_partials = pl.off_partials;
   p.off_lse = pl.off_lse;
+  p.skip_if = a->skip_if;
   // the shared-memory opt-in is per device; set it once so no attribute call happens while a
   // caller captures the stream into a CUDA graph
   static unsigned long long attr_done = 0;   // bit per device ordinal (< 64)
@@ -963,6 +1005,11 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
+    // The register raise of the softmax warpgroups waits until the block's pool (launch registers
+    // x threads) has room: refuse to launch unless the compiled kernel starts with enough.
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, attn_tc_kernel) != cudaSuccess) return TT_ERR_CUDA;
+    if (fa.numRegs * kThreads < 128 * kProducerRegs + 2 * 128 * kSoftmaxRegs) return TT_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
         cudaSuccess)
       return TT_ERR_CUDA;
@@ -985,6 +1032,7 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   mp.off_crange = pl.off_crange;
   mp.off_partials = pl.off_partials;
   mp.off_lse = pl.off_lse;
+  mp.skip_if = a->skip_if;
   const int M = G * pl.s_per_tile;
   const dim3 mgrid(pl.units, (M + kMergeRows - 1) / kMergeRows, pl.qtiles);
   if (launch_pdl(attn_merge_kernel, mgrid, dim3(256), 0, stream, mp) != cudaSuccess) return TT_ERR_CUDA;

@@ -5,7 +5,7 @@
 // this kernel appends the rows it produced and grows the page tables.
 //
 // One CTA per sequence. Thread 0 takes the pages the block newly needs from a device-side stack of
-// free page ids (one atomic per sequence, no spinning) and enters them in the page table; then the
+// free page ids (a compare-and-swap on the stack count) and enters them in the page table; then the
 // CTA copies the S x Hkv rows of K and V into their page slots with 16-byte vector copies and
 // advances ctx_lens[b] by S. A sequence whose pages cannot be provided (stack exhausted, page
 // table full) is left unchanged and the workspace error word is set.
@@ -17,6 +17,7 @@ namespace tt {
 namespace {
 
 constexpr int kAppendThreads = 256;
+constexpr int kMaxClaimRounds = 1 << 20;
 
 struct AppendParams {
   const uint4* k_new;
@@ -53,22 +54,45 @@ __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendP
       ok = 0;
     }
     if (ok && need > have) {
+      // Claim the top n entries of the free stack with a compare-and-swap that only ever moves
+      // the count from `top` to `top - n` when top >= n: a claim that cannot be served never
+      // changes the count, so concurrent failures cannot expose pages another sequence holds.
+      // The entries a claim would take are checked before the swap (the stack array is not
+      // written during the launch), so a bad page id leaves this sequence and the stack as they
+      // were. Every failed swap means another sequence's swap succeeded, so the loop ends within
+      // `batch` rounds; the bound below only guards against a count written concurrently by
+      // something outside this launch.
       const int n = (int)(need - have);
-      const int top = atomicSub(p.free_count, n);   // pages [top - n, top) of the stack are ours
-      if (top - n < 0) {
-        atomicAdd(p.free_count, n);
-        report_error(p.hdr, TT_ERR_DEVICE, kDetailOutOfPages);
-        ok = 0;
-      } else {
+      int top = *reinterpret_cast<volatile int*>(p.free_count);
+      ok = 0;
+      bool settled = false;   // claimed, or failed with an error reported
+      for (int attempt = 0; attempt < kMaxClaimRounds && !settled; ++attempt) {
+        if (top < n) {
+          report_error(p.hdr, TT_ERR_DEVICE, kDetailOutOfPages);
+          settled = true;
+          break;
+        }
+        bool valid = true;
         for (int i = 0; i < n; ++i) {
           const int pg = p.free_pages[top - n + i];
-          if (pg < 0 || pg >= p.num_pages) {
-            report_error(p.hdr, TT_ERR_DEVICE, kDetailBadPage);
-            ok = 0;
-          }
-          p.page_table[(size_t)b * p.max_pages + have + i] = pg;
+          valid = valid && pg >= 0 && pg < p.num_pages;
         }
+        if (!valid) {
+          report_error(p.hdr, TT_ERR_DEVICE, kDetailBadPage);
+          settled = true;
+          break;
+        }
+        const int prev = atomicCAS(p.free_count, top, top - n);
+        if (prev == top) {
+          for (int i = 0; i < n; ++i)
+            p.page_table[(size_t)b * p.max_pages + have + i] = p.free_pages[top - n + i];
+          ok = 1;
+          settled = true;
+          break;
+        }
+        top = prev;
       }
+      if (!settled) report_error(p.hdr, TT_ERR_DEVICE, kDetailClaimContended);
     }
     s_ok = ok;
     s_len = L;

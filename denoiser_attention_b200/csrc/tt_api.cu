@@ -1,5 +1,6 @@
 // C ABI entry points: host-side argument validation, workspace sizing and dispatch to the
 // sm_100a kernels. Nothing here allocates device memory or keeps mutable global state.
+#include <climits>
 #include <cstdio>
 #include <cstring>
 
@@ -17,12 +18,31 @@ int device_sm_count() {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The kernels index rows (batch * block_size) in 32 bits and cut the logits (rows * vocab
+// elements) into CTA ranges with 64-bit products of a CTA index and the element count; these
+// bounds keep both exact.
+static bool rows_fit(int32_t batch, int32_t block_size) {
+  return (long long)batch * (long long)block_size <= (long long)INT32_MAX;
+}
+static bool logits_fit(int32_t batch, int32_t block_size, int32_t vocab) {
+  return (long long)batch * (long long)block_size * (long long)vocab < (1LL << 40);
+}
+
+// Predict-and-noise arguments: either an explicit keep_masked >= 0 (noise_steps == 0), or a step
+// r in 1..T of the linear schedule (noise_steps = T > 0).
+static bool noise_schedule_valid(int32_t keep_masked, int32_t noise_steps, int32_t noise_step) {
+  if (noise_steps < 0) return false;
+  if (noise_steps == 0) return keep_masked >= 0;
+  return noise_step >= 1 && noise_step <= noise_steps;
+}
+
 static int validate_attn(const tt_attn_args_t* a) {
   if (!a) return TT_ERR_INVALID_ARGUMENT;
   if (a->batch < 1 || a->block_size < 1 || a->num_q_heads < 1 || a->num_kv_heads < 1 || a->head_dim < 1)
     return TT_ERR_INVALID_ARGUMENT;
   if (a->num_q_heads % a->num_kv_heads != 0) return TT_ERR_INVALID_ARGUMENT;
   if (a->dtype != TT_F32 && a->dtype != TT_BF16) return TT_ERR_INVALID_ARGUMENT;
+  if (!rows_fit(a->batch, a->block_size) || !rows_fit(a->batch, a->num_kv_heads)) return TT_ERR_UNSUPPORTED;
   if (!a->q || !a->k_blk || !a->v_blk || !a->k_ctx || !a->v_ctx || !a->ctx_lens || !a->out)
     return TT_ERR_INVALID_ARGUMENT;
   if (!(a->softmax_scale > 0.f) || !(a->softmax_scale < 3.0e38f)) return TT_ERR_INVALID_ARGUMENT;
@@ -33,7 +53,7 @@ static int validate_attn(const tt_attn_args_t* a) {
   }
   if (a->block_size > 64) return TT_ERR_UNSUPPORTED;
   if (a->dtype == TT_BF16 && !attn_tc_supported(a)) return TT_ERR_UNSUPPORTED;
-  if (a->dtype == TT_F32 && !attn_simt_supported(a)) return TT_ERR_UNSUPPORTED;
+  if (a->dtype == TT_F32 && !attn_tf32_supported(a)) return TT_ERR_UNSUPPORTED;
   return TT_OK;
 }
 
@@ -41,6 +61,8 @@ static int validate_unmask(const tt_unmask_args_t* a) {
   if (!a) return TT_ERR_INVALID_ARGUMENT;
   if (a->batch < 1 || a->block_size < 1 || a->vocab < 1) return TT_ERR_INVALID_ARGUMENT;
   if (a->dtype != TT_F32 && a->dtype != TT_BF16) return TT_ERR_INVALID_ARGUMENT;
+  if (!rows_fit(a->batch, a->block_size) || !logits_fit(a->batch, a->block_size, a->vocab))
+    return TT_ERR_UNSUPPORTED;
   if (!a->logits || !a->tokens || !a->is_masked || !a->n_committed || !a->n_masked) return TT_ERR_INVALID_ARGUMENT;
   if (!(a->inv_temperature > 0.f)) return TT_ERR_INVALID_ARGUMENT;
   if (a->remaining_steps < 0) return TT_ERR_INVALID_ARGUMENT;
@@ -49,7 +71,8 @@ static int validate_unmask(const tt_unmask_args_t* a) {
   const int W = (a->dtype == TT_BF16) ? 8 : 4;
   if (a->vocab % W != 0 || !aligned16(a->logits)) return TT_ERR_UNSUPPORTED;
   if (a->sampler != TT_SAMPLER_CONFIDENCE && a->sampler != TT_SAMPLER_PREDICT_NOISE) return TT_ERR_INVALID_ARGUMENT;
-  if (a->sampler == TT_SAMPLER_PREDICT_NOISE && a->keep_masked < 0) return TT_ERR_INVALID_ARGUMENT;
+  if (a->sampler == TT_SAMPLER_PREDICT_NOISE && !noise_schedule_valid(a->keep_masked, a->noise_steps, a->noise_step))
+    return TT_ERR_INVALID_ARGUMENT;
   return TT_OK;
 }
 
@@ -86,10 +109,12 @@ static int validate_adaln(const tt_adaln_args_t* a) {
 static int validate_lmhead(const tt_lmhead_unmask_args_t* a) {
   if (!a) return TT_ERR_INVALID_ARGUMENT;
   if (a->batch < 1 || a->block_size < 1 || a->hidden < 1 || a->vocab < 1) return TT_ERR_INVALID_ARGUMENT;
+  if (!rows_fit(a->batch, a->block_size)) return TT_ERR_UNSUPPORTED;
   if (!a->x || !a->w || !a->tokens || !a->is_masked || !a->n_committed || !a->n_masked) return TT_ERR_INVALID_ARGUMENT;
   if (!(a->inv_temperature > 0.f)) return TT_ERR_INVALID_ARGUMENT;
   if (a->sampler != TT_SAMPLER_CONFIDENCE && a->sampler != TT_SAMPLER_PREDICT_NOISE) return TT_ERR_INVALID_ARGUMENT;
-  if (a->sampler == TT_SAMPLER_PREDICT_NOISE && a->keep_masked < 0) return TT_ERR_INVALID_ARGUMENT;
+  if (a->sampler == TT_SAMPLER_PREDICT_NOISE && !noise_schedule_valid(a->keep_masked, a->noise_steps, a->noise_step))
+    return TT_ERR_INVALID_ARGUMENT;
   if (a->dtype != TT_BF16) return TT_ERR_UNSUPPORTED;
   if (a->hidden % 64 != 0 || a->vocab % 128 != 0 || a->block_size > 1024) return TT_ERR_UNSUPPORTED;
   if (!aligned16(a->x) || !aligned16(a->w)) return TT_ERR_UNSUPPORTED;
@@ -109,6 +134,20 @@ static int validate_kv_append(const tt_kv_append_args_t* a) {
   if (!aligned16(a->k_new) || !aligned16(a->v_new) || !aligned16(a->k_ctx) || !aligned16(a->v_ctx))
     return TT_ERR_UNSUPPORTED;
   return TT_OK;
+}
+
+// One thread waits on a barrier that nothing arrives on, with the kernels' bounded wait and the
+// given limit; it gives up, records the timeout in the workspace's error word and returns.
+__global__ void wait_probe_kernel(WsHeader* hdr, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    if (!mbar_wait_bounded_for(&bar, 0, &abort_flag, limit_ns))
+      report_error(hdr, TT_ERR_DEVICE_TIMEOUT, TT_DETAIL_WAIT_PROBE);
+  }
 }
 
 }  // namespace tt
@@ -135,7 +174,7 @@ int tt_version(void) { return 100; }
 size_t tt_denoise_attn_workspace_bytes(const tt_attn_args_t* a) {
   if (validate_attn(a) != TT_OK) return 0;
   const int sms = device_sm_count();
-  return a->dtype == TT_BF16 ? attn_tc_plan(a, sms).total : attn_simt_plan(a, sms).total;
+  return a->dtype == TT_BF16 ? attn_tc_plan(a, sms).total : attn_tf32_plan(a, sms).total;
 }
 
 int tt_denoise_attn(const tt_attn_args_t* a, void* ws, size_t ws_bytes, tt_stream_t stream) {
@@ -149,9 +188,9 @@ int tt_denoise_attn(const tt_attn_args_t* a, void* ws, size_t ws_bytes, tt_strea
     if (ws_bytes < pl.total) return TT_ERR_WORKSPACE_TOO_SMALL;
     return attn_tc_launch(a, pl, ws, s);
   }
-  const AttnPlan pl = attn_simt_plan(a, sms);
+  const AttnPlan pl = attn_tf32_plan(a, sms);
   if (ws_bytes < pl.total) return TT_ERR_WORKSPACE_TOO_SMALL;
-  return attn_simt_launch(a, pl, ws, s);
+  return attn_tf32_launch(a, pl, ws, s);
 }
 
 size_t tt_adaln_workspace_bytes(const tt_adaln_args_t* a) {
@@ -187,9 +226,10 @@ int tt_unmask_step_noalloc(const tt_unmask_args_t* a, tt_stream_t stream) {
   return unmask_launch_static(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, tt_stream_t stream) {
+int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, const int32_t* skip_if,
+                 tt_stream_t stream) {
   if (!is_masked || !tau || batch < 1 || block_size < 1) return TT_ERR_INVALID_ARGUMENT;
-  return block_tau_launch(is_masked, batch, block_size, tau, reinterpret_cast<cudaStream_t>(stream));
+  return block_tau_launch(is_masked, batch, block_size, tau, skip_if, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t tt_lmhead_unmask_workspace_bytes(const tt_lmhead_unmask_args_t* a) {
@@ -214,6 +254,18 @@ int tt_kv_append(const tt_kv_append_args_t* a, void* ws, size_t ws_bytes, tt_str
   if (!ws) return TT_ERR_INVALID_ARGUMENT;
   if (ws_bytes < kHeaderBytes) return TT_ERR_WORKSPACE_TOO_SMALL;
   return kv_append_launch(a, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int32_t tt_linear_schedule_keep(int32_t block_size, int32_t steps, int32_t step) {
+  if (block_size < 1 || steps < 1 || step < 1 || step > steps) return -1;
+  return linear_schedule_keep(block_size, steps, step);
+}
+
+int tt_probe_bounded_wait(void* ws, uint32_t limit_us, tt_stream_t stream) {
+  if (!ws || limit_us < 1 || limit_us > 1000000u) return TT_ERR_INVALID_ARGUMENT;
+  wait_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<WsHeader*>(ws),
+                                                                           (uint64_t)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? TT_OK : TT_ERR_CUDA;
 }
 
 int tt_get_device_error(void* ws, tt_stream_t stream, uint32_t* detail) {

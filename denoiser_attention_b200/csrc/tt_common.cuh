@@ -28,6 +28,7 @@ enum : uint32_t {
   kDetailNegativeLen = 3,    // negative context length
   kDetailOutOfPages = 4,     // block commit: the free-page stack cannot provide the pages needed
   kDetailPageTableFull = 5,  // block commit: the context would outgrow max_pages_per_seq pages
+  kDetailClaimContended = 6, // block commit: the free-stack count kept changing (written outside the launch)
   kDetailWaitQFull = 0x100,  // bounded waits: which wait gave up
   kDetailWaitKvFull = 0x101,
   kDetailWaitKvEmpty = 0x102,
@@ -88,16 +89,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete. Gives up (returns false) after the
-// time limit or as soon as *abort_flag becomes non-zero.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Waits for the phase with the given parity to complete. Gives up (returns false) after
+// limit_ns nanoseconds or as soon as *abort_flag becomes non-zero.
+__device__ __forceinline__ bool mbar_wait_bounded_for(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                      uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// The kernels' bounded wait: gives up after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait_bounded_for(bar, parity, abort_flag, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA (no multicast)
@@ -190,6 +197,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// ------------------------------------------------------------------ per-warpgroup register counts
+// Executed by all threads of a warpgroup: lower / raise its registers per thread to N. A raise
+// waits until the block's pool (launch registers x threads) has room, so the counts of all
+// warpgroups must add up to at most the launch pool.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // Every kernel of the library is launched with programmatic stream serialization: it may start
 // while the previous kernel on the stream is finishing, runs a prologue that reads no input,
@@ -214,6 +234,12 @@ inline cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Early exit of a multi-step loop: the optional loop-control word holds a non-zero value. Read
+// after pdl_wait(), so the value written by an earlier kernel of the stream is visible.
+__device__ __forceinline__ bool skip_requested(const int32_t* skip_if) {
+  return skip_if != nullptr && *reinterpret_cast<const volatile int32_t*>(skip_if) != 0;
+}
+
 // ------------------------------------------------------------------ arithmetic
 // Hardware base-2 exponential (MUFU.EX2 through the PTX ex2.approx instruction).
 __device__ __forceinline__ float ex2(float x) {
@@ -222,30 +248,49 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for |x| <= 126: Cody-Waite split x = n + f with n = round(x) (taken
-// from the low mantissa bits of x + 1.5 * 2^23) and f in [-0.5, 0.5], then 2^f from a degree-4
-// polynomial fitted here to the relative error of 2^f on that interval (max 2.7e-6), and 2^n
-// added to the exponent field. Used for a share of the softmax exponentials so that they do not
-// all queue on the MUFU pipe.
-__device__ __forceinline__ float ex2_fma(float x) {
-  const float t = x + 12582912.0f;
-  const float fr = x - (t - 12582912.0f);
-  const int n = __float_as_int(t) - 0x4B400000;
-  float p = 0.009570068679749966f;
-  p = fmaf(p, fr, 0.055917806923389435f);
-  p = fmaf(p, fr, 0.240247443318367f);
-  p = fmaf(p, fr, 0.6931218504905701f);
-  p = fmaf(p, fr, 0.9999992847442627f);
-  return __int_as_float(__float_as_int(p) + (n << 23));
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed pairs of fp32 values in one 64-bit register: (lo, hi). The f32x2 arithmetic of sm_100
+// does two fp32 operations per instruction, each rounded as its scalar form.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+// a * b + c, elementwise on the pairs (round to nearest)
+__device__ __forceinline__ uint64_t ffma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+// a * b, elementwise on the pairs (round to nearest)
+__device__ __forceinline__ uint64_t fmul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// a + b, elementwise on the pairs (round to nearest)
+__device__ __forceinline__ uint64_t fadd_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace tt

@@ -100,6 +100,10 @@ struct UnmaskParams {
   int32_t* n_masked;
   uint8_t* ws;
   size_t off_row_cnt, off_seq_cnt, off_partials, off_conf, off_argmax;
+  int32_t batch;               // B
+  size_t off_done;             // 64-bit word: (sequences committed << 32) + masked positions left
+  const int32_t* skip_if;      // early exit of a loop: non-zero => do nothing
+  int32_t* all_done;           // set to 1 when no sequence has a masked position left
 };
 
 constexpr int kUnmaskThreads = 256;
@@ -163,6 +167,19 @@ __device__ void commit_sequence(const UnmaskParams& p, int b, const float* conf_
     const int committed = min(K, n_masked);
     p.n_committed[b] = committed;
     p.n_masked[b] = n_masked - committed;
+    if (p.all_done) {
+      // one 64-bit ticket counts the committed sequences (high half) and sums their masked
+      // positions left (low half); the last sequence reads the total, returns the word to zero
+      // and raises the loop's done word when nothing is left masked
+      unsigned long long* word = reinterpret_cast<unsigned long long*>(p.ws + p.off_done);
+      const unsigned long long left = (unsigned long long)(unsigned)(n_masked - committed);
+      const unsigned long long old = atomicAdd(word, (1ull << 32) | left);
+      if ((old >> 32) == (unsigned long long)(p.batch - 1)) {
+        const unsigned long long total = (old & 0xffffffffull) + left;
+        *word = 0ull;
+        if (total == 0) *p.all_done = 1;
+      }
+    }
   }
 }
 
@@ -181,6 +198,11 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
   constexpr int N = VT::kN;
   pdl_trigger();
   pdl_wait();
+  if (skip_requested(p.skip_if)) {
+    // a step after the block completed: nothing to do; the done word stays raised
+    if (blockIdx.x == 0 && threadIdx.x == 0 && p.all_done) *p.all_done = 1;
+    return;
+  }
   const long long cta = blockIdx.x;
   if (cta >= p.p_eff) return;
   const int tid = threadIdx.x;
@@ -207,8 +229,13 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
     const int vb = (int)(seg - row_beg), ve = (int)(seg_end - row_beg);   // vectors of this row
     const uint4* vp = base + row_beg;
 
-    float m = -INFINITY, s = 0.f;
+    // running state: m, the lowest index attaining it, and sum 2^(c (x - m)) kept as two packed
+    // pairs of partial sums (four independent accumulation chains)
+    float m = -INFINITY;
     int32_t idx = 0x7fffffff;
+    const uint64_t c2 = pack_f32x2(c, c);
+    uint64_t nmc2 = pack_f32x2(0.f, 0.f);
+    uint64_t acc[2] = {pack_f32x2(0.f, 0.f), pack_f32x2(0.f, 0.f)};
     auto consume = [&](const uint4& raw, int vi_global) {
       const int vbase = vi_global * N;
       float x[N];
@@ -219,20 +246,32 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
         for (int k = 0; k < N; ++k)   // static indices keep x[] in registers
           if (k == r) x[k] = -INFINITY;
       }
-      float vm = x[0];
-      int vi = 0;
-#pragma unroll
-      for (int k = 1; k < N; ++k) {
-        if (x[k] > vm) { vm = x[k]; vi = k; }
+      float vm;
+      if constexpr (N == 8) {
+        vm = fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
+      } else {
+        vm = fmax3(x[0], x[1], fmaxf(x[2], x[3]));
       }
       if (vm > m) {
-        s = (m == -INFINITY) ? 0.f : s * ex2(c * (m - vm));
+        // a new running maximum (rare once a row's first vectors have been seen): its lowest
+        // index in this vector, and the partial sums moved to the new base
+        int vi = N - 1;
+#pragma unroll
+        for (int k = N - 1; k >= 0; --k)
+          if (x[k] == vm) vi = k;
+        const float f = (m == -INFINITY) ? 0.f : ex2(c * (m - vm));
+        const uint64_t f2 = pack_f32x2(f, f);
+        acc[0] = fmul_f32x2(acc[0], f2);
+        acc[1] = fmul_f32x2(acc[1], f2);
         m = vm;
         idx = vbase + vi;
+        nmc2 = pack_f32x2(-c * m, -c * m);
       }
-      const float nmc = -c * m;
 #pragma unroll
-      for (int k = 0; k < N; ++k) s += ex2(fmaf(x[k], c, nmc));
+      for (int k = 0; k < N / 2; ++k) {
+        const uint64_t e2 = ffma_f32x2(pack_f32x2(x[2 * k], x[2 * k + 1]), c2, nmc2);
+        acc[k & 1] = fadd_f32x2(acc[k & 1], pack_f32x2(ex2(lo_f32(e2)), ex2(hi_f32(e2))));
+      }
     };
     // this thread's vectors vb + tid + i * kUnmaskThreads, i < nv, stream through its ring: the
     // copy of vector i + kUnmaskRing is issued once vector i has been consumed, so kUnmaskRing
@@ -253,7 +292,8 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
     cp_async_wait<0>();
 
     // ---- CTA reduction (warp shuffles, then across warps), lowest index on ties
-    RedState st{m, s, idx};
+    const uint64_t accs = fadd_f32x2(acc[0], acc[1]);
+    RedState st{m, lo_f32(accs) + hi_f32(accs), idx};
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       RedState o;
@@ -322,6 +362,7 @@ static UnmaskLayout layout_for(int rows, int batch, int grid) {
   };
   L.row_cnt = take(sizeof(int) * (size_t)rows);
   L.seq_cnt = take(sizeof(int) * (size_t)batch);
+  L.done = take(sizeof(unsigned long long));
   L.partials = take(sizeof(UnmaskPartial) * ((size_t)rows + (size_t)grid));
   L.conf = take(sizeof(float) * (size_t)rows);
   L.argmax = take(sizeof(int32_t) * (size_t)rows);
@@ -356,7 +397,7 @@ int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cud
   p.exclude_mask_token = a->exclude_mask_token;
   p.remaining_steps = a->remaining_steps;
   p.sampler = a->sampler;
-  p.keep_masked = a->keep_masked;
+  p.keep_masked = predict_noise_keep(a->block_size, a->keep_masked, a->noise_steps, a->noise_step);
   p.tokens = a->tokens;
   p.is_masked = a->is_masked;
   p.conf_out = a->conf;
@@ -369,6 +410,10 @@ int unmask_launch(const tt_unmask_args_t* a, const UnmaskPlan& pl, void* ws, cud
   p.off_partials = pl.layout.partials;
   p.off_conf = pl.layout.conf;
   p.off_argmax = pl.layout.argmax;
+  p.batch = a->batch;
+  p.off_done = pl.layout.done;
+  p.skip_if = a->skip_if;
+  p.all_done = a->all_done;
   if (a->dtype == TT_BF16)
     launch_pdl(unmask_kernel<__nv_bfloat16>, dim3(pl.grid), dim3(kUnmaskThreads), 0, stream, p);
   else
@@ -456,6 +501,12 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_unmask_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (skip_requested(u.skip_if)) {
+    // a step after the block completed: release TMEM and leave; the done word stays raised
+    if (warp == 1) tmem_dealloc(tmem, kLmTmemCols);
+    if (blockIdx.x == 0 && tid == 0 && u.all_done) *u.all_done = 1;
+    return;
+  }
   volatile int* abort_flag = &sm.abort_flag;
   auto fail = [&](uint32_t detail) {
     report_error(hdr, TT_ERR_DEVICE_TIMEOUT, detail);
@@ -664,7 +715,7 @@ bool lm_make_map(CUtensorMap* m, const void* base, int D, long long rows) {
 
 struct LmLayout {
   int n_mt, nvr;
-  size_t parts, mt_cnt, seq_cnt, conf, argmax, total;
+  size_t parts, mt_cnt, seq_cnt, done, conf, argmax, total;
 };
 
 LmLayout lm_layout(const tt_lmhead_unmask_args_t* a, int num_sms) {
@@ -681,6 +732,7 @@ LmLayout lm_layout(const tt_lmhead_unmask_args_t* a, int num_sms) {
   L.parts = take(sizeof(UnmaskPartial) * (size_t)L.n_mt * L.nvr * 128);
   L.mt_cnt = take(sizeof(int) * (size_t)L.n_mt);
   L.seq_cnt = take(sizeof(int) * (size_t)a->batch);
+  L.done = take(sizeof(unsigned long long));
   L.conf = take(sizeof(float) * (size_t)M);
   L.argmax = take(sizeof(int32_t) * (size_t)M);
   L.total = off;
@@ -706,7 +758,7 @@ int lmhead_unmask_launch(const tt_lmhead_unmask_args_t* a, void* ws, cudaStream_
   u.exclude_mask_token = a->exclude_mask_token;
   u.remaining_steps = a->remaining_steps;
   u.sampler = a->sampler;
-  u.keep_masked = a->keep_masked;
+  u.keep_masked = predict_noise_keep(a->block_size, a->keep_masked, a->noise_steps, a->noise_step);
   u.tokens = a->tokens;
   u.is_masked = a->is_masked;
   u.conf_out = a->conf;
@@ -717,6 +769,10 @@ int lmhead_unmask_launch(const tt_lmhead_unmask_args_t* a, void* ws, cudaStream_
   u.off_seq_cnt = L.seq_cnt;
   u.off_conf = L.conf;
   u.off_argmax = L.argmax;
+  u.batch = a->batch;
+  u.off_done = L.done;
+  u.skip_if = a->skip_if;
+  u.all_done = a->all_done;
   p.M = M;
   p.D = a->hidden;
   p.V = a->vocab;
@@ -759,29 +815,53 @@ static __device__ __align__(256) uint8_t g_unmask_scratch[kStaticScratchBytes];
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
+// Per device: the context whose copy of the scratch was last set up, and its address. A context
+// that is destroyed and created again (cudaDeviceReset, or a runtime that tears down the primary
+// context) loads this module afresh, so the symbol may move: the set-up runs again whenever the
+// current context or the looked-up address differs from the recorded one.
+void* g_static_ctx[kMaxDevices] = {};
 uint8_t* g_static_ptr[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  }
+  return fn;
+}
 }  // namespace
 
 int unmask_launch_static(const tt_unmask_args_t* a, cudaStream_t stream) {
-  const int rows = a->batch * a->block_size;
+  const long long rows = (long long)a->batch * a->block_size;
   if (rows > kStaticMaxRows) return TT_ERR_WORKSPACE_TOO_SMALL;
   const UnmaskLayout L = layout_for(kStaticMaxRows, kStaticMaxRows, kStaticMaxGrid);
   if (L.total > kStaticScratchBytes) return TT_ERR_WORKSPACE_TOO_SMALL;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TT_ERR_CUDA;
-  uint8_t* ws = nullptr;
+  // The array's device address, looked up on every call: a host-side table lookup that allocates
+  // nothing (the host-side name g_unmask_scratch is only a stand-in, never a device address).
+  // The lookup also initialises the runtime's context for this device if nothing has yet.
+  void* sym = nullptr;
+  if (cudaGetSymbolAddress(&sym, g_unmask_scratch) != cudaSuccess || !sym) return TT_ERR_CUDA;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return TT_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(sym);
   {
     std::lock_guard<std::mutex> lock(g_static_mu);
-    ws = g_static_ptr[dev];
-    if (!ws) {
-      // Setup, once per device, with that device current: resolve the array's address and clear
-      // the header and the ticket counters (everything before the partial slots), stream-ordered
-      // before the first launch.
-      void* sym = nullptr;
-      if (cudaGetSymbolAddress(&sym, g_unmask_scratch) != cudaSuccess || !sym) return TT_ERR_CUDA;
-      if (cudaMemsetAsync(sym, 0, L.partials, stream) != cudaSuccess) return TT_ERR_CUDA;
-      ws = static_cast<uint8_t*>(sym);
+    if (g_static_ctx[dev] != static_cast<void*>(ctx) || g_static_ptr[dev] != ws) {
+      // Set-up, once per device and context, with that device current: clear the header and
+      // the ticket counters (everything before the partial slots), stream-ordered before the
+      // first launch. (A freshly loaded module holds zeros already; the clearing makes the state
+      // explicit rather than relying on it.)
+      if (cudaMemsetAsync(ws, 0, L.partials, stream) != cudaSuccess) return TT_ERR_CUDA;
       g_static_ptr[dev] = ws;
+      g_static_ctx[dev] = static_cast<void*>(ctx);
     }
   }
   UnmaskPlan pl = unmask_plan(a, device_sm_count());
@@ -796,9 +876,10 @@ int unmask_launch_static(const tt_unmask_args_t* a, cudaStream_t stream) {
 constexpr int kTauThreads = 128;
 
 __global__ void __launch_bounds__(kTauThreads) block_tau_kernel(const uint8_t* __restrict__ is_masked, int B, int S,
-                                                                float* __restrict__ tau) {
+                                                                float* __restrict__ tau, const int32_t* skip_if) {
   pdl_trigger();
   pdl_wait();
+  if (skip_requested(skip_if)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x * (kTauThreads / 32) + warp;
   if (b >= B) return;
@@ -809,9 +890,11 @@ __global__ void __launch_bounds__(kTauThreads) block_tau_kernel(const uint8_t* _
   if (lane == 0) tau[b] = (float)n / (float)S;
 }
 
-int block_tau_launch(const uint8_t* is_masked, int B, int S, float* tau, cudaStream_t stream) {
+int block_tau_launch(const uint8_t* is_masked, int B, int S, float* tau, const int32_t* skip_if,
+                     cudaStream_t stream) {
   const int per = kTauThreads / 32;
-  return launch_pdl(block_tau_kernel, dim3((B + per - 1) / per), dim3(kTauThreads), 0, stream, is_masked, B, S, tau) ==
+  return launch_pdl(block_tau_kernel, dim3((B + per - 1) / per), dim3(kTauThreads), 0, stream, is_masked, B, S, tau,
+                    skip_if) ==
                  cudaSuccess
              ? TT_OK
              : TT_ERR_CUDA;

@@ -27,6 +27,12 @@
  *     word in the caller's workspace, skips the offending work, and tt_get_device_error()
  *     reports it as TT_ERR_DEVICE or TT_ERR_DEVICE_TIMEOUT.
  *   - Inputs must be finite. NaN/Inf inputs give unspecified (but non-faulting) results.
+ *   - Early exit of a multi-step loop (Algorithm 2 finishes a block within T steps, often sooner):
+ *     every args struct (and tt_block_tau) takes an optional device word `skip_if`. When it is
+ *     non-NULL and holds a non-zero value once the kernel's inputs are ready, the call does
+ *     nothing: no output, workspace or error word is touched. The unmask entries can set such a
+ *     word (`all_done`) when no sequence of the batch has a masked position left, so the later
+ *     steps of a loop captured in one CUDA graph cost only their launches.
  *   - Workspaces must be zero-filled (cudaMemset) before their first use. Their layout depends
  *     on the argument sizes; the kernels restore the merge tickets of that layout to zero, so a
  *     workspace can be reused without re-zeroing by calls with the same sizes. Zero it again
@@ -107,6 +113,7 @@ typedef struct {
   int32_t ctx_stride;        /* contiguous: rows per sequence slab (>= every L_b) */
   void* out;
   float* lse;                /* optional */
+  const int32_t* skip_if;    /* optional device word: non-zero => the call does nothing */
 } tt_attn_args_t;
 
 /* Bytes of workspace tt_denoise_attn needs for these arguments (0 if the args are invalid). */
@@ -165,6 +172,7 @@ typedef struct {
   const float* norm_w;
   const void* f;
   void* out;
+  const int32_t* skip_if;    /* optional device word: non-zero => the call does nothing */
 } tt_adaln_args_t;
 
 size_t tt_adaln_workspace_bytes(const tt_adaln_args_t* args);
@@ -193,8 +201,10 @@ typedef enum {
  *   predicted and the least confident ones are re-masked following the noise schedule, i.e. the
  *   (n_masked - keep_masked) most confident masked positions are committed (confidence
  *   descending, position ascending) and min(n_masked, keep_masked) stay masked; gamma and
- *   remaining_steps are ignored. For the linear schedule alpha_t = 1 - t over T steps,
- *   keep_masked after step r is floor(S * (T - r) / T).
+ *   remaining_steps are ignored. With noise_steps = T > 0 the library derives keep_masked itself
+ *   from the linear schedule alpha_t = 1 - t (the paper §2.2, Eq. (3)): after step r = noise_step
+ *   of T the masked fraction is t = (T - r) / T, so keep_masked = floor(S * (T - r) / T)
+ *   (tt_linear_schedule_keep); the keep_masked field is then ignored.
  * Layouts: logits [B][S][V] E; tokens [B][S] int32 (in/out); is_masked [B][S] uint8 (in/out,
  *   0/1); conf [B][S] float and argmax [B][S] int32 (optional outputs, may be NULL);
  *   n_committed, n_masked [B] int32 outputs. exclude_mask_token != 0 removes the logit of
@@ -219,8 +229,20 @@ typedef struct {
   int32_t* n_committed;
   int32_t* n_masked;
   int32_t sampler;           /* tt_sampler_t; 0 (TT_SAMPLER_CONFIDENCE) when zero-initialised */
-  int32_t keep_masked;       /* TT_SAMPLER_PREDICT_NOISE: masked positions to keep, >= 0 */
+  int32_t keep_masked;       /* TT_SAMPLER_PREDICT_NOISE, noise_steps == 0: masked positions to keep, >= 0 */
+  int32_t noise_steps;       /* TT_SAMPLER_PREDICT_NOISE: T > 0 derives keep_masked from the linear
+                                schedule; 0 uses keep_masked as given */
+  int32_t noise_step;        /* r in 1..noise_steps when noise_steps > 0 */
+  const int32_t* skip_if;    /* optional device word: non-zero => the call does nothing */
+  int32_t* all_done;         /* optional device word: set to 1 when, after this step, no sequence
+                                has a masked position left (never cleared by the library) */
 } tt_unmask_args_t;
+
+/* The linear noise schedule of the predict-and-noise sampler, the paper §2.2 Eq. (3) with
+ * alpha_t = 1 - t: positions of a block of block_size that stay masked after step `step` of
+ * `steps`, floor(block_size * (steps - step) / steps). Host function; returns -1 unless
+ * block_size >= 1, steps >= 1 and 1 <= step <= steps. */
+int32_t tt_linear_schedule_keep(int32_t block_size, int32_t steps, int32_t step);
 
 size_t tt_unmask_workspace_bytes(const tt_unmask_args_t* args);
 int tt_unmask_step(const tt_unmask_args_t* args, void* workspace, size_t workspace_bytes,
@@ -282,6 +304,10 @@ typedef struct {
   int32_t* n_masked;
   int32_t sampler;
   int32_t keep_masked;
+  int32_t noise_steps;
+  int32_t noise_step;
+  const int32_t* skip_if;    /* as in tt_unmask_args_t */
+  int32_t* all_done;         /* as in tt_unmask_args_t */
 } tt_lmhead_unmask_args_t;
 
 size_t tt_lmhead_unmask_workspace_bytes(const tt_lmhead_unmask_args_t* args);
@@ -300,8 +326,9 @@ int tt_lmhead_unmask_step(const tt_lmhead_unmask_args_t* args, void* workspace, 
  * k_new[b] / v_new[b] through page_table[b] (position p lives in page page_table[b][p / page_size],
  * slot p % page_size); the pages holding positions >= ceil(L / page_size) * page_size are taken
  * from the top of the free stack, in order, and entered in page_table[b]; ctx_lens[b] += S.
- * Pages are allocated with one atomic per sequence, so which free pages a sequence receives
- * depends on the order the sequences run in (the content each sequence sees does not).
+ * Pages are claimed per sequence with a compare-and-swap on *free_count that never lowers it
+ * below the claim, so a sequence that cannot be served changes nothing; which free pages a
+ * sequence receives depends on the order the sequences run in (the content each sees does not).
  *
  *   k_new, v_new   device [batch][block_size][num_kv_heads][head_dim] (dtype)
  *   k_ctx, v_ctx   device paged pool [num_pages][page_size][num_kv_heads][head_dim] (dtype), written
@@ -311,8 +338,10 @@ int tt_lmhead_unmask_step(const tt_lmhead_unmask_args_t* args, void* workspace, 
  *   free_count     device int32 scalar, in/out (decreases by the pages taken)
  * Errors (host): TT_ERR_INVALID_ARGUMENT for null pointers or sizes < 1; TT_ERR_UNSUPPORTED unless
  * head_dim * element size is a multiple of 16 bytes and the four tensors are 16-byte aligned.
- * Errors (device, via tt_get_device_error; the sequence is left unchanged): the free stack is too
- * short, or the context would need more than max_pages_per_seq pages.
+ * Errors (device, via tt_get_device_error; the failing sequence, its page_table row and the free
+ * stack are left unchanged; the other sequences proceed): the free stack is too short, an entry
+ * it would hand out is not a page id in [0, num_pages), or the context would need more than
+ * max_pages_per_seq pages.
  * Workspace: tt_kv_append_workspace_bytes() (the error word), zero-filled before first use.
  * ------------------------------------------------------------------------------------------- */
 typedef struct {
@@ -339,10 +368,26 @@ int tt_kv_append(const tt_kv_append_args_t* args, void* workspace, size_t worksp
  * loop (captured in one CUDA graph) needs no host round trip between steps.
  *   is_masked  device u8 [batch][block_size], 1 = still masked
  *   tau        device float [batch], written
+ *   skip_if    optional device word (NULL = none): non-zero => nothing is written
  * Errors: TT_ERR_INVALID_ARGUMENT (null pointer, batch < 1, block_size < 1); TT_ERR_CUDA on a
  * failed launch. No workspace.
  * ------------------------------------------------------------------------------------------- */
-int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, tt_stream_t stream);
+int tt_block_tau(const uint8_t* is_masked, int32_t batch, int32_t block_size, float* tau, const int32_t* skip_if,
+                 tt_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * tt_probe_bounded_wait: a diagnostic of the library's failure path (the paper has no
+ * counterpart). Launches one thread that waits, with the same bounded wait the kernels use, on a
+ * shared-memory barrier that nothing ever arrives on. After limit_us microseconds (1 ..
+ * 1000000; the kernels' own limit is one second) the wait gives up, the kernel records
+ * TT_ERR_DEVICE_TIMEOUT with detail TT_DETAIL_WAIT_PROBE in the workspace's error word and
+ * returns: no trap, no endless wait, the context stays usable. tt_get_device_error() then
+ * reports it. workspace: any workspace of >= 256 bytes (its header is used). Errors (host):
+ * TT_ERR_INVALID_ARGUMENT for a null workspace or a limit outside 1 .. 1000000; TT_ERR_CUDA on
+ * a failed launch.
+ * ------------------------------------------------------------------------------------------- */
+#define TT_DETAIL_WAIT_PROBE 0x1ffu
+int tt_probe_bounded_wait(void* workspace, uint32_t limit_us, tt_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Device-side error word of a workspace (any of the three). Synchronises `stream`, reads the

@@ -46,10 +46,15 @@ def assert_close_bf16_rounded(gpu: torch.Tensor, ref: np.ndarray, what: str = ""
 
 
 def check_unmask(tokens_in, masked_in, logits, gamma, inv_temp, tokens_gpu, masked_gpu, nc_gpu, nm_gpu,
-                 conf_gpu=None, arg_gpu=None, exclude_token=None, remaining_steps=0):
+                 conf_gpu=None, arg_gpu=None, exclude_token=None, remaining_steps=0, oracle_conf_arg=None):
     """Compares one GPU unmask step with the oracle; returns the number of positions in the
-    gamma band (whose commit decision is allowed to differ)."""
-    conf, arg = O.confidence_argmax(np64(logits), inv_temp, exclude_token)
+    gamma band (whose commit decision is allowed to differ). oracle_conf_arg: the oracle's
+    (confidence, argmax) of these logits when the caller has them already (logits is then
+    unused)."""
+    if oracle_conf_arg is None:
+        conf, arg = O.confidence_argmax(np64(logits), inv_temp, exclude_token)
+    else:
+        conf, arg = oracle_conf_arg
     tin = tokens_in.cpu().numpy().astype(np.int64)
     min_ = masked_in.cpu().numpy().astype(bool)
     tg = tokens_gpu.cpu().numpy().astype(np.int64)

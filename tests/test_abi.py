@@ -164,10 +164,7 @@ def test_adaln_workspace(lib):
 ])
 def test_block_tau_host_validation(lib, ptrs, batch, S):
     # rejected on the host before any launch (the pointers are never dereferenced)
-    f = lib.tt_block_tau
-    f.restype = ctypes.c_int
-    f.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
-    assert f(ptrs[0], batch, S, ptrs[1], None) == 1   # TT_ERR_INVALID_ARGUMENT
+    assert lib.tt_block_tau(ptrs[0], batch, S, ptrs[1], None, None) == 1   # TT_ERR_INVALID_ARGUMENT
 
 
 def test_kv_append_host_validation(lib):
@@ -224,3 +221,65 @@ def test_lmhead_host_validation(lib):
         assert lib.tt_lmhead_unmask_step(ctypes.byref(a), ws, 1 << 20, None) == status, field
         setattr(a, field, good)
     assert lib.tt_lmhead_unmask_step(ctypes.byref(a), ws, 64, None) == Bd.TT_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_linear_schedule_keep_is_the_golden_table(lib):
+    # the library's schedule (a host function) against the hand-derived table
+    import json
+    cases = json.load(open(os.path.join(ROOT, "tests", "golden", "noise_schedule_linear.json")))["cases"]
+    for c in cases:
+        got = [lib.tt_linear_schedule_keep(c["S"], c["T"], r) for r in range(1, c["T"] + 1)]
+        assert got == c["keep"], c
+    for S, T, r in ((0, 4, 1), (16, 0, 1), (16, 4, 0), (16, 4, 5)):
+        assert lib.tt_linear_schedule_keep(S, T, r) == -1
+
+
+def test_noise_schedule_fields_validated(lib):
+    from denoiser_attention_b200 import binding as Bd
+    a = Bd.UnmaskArgs()
+    a.batch, a.block_size, a.vocab, a.dtype = 2, 16, 1024, Bd.TT_F32
+    for name in ("logits", "tokens", "is_masked", "n_committed", "n_masked"):
+        setattr(a, name, 0x1000)
+    a.gamma, a.inv_temperature = 0.8, 1.0
+    a.sampler, a.keep_masked = Bd.TT_SAMPLER_PREDICT_NOISE, -1      # ignored once a schedule is given
+    for steps, step, ok in ((6, 1, True), (6, 6, True), (6, 0, False), (6, 7, False), (-1, 1, False)):
+        a.noise_steps, a.noise_step = steps, step
+        assert (lib.tt_unmask_workspace_bytes(ctypes.byref(a)) > 0) == ok, (steps, step)
+    m = Bd.LmheadUnmaskArgs()
+    m.batch, m.block_size, m.hidden, m.vocab, m.dtype = 2, 16, 256, 4096, Bd.TT_BF16
+    for name in ("x", "w", "tokens", "is_masked", "n_committed", "n_masked"):
+        setattr(m, name, 0x1000)
+    m.gamma, m.inv_temperature = 0.8, 1.0
+    m.sampler, m.keep_masked, m.noise_steps, m.noise_step = Bd.TT_SAMPLER_PREDICT_NOISE, -1, 16, 17
+    assert lib.tt_lmhead_unmask_workspace_bytes(ctypes.byref(m)) == 0
+    m.noise_step = 16
+    assert lib.tt_lmhead_unmask_workspace_bytes(ctypes.byref(m)) > 0
+
+
+def test_sizes_beyond_32_bit_rows_rejected(lib):
+    # batch * block_size must fit the kernels' 32-bit row index; rows * vocab their 64-bit cuts
+    from denoiser_attention_b200 import binding as Bd
+    a = Bd.UnmaskArgs()
+    a.dtype, a.gamma, a.inv_temperature = Bd.TT_F32, 0.8, 1.0
+    for name in ("logits", "tokens", "is_masked", "n_committed", "n_masked"):
+        setattr(a, name, 0x1000)
+    a.batch, a.block_size, a.vocab = 1 << 22, 1024, 4                  # 2^32 rows
+    assert lib.tt_unmask_step(ctypes.byref(a), ctypes.c_void_p(0x2000), 1 << 40, None) == Bd.TT_ERR_UNSUPPORTED
+    assert lib.tt_unmask_step_noalloc(ctypes.byref(a), None) == Bd.TT_ERR_UNSUPPORTED
+    a.batch, a.block_size, a.vocab = 1 << 14, 1024, 1 << 20            # 2^44 logits
+    assert lib.tt_unmask_workspace_bytes(ctypes.byref(a)) == 0
+    m = Bd.LmheadUnmaskArgs()
+    m.batch, m.block_size, m.hidden, m.vocab, m.dtype = 1 << 22, 1024, 256, 4096, Bd.TT_BF16
+    for name in ("x", "w", "tokens", "is_masked", "n_committed", "n_masked"):
+        setattr(m, name, 0x1000)
+    m.gamma, m.inv_temperature = 0.8, 1.0
+    assert lib.tt_lmhead_unmask_workspace_bytes(ctypes.byref(m)) == 0
+    t = _attn_args(batch=1 << 22, block_size=1024)
+    assert lib.tt_denoise_attn_workspace_bytes(ctypes.byref(t)) == 0
+
+
+def test_probe_bounded_wait_host_validation(lib):
+    ws = ctypes.c_void_p(0x2000)
+    assert lib.tt_probe_bounded_wait(None, 100, None) == B.TT_ERR_INVALID_ARGUMENT
+    assert lib.tt_probe_bounded_wait(ws, 0, None) == B.TT_ERR_INVALID_ARGUMENT
+    assert lib.tt_probe_bounded_wait(ws, 1000001, None) == B.TT_ERR_INVALID_ARGUMENT

@@ -128,3 +128,61 @@ def test_attention_over_the_grown_cache(cuda_lib):
         ks[b, :new_lens[b]], vs[b, :new_lens[b]] = ck[b], cv[b]
     want = O.denoise_attention(np64(q), np64(kb), np64(vb), ks, vs, new_lens)
     assert_close_attn(out.cpu(), want, torch.bfloat16, "grown cache")
+
+
+@pytest.mark.parametrize("trial", range(4))
+def test_concurrent_out_of_pages_keeps_the_stack_consistent(cuda_lib, trial):
+    # 96 sequences claim 1 or 2 pages each from a stack holding far fewer than they need, in one
+    # launch: the sequences that advance hold distinct pages, exactly the top of the stack; the
+    # count says how many entries are left; the sequences that fail are untouched
+    rs = np.random.default_rng(50 + trial)
+    Bn, S, page_size, Hkv, d = 96, 16, 16, 1, 64
+    lens = [int(x) for x in rs.integers(0, 64, Bn)]
+    have = [(L + page_size - 1) // page_size for L in lens]
+    need = [(L + S + page_size - 1) // page_size - h for L, h in zip(lens, have)]
+    max_pages = max(h + n for h, n in zip(have, need)) + 1
+    n_free = sum(need) // 3
+    num_pages = sum(have) + n_free + 5
+    k_ctx, v_ctx, table, _, k_new, v_new = _pool(lens, S, Hkv, d, torch.float32, page_size, num_pages, max_pages,
+                                                 seed=60 + trial)
+    used = set(table[table >= 0].tolist())
+    free = torch.tensor([p for p in rs.permutation(num_pages).tolist() if p not in used][:n_free],
+                        dtype=torch.int32)
+    t, st, detail = _run(k_ctx, v_ctx, table, free, k_new, v_new, lens)
+    assert st == B.TT_ERR_DEVICE and detail == 4
+    new_lens = t["lens"].cpu().tolist()
+    tab = t["table"].cpu()
+    count = int(t["count"].item())
+    ok = [nl == L + S for nl, L in zip(new_lens, lens)]
+    assert all(nl in (L, L + S) for nl, L in zip(new_lens, lens))
+    assert any(ok) and not all(ok)
+    claimed = []
+    for b in range(Bn):
+        assert tab[b, :have[b]].tolist() == table[b, :have[b]].tolist()
+        if ok[b]:
+            claimed += tab[b, have[b]:have[b] + need[b]].tolist()
+        else:
+            assert tab[b].tolist() == table[b].tolist()        # a failed sequence keeps its row
+    assert len(set(claimed)) == len(claimed)                    # no page handed out twice
+    assert count == n_free - len(claimed)                       # the count matches what was taken
+    assert sorted(claimed) == sorted(free[count:].tolist())     # exactly the top of the stack
+    assert not (set(claimed) & used)
+    # content of the sequences that advanced
+    old_k, old_v = O.gather_context(np64(k_ctx), np64(v_ctx), lens, table.numpy(), page_size)
+    want_k, want_v, _ = O.append_block(old_k, old_v, np64(k_new), np64(v_new))
+    got_k, got_v = O.gather_context(np64(t["k_ctx"]), np64(t["v_ctx"]), new_lens, tab.numpy(), page_size)
+    for b in range(Bn):
+        if ok[b]:
+            np.testing.assert_array_equal(got_k[b], want_k[b])
+            np.testing.assert_array_equal(got_v[b], want_v[b])
+
+
+def test_bad_page_id_in_the_stack_changes_nothing(cuda_lib):
+    lens, S, page_size = [0, 16], 16, 16
+    k_ctx, v_ctx, table, free, k_new, v_new = _pool(lens, S, 1, 64, torch.float32, page_size, 6, 4, seed=7)
+    free = torch.tensor([free[0].item(), 99], dtype=torch.int32)       # the top entry is not a page id
+    t, st, detail = _run(k_ctx, v_ctx, table, free, k_new, v_new, lens)
+    assert st == B.TT_ERR_DEVICE and detail == 1
+    assert int(t["count"].item()) == 2
+    assert t["lens"].cpu().tolist() == lens
+    assert torch.equal(t["table"].cpu(), table)

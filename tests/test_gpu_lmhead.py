@@ -113,3 +113,49 @@ def test_lmhead_excludes_mask_token(cuda_lib):
     conf_or, arg_or = O.confidence_argmax(logits, 1.0, exclude_token=3)
     assert int(arg[0, 0]) == int(arg_or[0, 0]) != 3
     assert np.all(np.abs(conf.cpu().double().numpy() - conf_or) <= 2e-5 * conf_or + 1e-7)
+
+
+@pytest.mark.parametrize("rem", [1, 3])
+def test_lmhead_remaining_steps_matches_oracle(cuda_lib, rem):
+    # the confidence sampler with remaining_steps > 0 (the T - r + 1 of Algorithm 2): at least
+    # ceil(n_masked / remaining_steps) of the most confident masked positions commit
+    B, S, D, V, gamma = 6, 16, 256, 4096, 0.97
+    x, w, tokens, masked = _inputs(B, S, D, V, seed=40 + rem)
+    dev = "cuda"
+    t, m = tokens.to(dev), masked.to(dev)
+    nc, nm, conf, arg = api.lmhead_unmask_step(x.to(dev), w.to(dev), t, m, gamma=gamma, remaining_steps=rem)
+    torch.cuda.synchronize()
+    logits = O.lmhead_logits(np64(x), np64(w))
+    conf_or, arg_or, clear = _check_reduction(logits, conf.cpu().double().numpy(), arg.cpu().numpy())
+    t_or, m_or, nc_or, nm_or, _, _ = O.unmask_step(tokens.numpy(), masked.numpy().astype(bool), logits, gamma,
+                                                   remaining_steps=rem)
+    # the schedule's count is exact; the chosen positions compare where the ranking and the
+    # threshold are separated by more than the fp32 accumulation error
+    n_in = masked.numpy().astype(np.int64).sum(axis=1)
+    need = np.where(n_in > 0, -(-n_in // rem), 0)
+    assert (nc.cpu().numpy() >= need).all()
+    np.testing.assert_array_equal(nc.cpu().numpy() + nm.cpu().numpy(), n_in)
+    safe = []
+    for b in range(B):
+        c = np.sort(conf_or[b][masked.numpy()[b].astype(bool)])
+        sep = len(c) < 2 or np.min(np.diff(c)) > 1e-4 * c.max()
+        safe.append(sep and not (np.abs(conf_or[b] - gamma) <= 1e-4).any() and clear[b].all())
+    safe = np.array(safe)
+    assert safe.sum() >= 1
+    np.testing.assert_array_equal(m.cpu().numpy().astype(bool)[safe], m_or[safe])
+    np.testing.assert_array_equal(t.cpu().numpy()[safe], t_or[safe])
+    np.testing.assert_array_equal(nc.cpu().numpy()[safe], nc_or[safe])
+
+
+def test_lmhead_noise_schedule_in_the_library(cuda_lib):
+    # predict-and-noise from hidden states at step r of T of the linear schedule: the library
+    # derives keep_masked = floor(S (T - r) / T)
+    B, S, D, V, T = 3, 16, 256, 2048, 6
+    x, w, _, _ = _inputs(B, S, D, V, seed=61)
+    dev = "cuda"
+    for r, keep in ((1, 13), (4, 5), (6, 0)):
+        t = torch.full((B, S), 3, dtype=torch.int32, device=dev)
+        m = torch.ones((B, S), dtype=torch.uint8, device=dev)
+        nc, nm, _, _ = api.lmhead_unmask_step(x.to(dev), w.to(dev), t, m, gamma=0.8, noise_schedule=(T, r))
+        torch.cuda.synchronize()
+        assert nm.cpu().tolist() == [keep] * B and nc.cpu().tolist() == [S - keep] * B

@@ -40,11 +40,14 @@ def test_refinement_step_matches_oracle(cuda_lib, name):
     attn = O.denoise_attention(f64(inp.q), f64(inp.k_blk), f64(inp.v_blk), f64(inp.k_ctx), f64(inp.v_ctx),
                                inp.ctx_lens.tolist())
     h_new = O.adaln_gated_residual(f64(ad.h), f64(ad.f), mod)
+    y = O.adaln_norm_modulate(f64(ad.h), f64(ad.norm_w), mod, ad.eps)
     assert_close_attn(out["attn"], attn, w.attn.dtype, name)
     if w.attn.dtype == torch.bfloat16:
         assert_close_bf16_rounded(out["h"], h_new, "residual")
+        assert_close_bf16_rounded(out["y"], y, "modulated RMSNorm")
     else:
         assert np.abs(f64(out["h"]) - h_new).max() <= 1e-5
+        assert np.abs(f64(out["y"]) - y).max() <= 1e-5
     check_unmask(tokens, masked, logits, w.gamma, 1.0, out["tokens"], out["is_masked"], out["n_committed"],
                  out["n_masked"])
 

@@ -154,10 +154,114 @@ def test_predict_noise_schedule_loop(cuda_lib):
     t_or, m_or = np.full((B, S), 3), np.ones((B, S), bool)
     for r in range(1, T + 1):
         logits = synth.logits_normal(100 + r, B, S, V, 3.0, torch.bfloat16)
-        keep = api.linear_schedule_keep(S, T, r)
+        keep = api.linear_schedule_keep(S, T, r)     # computed by the library (tt_linear_schedule_keep)
         api.unmask_step(logits.to(dev), t, m, gamma=0.8, keep_masked=keep)
         t_or, m_or, _, _, _, _ = O.predict_noise_step(t_or, m_or, np64(logits), O.linear_schedule_keep(S, T, r))
         torch.cuda.synchronize()
         assert int(m.sum()) == B * keep
         np.testing.assert_array_equal(t.cpu().numpy(), t_or)
+    assert int(m.sum()) == 0
+
+
+# ---------------------------------------------------------------- the block-sweep workload's grid
+# block sizes S in {4, 8, 16, 32, 64} x softmax temperatures {0.5, 1, 2} (inv_temperature 2, 1,
+# 0.5) x gamma in {0.5, 0.7, 0.8, 0.9, 0.95}, on the full batch of 32 sequences with vocabulary
+# 131072; the oracle's confidences are computed once per (S, temperature) on the host.
+SWEEP_GAMMAS = (0.5, 0.7, 0.8, 0.9, 0.95)
+
+
+def _oracle_conf_chunked(logits, inv_temp, rows=256, exclude_token=None):
+    from oracle import tt_oracle as O
+    B, S, V = logits.shape
+    flat = logits.reshape(B * S, V)
+    conf, arg = [], []
+    for i in range(0, B * S, rows):
+        c, a = O.confidence_argmax(flat[i:i + rows].double().numpy(), inv_temp, exclude_token)
+        conf.append(c)
+        arg.append(a)
+    return np.concatenate(conf).reshape(B, S), np.concatenate(arg).reshape(B, S)
+
+
+@pytest.mark.parametrize("S", [4, 8, 16, 32, 64])
+def test_block_sweep_grid_matches_oracle(cuda_lib, S):
+    from oracle import tt_oracle as O
+    w = synth.workload("sweep_bf16", block_size=S)
+    B = w.attn.batch
+    logits = synth.workload_logits(w)
+    dev = "cuda"
+    lg = logits.to(dev)
+    tokens0 = torch.full((B, S), 3, dtype=torch.int32)
+    masked0 = torch.ones((B, S), dtype=torch.uint8)
+    band = 0
+    for inv_temp in (2.0, 1.0, 0.5):
+        conf_or, arg_or = _oracle_conf_chunked(logits, inv_temp)
+        for gamma in SWEEP_GAMMAS:
+            t, m = tokens0.to(dev), masked0.to(dev)
+            nc, nm, conf, arg = api.unmask_step(lg, t, m, gamma=gamma, inv_temperature=inv_temp)
+            torch.cuda.synchronize()
+            band += check_unmask(tokens0, masked0, None, gamma, inv_temp, t, m, nc, nm, conf, arg,
+                                 oracle_conf_arg=(conf_or, arg_or))
+    print(f"S={S}: positions in the 1e-5 band around gamma over the grid: {band}")
+
+
+def test_batch_workload_unmask_full_size(cuda_lib):
+    # the batch workload's logits at full size: 64 sequences x 16 positions x 131072 (1024 rows,
+    # every CTA range straddles rows and every sequence ticket sees its 16 rows)
+    w = synth.workload("batch_bf16")
+    B, S = w.attn.batch, w.attn.block_size
+    logits = synth.workload_logits(w)
+    g = torch.Generator().manual_seed(2)
+    masked = (torch.rand((B, S), generator=g) < 9 / 16).to(torch.uint8)   # t = 8 of 16: about 9/16 masked
+    tokens = torch.randint(0, 1000, (B, S), generator=g, dtype=torch.int32)
+    tokens[masked.bool()] = 3
+    t, m, nc, nm, conf, arg = _step(logits, tokens, masked, gamma=w.gamma)
+    check_unmask(tokens, masked, logits, w.gamma, 1.0, t, m, nc, nm, conf, arg)
+
+
+@pytest.mark.parametrize("B,S,V,dtype,keep", [
+    (4, 16, 131072, torch.bfloat16, 6),
+    (3, 8, 2048, torch.float32, 2),
+])
+def test_predict_noise_excluding_mask_token(cuda_lib, B, S, V, dtype, keep):
+    from oracle import tt_oracle as O
+    logits = synth.logits_normal(V + keep + 1, B, S, V, 2.0, dtype)
+    logits[:, :, 3] = 40.0                      # the [MASK] logit would win every position unless excluded
+    tokens, masked = _state(B, S, seed=V + 1, frac_masked=0.9)
+    dev = "cuda"
+    t, m = tokens.to(dev), masked.to(dev)
+    nc, nm, conf, arg = api.unmask_step(logits.to(dev), t, m, gamma=0.8, keep_masked=keep, exclude_mask_token=True,
+                                        mask_token_id=3)
+    torch.cuda.synchronize()
+    t_or, m_or, nc_or, nm_or, conf_or, arg_or = O.predict_noise_step(
+        tokens.numpy(), masked.numpy().astype(bool), np64(logits), keep, exclude_token=3)
+    assert (arg.cpu().numpy() != 3).all()
+    np.testing.assert_array_equal(arg.cpu().numpy(), arg_or)
+    assert np.abs(conf.cpu().double().numpy() - conf_or).max() <= 1e-5
+    np.testing.assert_array_equal(nc.cpu().numpy(), nc_or)
+    np.testing.assert_array_equal(nm.cpu().numpy(), nm_or)
+    np.testing.assert_array_equal(t.cpu().numpy(), t_or)
+    np.testing.assert_array_equal(m.cpu().numpy().astype(bool), m_or)
+
+
+def test_predict_noise_schedule_in_the_library(cuda_lib):
+    # noise_schedule=(T, r): the library derives keep_masked from the linear schedule; the T-step
+    # trajectory follows the hand-derived table and the oracle
+    import json
+    import os
+    from oracle import tt_oracle as O
+    golden = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "noise_schedule_linear.json")))
+    case = [c for c in golden["cases"] if c["S"] == 16 and c["T"] == 6][0]
+    B, S, T, V = 3, 16, 6, 4096
+    dev = "cuda"
+    t = torch.full((B, S), 3, dtype=torch.int32, device=dev)
+    m = torch.ones((B, S), dtype=torch.uint8, device=dev)
+    t_or, m_or = np.full((B, S), 3), np.ones((B, S), bool)
+    for r in range(1, T + 1):
+        logits = synth.logits_normal(300 + r, B, S, V, 3.0, torch.bfloat16)
+        nc, nm, _, _ = api.unmask_step(logits.to(dev), t, m, gamma=0.8, noise_schedule=(T, r))
+        t_or, m_or, _, _, _, _ = O.predict_noise_step(t_or, m_or, np64(logits), case["keep"][r - 1])
+        torch.cuda.synchronize()
+        assert nm.cpu().tolist() == [case["keep"][r - 1]] * B
+        np.testing.assert_array_equal(t.cpu().numpy(), t_or)
+        np.testing.assert_array_equal(m.cpu().numpy().astype(bool), m_or)
     assert int(m.sum()) == 0
