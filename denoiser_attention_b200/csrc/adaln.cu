@@ -3,9 +3,10 @@
 // PixArt-alpha: one global MLP from the diffusion time to shared shift/scale/gate, plus a learned
 // per-layer embedding).
 //
-//   COND             tau -> mod[B][3][D]   two launches: per sequence the sinusoid and the two
-//                                          W-wide layers; then the W->3D layer tiled over 32-row
-//                                          slices of W3, each read once for the whole batch
+//   COND             tau -> mod[B][3][D]   three launches, one per layer (F->W with the sinusoid,
+//                                          W->W, W->3D), each tiled over 32-row slices of the
+//                                          weight x 16-sequence chunks, operands staged in shared
+//                                          memory with asynchronous copies
 //   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one CTA per token row
 //   GATED_RESIDUAL   h + gate * f: a vectorised elementwise pass
 // All arithmetic is fp32 (the timestep sinusoid in fp64); bf16 tensors are widened on load and
@@ -48,119 +49,89 @@ __device__ __forceinline__ void phi_row(float tau, int F, float* dst, int tid, i
 
 constexpr int kMaxWidth = 1024;   // F and W bound (host-validated)
 
-// y[o] = act(W[o, :] . x + bias[o]) for o < OUT, x in shared memory; each warp takes four rows at
-// a time (four independent dot products and reductions in flight), lanes stride the row in float4.
-template <bool kSilu>
-__device__ __forceinline__ void cta_gemv(const float* __restrict__ Wt, const float* __restrict__ bias,
-                                         const float* x, int IN, int OUT, float* y) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int o0 = warp * 4; o0 < OUT; o0 += nwarps * 4) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = lane * 4; i < IN; i += 128) {
-      const float4 xv = *reinterpret_cast<const float4*>(x + i);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        if (o0 + r < OUT) {
-          const float4 wv = *reinterpret_cast<const float4*>(Wt + (size_t)(o0 + r) * IN + i);
-          acc[r] = fmaf(wv.x, xv.x, fmaf(wv.y, xv.y, fmaf(wv.z, xv.z, fmaf(wv.w, xv.w, acc[r]))));
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) acc[r] = warp_sum(acc[r]);
-    if (lane < 4 && o0 + lane < OUT) {
-      const float v = (lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3]) + bias[o0 + lane];
-      y[o0 + lane] = kSilu ? silu_f(v) : v;
-    }
-  }
+// 16-byte asynchronous copy global -> shared (L2 only); all of a stage's copies are in flight at
+// once and completed with one wait.
+__device__ __forceinline__ void cp_async16_g2s(void* smem, const void* gmem) {
+  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// COND, first launch: one CTA per sequence b computes a2[b] = SiLU(W2 SiLU(W1 phi(tau_b) + b1) + b2).
-__global__ void __launch_bounds__(kAdalnThreads) adaln_hidden_kernel(const float* __restrict__ tau,
-                                                                     const float* __restrict__ w1,
-                                                                     const float* __restrict__ b1,
-                                                                     const float* __restrict__ w2,
-                                                                     const float* __restrict__ b2, int F, int W,
-                                                                     float* __restrict__ a2,
-                                                                     const int32_t* skip_if) {
-  __shared__ __align__(16) float s_phi[kMaxWidth];
-  __shared__ __align__(16) float s_a1[kMaxWidth];
-  pdl_trigger();
-  pdl_wait();
-  if (skip_requested(skip_if)) return;
-  const int b = blockIdx.x;
-  phi_row(tau[b], F, s_phi, threadIdx.x, blockDim.x);
-  __syncthreads();
-  cta_gemv<true>(w1, b1, s_phi, F, W, s_a1);
-  __syncthreads();
-  cta_gemv<true>(w2, b2, s_a1, W, W, a2 + (size_t)b * W);
+// One layer of the conditioning MLP for a slice of its outputs and a chunk of the sequences:
+//   y[b][o] = act(W[o, :] . x_b + bias[o]) (+ extra[o]),  o in [32 i, 32 i + 32), b in [16 j, 16 j + 16)
+// x_b is phi(tau_b) (kPhi: the timestep sinusoid, computed here) or row b of x. The CTA stages its
+// 32 rows of W (rows padded by 4 floats, so that the quarter-warp float4 reads of 8 rows hit
+// distinct banks) and its 16 input rows in shared memory with asynchronous copies; then lane =
+// output row and warp = a pair of sequences, whose input rows are read as broadcasts.
+constexpr int kRowSlice = 32;
+constexpr int kSeqChunk = 16;
+
+inline size_t rows_smem_bytes(int IN) {
+  return sizeof(float) * ((size_t)kRowSlice * (IN + 4) + (size_t)kSeqChunk * IN);
 }
 
-// COND, second launch: mod[b][o] = W3[o, :] . a2[b] + b3[o] + layer_emb[o] for o < 3D. A CTA
-// owns 32 rows of W3 (in shared memory, rows padded by 4 floats so that the quarter-warp float4
-// reads of 8 rows hit distinct banks) and every sequence: lane = row, warp = a group of sequences
-// whose a2 rows are read as broadcasts; chunks of up to 64 sequences at a time (fewer for wide W,
-// so that the chunk and the W3 slice fit in shared memory).
-constexpr int kOutRows = 32;
-constexpr int kOutSeqChunk = 64;
-inline int out_seq_chunk(int W) { return W <= 256 ? 64 : (W <= 512 ? 32 : 16); }
-inline size_t out_smem_bytes(int W) {
-  return sizeof(float) * ((size_t)kOutRows * (W + 4) + (size_t)out_seq_chunk(W) * W);
-}
-
-__global__ void __launch_bounds__(kAdalnThreads) adaln_out_kernel(const float* __restrict__ w3,
-                                                                  const float* __restrict__ b3,
-                                                                  const float* __restrict__ emb,
-                                                                  const float* __restrict__ a2, int B, int W,
-                                                                  int OUT, int chunk, float* __restrict__ mod,
-                                                                  const int32_t* skip_if) {
+template <bool kPhi, bool kSilu>
+__global__ void __launch_bounds__(kAdalnThreads) adaln_rows_kernel(const float* __restrict__ Wt,
+                                                                   const float* __restrict__ bias,
+                                                                   const float* __restrict__ extra,
+                                                                   const float* __restrict__ x, int B, int IN,
+                                                                   int OUT, float* __restrict__ y,
+                                                                   const int32_t* skip_if) {
   extern __shared__ __align__(16) float s_dyn[];
-  const int WP = W + 4;
-  float* s_w = s_dyn;                          // [32][W + 4]
-  float* s_a = s_dyn + kOutRows * WP;          // [chunk][W]
+  const int INP = IN + 4;
+  float* s_w = s_dyn;                          // [32][IN + 4]
+  float* s_x = s_dyn + kRowSlice * INP;        // [16][IN]
   pdl_trigger();
   pdl_wait();
   if (skip_requested(skip_if)) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int o0 = blockIdx.x * kOutRows;
-  const int nrow = min(kOutRows, OUT - o0);
-  const int wv = W / 4;
-  for (int i = threadIdx.x; i < kOutRows * wv; i += blockDim.x) {
-    const int r = i / wv, c = i - r * wv;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < nrow) v = reinterpret_cast<const float4*>(w3 + (size_t)(o0 + r) * W)[c];
-    *reinterpret_cast<float4*>(s_w + r * WP + 4 * c) = v;
+  const int o0 = blockIdx.x * kRowSlice, b0 = blockIdx.y * kSeqChunk;
+  const int nrow = min(kRowSlice, OUT - o0), nb = min(kSeqChunk, B - b0);
+  const int iv = IN / 4;
+  for (int i = threadIdx.x; i < nrow * iv; i += blockDim.x) {
+    const int r = i / iv, c = i - r * iv;
+    cp_async16_g2s(s_w + r * INP + 4 * c, Wt + (size_t)(o0 + r) * IN + 4 * c);
+  }
+  if (kPhi) {
+    for (int bb = 0; bb < nb; ++bb) phi_row(x[b0 + bb], IN, s_x + bb * IN, threadIdx.x, blockDim.x);
+  } else {
+    for (int i = threadIdx.x; i < nb * iv; i += blockDim.x)
+      cp_async16_g2s(s_x + 4 * i, x + (size_t)b0 * IN + 4 * i);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int bA = 2 * warp, bB = 2 * warp + 1;   // this warp's two sequences of the chunk
+  if (lane >= nrow || bA >= nb) return;
+  float accA = 0.f, accB = 0.f;
+  const float* wrow = s_w + lane * INP;
+  const float* xa = s_x + bA * IN;
+  const float* xb = s_x + (bB < nb ? bB : bA) * IN;
+  for (int k = 0; k < IN; k += 4) {
+    const float4 w = *reinterpret_cast<const float4*>(wrow + k);
+    const float4 u = *reinterpret_cast<const float4*>(xa + k);
+    const float4 v = *reinterpret_cast<const float4*>(xb + k);
+    accA = fmaf(w.x, u.x, fmaf(w.y, u.y, fmaf(w.z, u.z, fmaf(w.w, u.w, accA))));
+    accB = fmaf(w.x, v.x, fmaf(w.y, v.y, fmaf(w.z, v.z, fmaf(w.w, v.w, accB))));
   }
   const int o = o0 + lane;
-  const float add = (lane < nrow) ? b3[o] + emb[o] : 0.f;
-  for (int c0 = 0; c0 < B; c0 += chunk) {
-    const int nb = min(chunk, B - c0);
-    __syncthreads();   // the previous chunk is consumed (and, the first time, s_w is written)
-    for (int i = threadIdx.x; i < nb * wv; i += blockDim.x)
-      reinterpret_cast<float4*>(s_a)[i] = reinterpret_cast<const float4*>(a2 + (size_t)c0 * W)[i];
-    __syncthreads();
-    float acc[kOutSeqChunk / 8];
-#pragma unroll
-    for (int i = 0; i < kOutSeqChunk / 8; ++i) acc[i] = 0.f;
-    for (int k = 0; k < W; k += 4) {
-      const float4 w = *reinterpret_cast<const float4*>(s_w + lane * WP + k);
-#pragma unroll
-      for (int i = 0; i < kOutSeqChunk / 8; ++i) {
-        const int bb = warp + 8 * i;
-        if (bb < nb) {
-          const float4 x = *reinterpret_cast<const float4*>(s_a + bb * W + k);
-          acc[i] = fmaf(w.x, x.x, fmaf(w.y, x.y, fmaf(w.z, x.z, fmaf(w.w, x.w, acc[i]))));
-        }
-      }
-    }
-    if (lane < nrow) {
-#pragma unroll
-      for (int i = 0; i < kOutSeqChunk / 8; ++i) {
-        const int bb = warp + 8 * i;
-        if (bb < nb) mod[(size_t)(c0 + bb) * OUT + o] = acc[i] + add;
-      }
-    }
+  const float add = bias[o] + (extra ? extra[o] : 0.f);
+  float ya = accA + add, yb = accB + add;
+  if (kSilu) {
+    ya = silu_f(ya);
+    yb = silu_f(yb);
   }
+  y[(size_t)(b0 + bA) * OUT + o] = ya;
+  if (bB < nb) y[(size_t)(b0 + bB) * OUT + o] = yb;
+}
+
+template <bool kPhi, bool kSilu>
+static cudaError_t launch_rows(const float* Wt, const float* bias, const float* extra, const float* x, int B, int IN,
+                               int OUT, float* y, const int32_t* skip_if, cudaStream_t stream) {
+  const dim3 grid((OUT + kRowSlice - 1) / kRowSlice, (B + kSeqChunk - 1) / kSeqChunk);
+  return launch_pdl(adaln_rows_kernel<kPhi, kSilu>, grid, dim3(kAdalnThreads), rows_smem_bytes(IN), stream, Wt, bias,
+                    extra, x, B, IN, OUT, y, skip_if);
 }
 
 template <typename T>
@@ -270,32 +241,36 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_gated_residual_kernel(con
 }
 
 size_t adaln_workspace_bytes(const tt_adaln_args_t* a) {
-  if (a->op == TT_ADALN_COND) return kHeaderBytes + sizeof(float) * (size_t)a->batch * a->mlp_width;
+  if (a->op == TT_ADALN_COND) return kHeaderBytes + 2 * sizeof(float) * (size_t)a->batch * a->mlp_width;
   return kHeaderBytes;
 }
 
 int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
   const int B = a->batch, D = a->hidden;
   if (a->op == TT_ADALN_COND) {
-    float* a2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+    float* a1 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+    float* a2 = a1 + (size_t)B * a->mlp_width;
     const int F = a->freq_dim, W = a->mlp_width, OUT = 3 * D;
-    launch_pdl(adaln_hidden_kernel, dim3(B), dim3(kAdalnThreads), 0, stream, a->tau, a->w1, a->b1, a->w2, a->b2, F,
-               W, a2, a->skip_if);
-    const size_t smem = out_smem_bytes(W);
-    static unsigned long long attr_done = 0;   // bit per device ordinal (< 64): the opt-in for W up to 1024
+    // the shared-memory opt-in for inputs up to kMaxWidth wide, once per device (so that no
+    // attribute call happens while a caller captures the stream into a CUDA graph)
+    static unsigned long long attr_done = 0;   // bit per device ordinal (< 64)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
-      size_t max_smem = 0;
-      for (int w = 256; w <= kMaxWidth; w *= 2) max_smem = std::max(max_smem, out_smem_bytes(w));
-      if (cudaFuncSetAttribute(adaln_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem) !=
-          cudaSuccess)
+      const int max_smem = (int)rows_smem_bytes(kMaxWidth);
+      if (cudaFuncSetAttribute(adaln_rows_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(adaln_rows_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(adaln_rows_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               max_smem) != cudaSuccess)
         return TT_ERR_CUDA;
       __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
     }
-    launch_pdl(adaln_out_kernel, dim3((OUT + kOutRows - 1) / kOutRows), dim3(kAdalnThreads), smem, stream, a->w3,
-               a->b3, a->layer_emb, a2, B, W, OUT, out_seq_chunk(W), a->mod, a->skip_if);
+    launch_rows<true, true>(a->w1, a->b1, nullptr, a->tau, B, F, W, a1, a->skip_if, stream);
+    launch_rows<false, true>(a->w2, a->b2, nullptr, a1, B, W, W, a2, a->skip_if, stream);
+    launch_rows<false, false>(a->w3, a->b3, a->layer_emb, a2, B, W, OUT, a->mod, a->skip_if, stream);
   } else if (a->op == TT_ADALN_NORM_MODULATE) {
     const int rows = B * a->block_size;
     if (a->dtype == TT_BF16)

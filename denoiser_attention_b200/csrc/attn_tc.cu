@@ -19,7 +19,7 @@
 // Inside a CTA (384 threads: warpgroup 0 load and MMA, warpgroups 1-2 softmax), two independent
 // softmax streams, one per query tile:
 //   warps 0, 2 TMA producers: warp 0 the CTA's query tiles of the group and the K tiles of 128
-//              tokens (3-stage ring), warp 2 the V tiles (2-stage ring), so that neither ring
+//              tokens (2-stage ring), warp 2 the V tiles (2-stage ring), so that neither ring
 //              waits for the other (128B-swizzled boxes; no multicast)
 //   warp 1     MMA issuer (one thread): for stream j, S_j = Q_j K^T (M=128, N=128, K=128, both
 //              operands from shared memory) and O_j += P_j V (A = P_j from TMEM, B = V). Per key
@@ -48,7 +48,7 @@ namespace {
 
 constexpr int kD = 128;           // head dim handled by this kernel
 constexpr int kTile = 128;        // keys per tile
-constexpr int kKStages = 3;       // K ring depth
+constexpr int kKStages = 2;       // K ring depth
 constexpr int kVStages = 2;       // V ring depth
 constexpr bool kSplitProducers = true;   // V loads from their own thread (warp 2), K and Q from warp 0
 constexpr int kRows = 128;        // query rows per query tile (one M=128 MMA)
@@ -73,7 +73,6 @@ constexpr uint32_t kSmemV = kSmemK + kKStages * kKBytesPerStage;
 constexpr uint32_t kSmemBar = kSmemV + kVStages * kKBytesPerStage;
 constexpr uint32_t kSmemBytes = kSmemBar + 1024 + 1024;        // barriers + alignment slack
 
-constexpr int kMergeRows = 8;     // rows per merge CTA (one per warp)
 
 // Instruction descriptors (kind::f16): D fp32, A/B bf16, A K-major.
 constexpr uint32_t make_idesc(int M, int N, bool b_mn_major) {
@@ -234,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
     for (int j = 0; j < kStreams; ++j) {
       mbar_init(&sm.s_full[j], 1);
-      mbar_init(&sm.p_full[j], kRows);
+      mbar_init(&sm.p_full[j], kRows / 32);   // one arrival per softmax warp
       mbar_init(&sm.o_full[j], 1);
     }
     mbar_init(&sm.drain, 1);
@@ -741,8 +740,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           }
           m_used = m_new;
+          // every lane's TMEM stores (and O rescale) are complete and fenced before the warp's one
+          // arrival hands P to the MMA thread
           tc_fence_before();
-          mbar_arrive(&sm.p_full[j]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full[j]);
         }
         if (!ok) break;
         // ---- epilogue of the segment: wait for the last PV product, then O / l for the row
@@ -817,10 +819,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
-// Merges the partials of groups cut between teams (flash-decoding combine). One warp per query
-// row, 8 rows per CTA; lane j reads contributor j's log2-sum-exp, and every lane reads 4 of the
-// 128 dims of every contributor's row (coalesced 512-byte rows), 8 contributors in flight:
+// Merges the partials of groups cut between teams (flash-decoding combine):
 //   O = sum_j 2^(lse_j - M) O_j / sum_j 2^(lse_j - M),  M = max_j lse_j.
+// A CTA takes 32 query rows of one (group, query tile), 8 threads per row, each thread 16 of the
+// 128 dims: it reads its row's log2-sum-exps (the 8 threads of a row read the same words) and its
+// 64-byte slice of every contributor's row, issued together, 4 contributors at a time. CTAs of a
+// group that one team held whole return after reading the group's contributor range.
+constexpr int kMergeRowsPerCta = 32;
+constexpr int kMergeThreads = 256;   // 8 threads per row
+
 struct MergeParams {
   int32_t S, Hq, Hkv, G, nq, s_per_tile, groups;
   __nv_bfloat16* out;
@@ -830,13 +837,13 @@ struct MergeParams {
   const int32_t* skip_if;
 };
 
-__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergeParams p) {
   pdl_wait();
   if (skip_requested(p.skip_if)) return;
   const int u = blockIdx.x;             // group
   const int qt = blockIdx.z;            // query tile
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.y * kMergeRows + warp;
+  const int row = blockIdx.y * kMergeRowsPerCta + (threadIdx.x >> 3);
+  const int part = threadIdx.x & 7;     // dims [16 part, 16 part + 16)
   const AttnMeta* meta = reinterpret_cast<const AttnMeta*>(p.ws + p.off_meta);
   // the two reads are independent: issued together, one round trip
   const long long T = meta->total_tiles;
@@ -852,43 +859,55 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   const int n = (int)(c_hi - c_lo + 1);
   auto slot_of = [&](int j) { return ((size_t)u + (size_t)(c_lo + j)) * (size_t)p.nq + (size_t)qt; };
   float mx = -INFINITY;
-  for (int j = lane; j < n; j += 32) mx = fmaxf(mx, plse[slot_of(j) * kRows + row]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < n; ++j) mx = fmaxf(mx, __ldg(plse + slot_of(j) * kRows + row));
+  float4 acc[4] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f),
+                   make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
   float wsum = 0.f;
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const int cnt = min(32, n - j0);
-    const float wl = (lane < cnt) ? ex2(plse[slot_of(j0 + lane) * kRows + row] - mx) : 0.f;
-    float part = wl;
+  for (int j0 = 0; j0 < n; j0 += 4) {
+    float4 v[4][4];
+    float wl[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    wsum += part;
-    for (int jj = 0; jj < cnt; jj += 8) {
-      float4 v[8];
+    for (int q = 0; q < 4; ++q) {
+      wl[q] = 0.f;
+      if (j0 + q < n) {
+        const size_t sl = slot_of(j0 + q);
+        wl[q] = __ldg(plse + sl * kRows + row);
+        const float4* src = reinterpret_cast<const float4*>(partials + (sl * kRows + row) * kD) + 4 * part;
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        v[q] = (jj + q < cnt) ? reinterpret_cast<const float4*>(partials + (slot_of(j0 + jj + q) * kRows + row) * kD)[lane]
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < 4; ++c) v[q][c] = __ldg(src + c);
+      }
+    }
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float wq = __shfl_sync(0xffffffffu, wl, (jj + q) & 31);
-        acc.x = fmaf(wq, v[q].x, acc.x);
-        acc.y = fmaf(wq, v[q].y, acc.y);
-        acc.z = fmaf(wq, v[q].z, acc.z);
-        acc.w = fmaf(wq, v[q].w, acc.w);
+    for (int q = 0; q < 4; ++q) {
+      if (j0 + q < n) {
+        const float wq = ex2(wl[q] - mx);
+        wsum += wq;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[c].x = fmaf(wq, v[q][c].x, acc[c].x);
+          acc[c].y = fmaf(wq, v[q][c].y, acc[c].y);
+          acc[c].z = fmaf(wq, v[q][c].z, acc[c].z);
+          acc[c].w = fmaf(wq, v[q][c].w, acc[c].w);
+        }
       }
     }
   }
   const float inv = 1.0f / wsum;
   const int s_idx = qt * p.s_per_tile + row / p.G;
   const int hq = kvh * p.G + row % p.G;
-  __nv_bfloat16* orow = p.out + (((size_t)b * p.S + s_idx) * p.Hq + hq) * kD;
-  uint2 o;
-  o.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-  o.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-  reinterpret_cast<uint2*>(orow)[lane] = o;
-  if (p.lse && lane == 0) p.lse[((size_t)b * p.Hq + hq) * p.S + s_idx] = (mx + log2f(wsum)) * 0.69314718055994531f;
+  __nv_bfloat16* orow = p.out + (((size_t)b * p.S + s_idx) * p.Hq + hq) * kD + 16 * part;
+  uint4 o0, o1;
+  o0.x = pack_bf16x2(acc[0].x * inv, acc[0].y * inv);
+  o0.y = pack_bf16x2(acc[0].z * inv, acc[0].w * inv);
+  o0.z = pack_bf16x2(acc[1].x * inv, acc[1].y * inv);
+  o0.w = pack_bf16x2(acc[1].z * inv, acc[1].w * inv);
+  o1.x = pack_bf16x2(acc[2].x * inv, acc[2].y * inv);
+  o1.y = pack_bf16x2(acc[2].z * inv, acc[2].w * inv);
+  o1.z = pack_bf16x2(acc[3].x * inv, acc[3].y * inv);
+  o1.w = pack_bf16x2(acc[3].z * inv, acc[3].w * inv);
+  reinterpret_cast<uint4*>(orow)[0] = o0;
+  reinterpret_cast<uint4*>(orow)[1] = o1;
+  if (p.lse && part == 0) p.lse[((size_t)b * p.Hq + hq) * p.S + s_idx] = (mx + log2f(wsum)) * 0.69314718055994531f;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -1034,8 +1053,8 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   mp.off_lse = pl.off_lse;
   mp.skip_if = a->skip_if;
   const int M = G * pl.s_per_tile;
-  const dim3 mgrid(pl.units, (M + kMergeRows - 1) / kMergeRows, pl.qtiles);
-  if (launch_pdl(attn_merge_kernel, mgrid, dim3(256), 0, stream, mp) != cudaSuccess) return TT_ERR_CUDA;
+  const dim3 mgrid(pl.units, (M + kMergeRowsPerCta - 1) / kMergeRowsPerCta, pl.qtiles);
+  if (launch_pdl(attn_merge_kernel, mgrid, dim3(kMergeThreads), 0, stream, mp) != cudaSuccess) return TT_ERR_CUDA;
   return TT_OK;
 }
 

@@ -51,6 +51,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Bounded waits give up after this many nanoseconds (about one second).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// The waits on a kernel's hot path count SM cycles instead (the clock64 counter is a cheap
+// register read; the global timer is not): 2^31 cycles is at least one second at the B200's
+// highest SM clock (1965 MHz), longer at lower clocks.
+constexpr long long kWaitLimitCycles = 1ll << 31;
+
+__device__ __forceinline__ long long sm_clock() {
+  long long c;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+  return c;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -89,6 +99,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete. Gives up (returns false) after
 // limit_ns nanoseconds or as soon as *abort_flag becomes non-zero.
 __device__ __forceinline__ bool mbar_wait_bounded_for(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -102,9 +125,16 @@ __device__ __forceinline__ bool mbar_wait_bounded_for(uint64_t* bar, uint32_t pa
   }
 }
 
-// The kernels' bounded wait: gives up after kWaitLimitNs.
+// The kernels' bounded wait: gives up after kWaitLimitCycles SM cycles (at least one second) or
+// as soon as *abort_flag becomes non-zero.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return mbar_wait_bounded_for(bar, parity, abort_flag, kWaitLimitNs);
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long c0 = sm_clock();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (sm_clock() - c0 > kWaitLimitCycles) return false;
+  }
 }
 
 // ------------------------------------------------------------------ TMA (no multicast)

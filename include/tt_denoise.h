@@ -90,7 +90,8 @@ int tt_version(void);
  *   out     [B][S][Hq][d]   E, rounded to nearest from the fp32 result
  *   lse     [B][Hq][S] float or NULL: natural-log log-sum-exp of the scaled scores per row
  * Supported: TT_BF16 with d = 128 (tensor-core path, S*Hq/Hkv rows per tile, S <= 64,
- * page_size a multiple of 128); TT_F32 with d in {64, 128}. Others: TT_ERR_UNSUPPORTED.
+ * page_size a multiple of 128); TT_F32 with d in {64, 128} (tensor cores, tf32 with the split
+ * operands). Others: TT_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------------------------- */
 typedef struct {
   int32_t batch;             /* B >= 1 */
