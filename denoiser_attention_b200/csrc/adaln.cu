@@ -5,8 +5,8 @@
 //
 //   COND             tau -> mod[B][3][D]   three launches, one per layer (F->W with the sinusoid,
 //                                          W->W, W->3D), each tiled over 32-row slices of the
-//                                          weight x 16-sequence chunks, operands staged in shared
-//                                          memory with asynchronous copies
+//                                          weight x chunks of 64, 16 or 8 sequences, operands
+//                                          staged in shared memory with asynchronous copies
 //   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one CTA per token row
 //   GATED_RESIDUAL   h + gate * f: a vectorised elementwise pass
 // All arithmetic is fp32 (the timestep sinusoid in fp64); bf16 tensors are widened on load and
@@ -29,21 +29,23 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// phi(tau) = [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)). The angle (up to
-// 1000 rad) is formed and reduced modulo 2 pi in double, so the single-precision sincos only sees
-// |angle| <= pi.
-__device__ __forceinline__ void phi_row(float tau, int F, float* dst, int tid, int nthreads) {
+// phi(tau) = [cos(1000 tau w_k), sin(1000 tau w_k)], w_k = 10000^(-k/(F/2)), for nb sequences
+// (row bb of dst from tau[bb]). A thread computes its frequencies once and forms each sequence's
+// angle (up to 1000 rad) and its reduction modulo 2 pi in double, so the single-precision sincos
+// only sees |angle| <= pi.
+__device__ __forceinline__ void phi_rows(const float* tau, int nb, int F, float* dst, int tid, int nthreads) {
   const int half = F / 2;
-  const double t = 1000.0 * (double)tau;
   const double two_pi = 6.283185307179586476925286766559;
   for (int k = tid; k < half; k += nthreads) {
-    const double w = exp(-9.2103403719761836 * (double)k / (double)half);   // ln(10000) = 9.2103...
-    double a = t * w;
-    a -= two_pi * rint(a * (1.0 / two_pi));
-    float sv, cv;
-    sincosf((float)a, &sv, &cv);
-    dst[k] = cv;
-    dst[half + k] = sv;
+    const double w = 1000.0 * exp(-9.2103403719761836 * (double)k / (double)half);   // ln(10000) = 9.2103...
+    for (int bb = 0; bb < nb; ++bb) {
+      double a = (double)tau[bb] * w;
+      a -= two_pi * rint(a * (1.0 / two_pi));
+      float sv, cv;
+      sincosf((float)a, &sv, &cv);
+      dst[bb * F + k] = cv;
+      dst[bb * F + half + k] = sv;
+    }
   }
 }
 
@@ -60,78 +62,106 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 // One layer of the conditioning MLP for a slice of its outputs and a chunk of the sequences:
-//   y[b][o] = act(W[o, :] . x_b + bias[o]) (+ extra[o]),  o in [32 i, 32 i + 32), b in [16 j, 16 j + 16)
+//   y[b][o] = act(W[o, :] . x_b + bias[o]) (+ extra[o]),  o in [32 i, 32 i + 32), b in chunk j
 // x_b is phi(tau_b) (kPhi: the timestep sinusoid, computed here) or row b of x. The CTA stages its
 // 32 rows of W (rows padded by 4 floats, so that the quarter-warp float4 reads of 8 rows hit
-// distinct banks) and its 16 input rows in shared memory with asynchronous copies; then lane =
-// output row and warp = a pair of sequences, whose input rows are read as broadcasts.
+// distinct banks) and its chunk's input rows in shared memory with asynchronous copies; then
+// lane = output row and warp = kSeqPerWarp sequences, whose input rows are read as broadcasts.
+// Chunks of 64 sequences (8 per warp) serve inputs up to 256 wide; wider inputs take chunks of 16.
 constexpr int kRowSlice = 32;
-constexpr int kSeqChunk = 16;
 
-inline size_t rows_smem_bytes(int IN) {
-  return sizeof(float) * ((size_t)kRowSlice * (IN + 4) + (size_t)kSeqChunk * IN);
+inline size_t rows_smem_bytes(int IN, int chunk) {
+  return sizeof(float) * ((size_t)kRowSlice * (IN + 4) + (size_t)chunk * IN);
 }
 
-template <bool kPhi, bool kSilu>
+template <bool kPhi, bool kSilu, int kSeqPerWarp>
 __global__ void __launch_bounds__(kAdalnThreads) adaln_rows_kernel(const float* __restrict__ Wt,
                                                                    const float* __restrict__ bias,
                                                                    const float* __restrict__ extra,
                                                                    const float* __restrict__ x, int B, int IN,
                                                                    int OUT, float* __restrict__ y,
                                                                    const int32_t* skip_if) {
+  constexpr int kChunk = kSeqPerWarp * (kAdalnThreads / 32);
   extern __shared__ __align__(16) float s_dyn[];
   const int INP = IN + 4;
   float* s_w = s_dyn;                          // [32][IN + 4]
-  float* s_x = s_dyn + kRowSlice * INP;        // [16][IN]
+  float* s_x = s_dyn + kRowSlice * INP;        // [kChunk][IN]
   pdl_trigger();
   pdl_wait();
   if (skip_requested(skip_if)) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int o0 = blockIdx.x * kRowSlice, b0 = blockIdx.y * kSeqChunk;
-  const int nrow = min(kRowSlice, OUT - o0), nb = min(kSeqChunk, B - b0);
+  const int o0 = blockIdx.x * kRowSlice, b0 = blockIdx.y * kChunk;
+  const int nrow = min(kRowSlice, OUT - o0), nb = min(kChunk, B - b0);
   const int iv = IN / 4;
   for (int i = threadIdx.x; i < nrow * iv; i += blockDim.x) {
     const int r = i / iv, c = i - r * iv;
     cp_async16_g2s(s_w + r * INP + 4 * c, Wt + (size_t)(o0 + r) * IN + 4 * c);
   }
   if (kPhi) {
-    for (int bb = 0; bb < nb; ++bb) phi_row(x[b0 + bb], IN, s_x + bb * IN, threadIdx.x, blockDim.x);
+    phi_rows(x + b0, nb, IN, s_x, threadIdx.x, blockDim.x);
   } else {
     for (int i = threadIdx.x; i < nb * iv; i += blockDim.x)
       cp_async16_g2s(s_x + 4 * i, x + (size_t)b0 * IN + 4 * i);
   }
   cp_async_wait_all();
   __syncthreads();
-  const int bA = 2 * warp, bB = 2 * warp + 1;   // this warp's two sequences of the chunk
-  if (lane >= nrow || bA >= nb) return;
-  float accA = 0.f, accB = 0.f;
+  const int bw = kSeqPerWarp * warp;   // this warp's first sequence of the chunk
+  if (lane >= nrow || bw >= nb) return;
+  float acc[kSeqPerWarp];
+#pragma unroll
+  for (int q = 0; q < kSeqPerWarp; ++q) acc[q] = 0.f;
   const float* wrow = s_w + lane * INP;
-  const float* xa = s_x + bA * IN;
-  const float* xb = s_x + (bB < nb ? bB : bA) * IN;
   for (int k = 0; k < IN; k += 4) {
-    const float4 w = *reinterpret_cast<const float4*>(wrow + k);
-    const float4 u = *reinterpret_cast<const float4*>(xa + k);
-    const float4 v = *reinterpret_cast<const float4*>(xb + k);
-    accA = fmaf(w.x, u.x, fmaf(w.y, u.y, fmaf(w.z, u.z, fmaf(w.w, u.w, accA))));
-    accB = fmaf(w.x, v.x, fmaf(w.y, v.y, fmaf(w.z, v.z, fmaf(w.w, v.w, accB))));
+    const float4 wv = *reinterpret_cast<const float4*>(wrow + k);
+#pragma unroll
+    for (int q = 0; q < kSeqPerWarp; ++q) {
+      const int bq = bw + q < nb ? bw + q : bw;   // past the chunk's end: a valid row, result unused
+      const float4 u = *reinterpret_cast<const float4*>(s_x + bq * IN + k);
+      acc[q] = fmaf(wv.x, u.x, fmaf(wv.y, u.y, fmaf(wv.z, u.z, fmaf(wv.w, u.w, acc[q]))));
+    }
   }
   const int o = o0 + lane;
   const float add = bias[o] + (extra ? extra[o] : 0.f);
-  float ya = accA + add, yb = accB + add;
-  if (kSilu) {
-    ya = silu_f(ya);
-    yb = silu_f(yb);
+#pragma unroll
+  for (int q = 0; q < kSeqPerWarp; ++q) {
+    if (bw + q < nb) {
+      float v = acc[q] + add;
+      if (kSilu) v = silu_f(v);
+      y[(size_t)(b0 + bw + q) * OUT + o] = v;
+    }
   }
-  y[(size_t)(b0 + bA) * OUT + o] = ya;
-  if (bB < nb) y[(size_t)(b0 + bB) * OUT + o] = yb;
+}
+
+// Chunk choice: the widest chunk (64, 16 or 8 sequences) that still gives at least one CTA per
+// SM, so that narrow layers (few 32-row slices) spread over more CTAs; 64-sequence chunks only
+// while the staged rows fit in kWideChunkSmem (inputs up to 256 wide).
+constexpr size_t kWideChunkSmem = 100 * 1024;
+constexpr int kFillCtas = 148;
+
+template <bool kPhi, bool kSilu, int kSeqPerWarp>
+static cudaError_t launch_rows_spw(const float* Wt, const float* bias, const float* extra, const float* x, int B,
+                                   int IN, int OUT, float* y, const int32_t* skip_if, cudaStream_t stream) {
+  constexpr int kChunk = kSeqPerWarp * (kAdalnThreads / 32);
+  const dim3 grid((OUT + kRowSlice - 1) / kRowSlice, (B + kChunk - 1) / kChunk);
+  return launch_pdl(adaln_rows_kernel<kPhi, kSilu, kSeqPerWarp>, grid, dim3(kAdalnThreads),
+                    rows_smem_bytes(IN, kChunk), stream, Wt, bias, extra, x, B, IN, OUT, y, skip_if);
 }
 
 template <bool kPhi, bool kSilu>
 static cudaError_t launch_rows(const float* Wt, const float* bias, const float* extra, const float* x, int B, int IN,
                                int OUT, float* y, const int32_t* skip_if, cudaStream_t stream) {
-  const dim3 grid((OUT + kRowSlice - 1) / kRowSlice, (B + kSeqChunk - 1) / kSeqChunk);
-  return launch_pdl(adaln_rows_kernel<kPhi, kSilu>, grid, dim3(kAdalnThreads), rows_smem_bytes(IN), stream, Wt, bias,
-                    extra, x, B, IN, OUT, y, skip_if);
+  const long long rows = (OUT + kRowSlice - 1) / kRowSlice;
+  if (rows_smem_bytes(IN, 64) <= kWideChunkSmem && rows * ((B + 63) / 64) >= kFillCtas)
+    return launch_rows_spw<kPhi, kSilu, 8>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
+  if (rows * ((B + 15) / 16) >= kFillCtas)
+    return launch_rows_spw<kPhi, kSilu, 2>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
+  return launch_rows_spw<kPhi, kSilu, 1>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
+}
+
+template <bool kPhi, bool kSilu, int kSeqPerWarp>
+static bool set_rows_smem(int bytes) {
+  return cudaFuncSetAttribute(adaln_rows_kernel<kPhi, kSilu, kSeqPerWarp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              bytes) == cudaSuccess;
 }
 
 template <typename T>
@@ -258,19 +288,21 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
     if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
-      const int max_smem = (int)rows_smem_bytes(kMaxWidth);
-      if (cudaFuncSetAttribute(adaln_rows_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
-              cudaSuccess ||
-          cudaFuncSetAttribute(adaln_rows_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
-              cudaSuccess ||
-          cudaFuncSetAttribute(adaln_rows_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               max_smem) != cudaSuccess)
+      const int s8 = (int)kWideChunkSmem, s2 = (int)rows_smem_bytes(kMaxWidth, 16),
+                s1 = (int)rows_smem_bytes(kMaxWidth, 8);
+      if (!set_rows_smem<true, true, 8>(s8) || !set_rows_smem<false, true, 8>(s8) ||
+          !set_rows_smem<false, false, 8>(s8) || !set_rows_smem<true, true, 2>(s2) ||
+          !set_rows_smem<false, true, 2>(s2) || !set_rows_smem<false, false, 2>(s2) ||
+          !set_rows_smem<true, true, 1>(s1) || !set_rows_smem<false, true, 1>(s1) ||
+          !set_rows_smem<false, false, 1>(s1))
         return TT_ERR_CUDA;
       __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
     }
-    launch_rows<true, true>(a->w1, a->b1, nullptr, a->tau, B, F, W, a1, a->skip_if, stream);
-    launch_rows<false, true>(a->w2, a->b2, nullptr, a1, B, W, W, a2, a->skip_if, stream);
-    launch_rows<false, false>(a->w3, a->b3, a->layer_emb, a2, B, W, OUT, a->mod, a->skip_if, stream);
+    if (launch_rows<true, true>(a->w1, a->b1, nullptr, a->tau, B, F, W, a1, a->skip_if, stream) != cudaSuccess ||
+        launch_rows<false, true>(a->w2, a->b2, nullptr, a1, B, W, W, a2, a->skip_if, stream) != cudaSuccess ||
+        launch_rows<false, false>(a->w3, a->b3, a->layer_emb, a2, B, W, OUT, a->mod, a->skip_if, stream) !=
+            cudaSuccess)
+      return TT_ERR_CUDA;
   } else if (a->op == TT_ADALN_NORM_MODULATE) {
     const int rows = B * a->block_size;
     if (a->dtype == TT_BF16)
