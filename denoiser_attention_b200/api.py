@@ -227,9 +227,9 @@ class RefinementStep:
 
     SCHEDULES = ("branches", "attn_then_unmask", "unmask_then_attn", "serial")
 
-    # kernel launches per step: adaLN COND (2: hidden layers, output layer), RMSNorm prologue,
-    # attention + split-KV merge, gated residual, unmask
-    LAUNCHES = 7
+    # kernel launches per step: adaLN COND (3, one per MLP layer), RMSNorm prologue, attention and
+    # its split-KV merge, gated residual, unmask
+    LAUNCHES = 8
 
     def __init__(self, weights: Dict[str, torch.Tensor], *, gamma: float, inv_temperature: float = 1.0,
                  mask_token_id: int = 3, page_size: int = 0, ctx_stride: int = 0, softmax_scale: float = 1.0,
