@@ -432,6 +432,23 @@ def run_ours(args):
     return result
 
 
+def lmhead_inputs(dev, B: int = 8, S: int = 16, D: int = 2048, V: int = 131072, seed: int = 5):
+    """Hidden states x [B][S][D] ~ N(0, 1) and an LM-head weight W [V][D] ~ N(0, 3^2 / D) (bf16,
+    seeded), every position masked: the decode shape of the fused LM head + unmask."""
+    import torch
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((B, S, D), generator=g).to(torch.bfloat16).to(dev)
+    w = (torch.randn((V, D), generator=g) * (3.0 / D ** 0.5)).to(torch.bfloat16).to(dev)
+    tokens = torch.full((B, S), 3, dtype=torch.int32, device=dev)
+    masked = torch.ones((B, S), dtype=torch.uint8, device=dev)
+    return x, w, tokens, masked
+
+
+def lmhead_op(gamma: float = 0.8):
+    from denoiser_attention_b200 import api
+    return lambda b, o: api.lmhead_unmask_step(b[0], b[1], b[2], b[3], gamma=gamma, want_conf=False)
+
+
 def run_set_mb(inp, ad, logits) -> float:
     return sum(t.numel() * t.element_size() for t in (inp.k_ctx, inp.v_ctx, logits, inp.q, ad.h, ad.f)) / 1e6
 
@@ -525,6 +542,19 @@ def run_extras(args, dev, peak):
     out["sweep_unmask"] = {"unmask_us_by_S": times, "cells": table,
                            "note": "committed tokens per step: mean over the 32 sequences of the first step "
                                    "(every position masked), confidence sampler"}
+    # ---- the fused LM head + unmask on the decode shape (128 rows, D 2048, vocabulary 131072):
+    # the 537 MB weight stream is the algorithmic traffic (larger than L2 by itself)
+    lm = lmhead_inputs(dev)
+    lmhead_op()(lm, None)
+    torch.cuda.synchronize()
+    ms = isolated_ms(lmhead_op(), [lm], [None], torch.cuda.Stream(device=dev), reps=50)
+    wbytes = lm[1].numel() * 2
+    flops = 2 * lm[0].shape[0] * lm[0].shape[1] * lm[0].shape[2] * lm[1].shape[0]
+    out["lmhead_unmask"] = {"shape": "x 8x16x2048, W 131072x2048 bf16", "us": ms * 1e3,
+                            "weight_gbs": wbytes / (ms * 1e-3) / 1e9, "frac": wbytes / (ms * 1e-3) / 1e9 / peak,
+                            "tflops": flops / (ms * 1e-3) / 1e12}
+    del lm
+    torch.cuda.empty_cache()
     return out
 
 
@@ -590,6 +620,55 @@ def cpu_baseline(w, inp, ad, logits):
             "sample": f"{k} query tokens of the workload (all heads, adaLN, unmask of that position), {el:.1f} s"}
 
 
+def run_kernel(args):
+    """One kernel alone on one workload, eager launches: --warmup untimed, then --steps timed with
+    CUDA events; one JSON line with its mean time (for profiling captures that should hold only
+    that kernel's buffers)."""
+    import torch
+    from denoiser_attention_b200 import api, build, synth
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    build.build()
+    if args.kernel == "lmhead":
+        bufs, out, op, nbytes = lmhead_inputs(dev), None, lmhead_op(), 131072 * 2048 * 2
+        desc = "x 8x16x2048, W 131072x2048 bf16"
+    else:
+        w = synth.workload(args.workload)
+        if args.kernel == "attn":
+            a = synth.attention_inputs(w.attn, seed=w.seed)
+            bufs = api.StepBuffers(tau=None, h=None, f=None, q=a.q.to(dev), k_blk=a.k_blk.to(dev),
+                                   v_blk=a.v_blk.to(dev), k_ctx=a.k_ctx.to(dev), v_ctx=a.v_ctx.to(dev),
+                                   ctx_lens=a.ctx_lens.to(dev),
+                                   page_table=None if a.page_table is None else a.page_table.to(dev), logits=None,
+                                   tokens=None, is_masked=None)
+            out = torch.empty_like(bufs.q)
+            op = attn_op(api.RefinementStep({}, gamma=w.gamma, page_size=w.attn.page_size, ctx_stride=a.ctx_stride))
+            nbytes = kv_bytes_of(w.attn)
+        else:
+            B, S = w.attn.batch, w.attn.block_size
+            bufs = api.StepBuffers(tau=None, h=None, f=None, q=None, k_blk=None, v_blk=None, k_ctx=None, v_ctx=None,
+                                   ctx_lens=None, page_table=None, logits=synth.workload_logits(w).to(dev),
+                                   tokens=torch.full((B, S), 3, dtype=torch.int32, device=dev),
+                                   is_masked=torch.ones((B, S), dtype=torch.uint8, device=dev))
+            out = None
+            op = unmask_op(api.RefinementStep({}, gamma=w.gamma, inv_temperature=w.inv_temperature))
+            nbytes = bufs.logits.numel() * bufs.logits.element_size()
+        desc = workload_desc(w)
+    for _ in range(args.warmup):
+        op(bufs, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        op(bufs, out)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    print(json.dumps({"kernel": args.kernel, "workload": desc, "us_per_launch": us, "launches": args.steps,
+                      "algorithmic_bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
+                      "note": "eager launches on one buffer set (warm L2 when the data fits it); for profiling"}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -600,13 +679,17 @@ def main():
                     help="the step's workload (default: the batch-generation workload, the headline)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the extra keys (decode step, attention per workload, block-sweep unmask table)")
-    ap.add_argument("--schedule", choices=list(SCHEDULE_TEXT), default="branches",
+    ap.add_argument("--schedule", choices=list(SCHEDULE_TEXT), default="serial",
                     help="how the step's three branches are put on streams")
+    ap.add_argument("--kernel", choices=["attn", "unmask", "lmhead"], default=None,
+                    help="time one kernel alone on --workload (for profiling captures), not the step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.kernel is not None:
+        run_kernel(args)
     else:
         run_ours(args)
 
