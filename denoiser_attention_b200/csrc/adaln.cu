@@ -4,8 +4,8 @@
 // per-layer embedding).
 //
 //   COND             tau -> mod[B][3][D]   three launches, one per layer (F->W with the sinusoid,
-//                                          W->W, W->3D), each tiled over 32-row slices of the
-//                                          weight x chunks of 64, 16 or 8 sequences, operands
+//                                          W->W, W->3D), each tiled over slices of 64 or 32
+//                                          weight rows x chunks of 32, 16 or 8 sequences, operands
 //                                          staged in shared memory with asynchronous copies
 //   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one CTA per token row
 //   GATED_RESIDUAL   h + gate * f: a vectorised elementwise pass
@@ -62,36 +62,38 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 // One layer of the conditioning MLP for a slice of its outputs and a chunk of the sequences:
-//   y[b][o] = act(W[o, :] . x_b + bias[o]) (+ extra[o]),  o in [32 i, 32 i + 32), b in chunk j
+//   y[b][o] = act(W[o, :] . x_b + bias[o]) (+ extra[o]),  o in slice i, b in chunk j
 // x_b is phi(tau_b) (kPhi: the timestep sinusoid, computed here) or row b of x. The CTA stages its
-// 32 rows of W (rows padded by 4 floats, so that the quarter-warp float4 reads of 8 rows hit
-// distinct banks) and its chunk's input rows in shared memory with asynchronous copies; then
-// lane = output row and warp = kSeqPerWarp sequences, whose input rows are read as broadcasts.
-// Chunks of 64 sequences (8 per warp) serve inputs up to 256 wide; wider inputs take chunks of 16.
-constexpr int kRowSlice = 32;
+// 32 kRows rows of W (rows padded by 4 floats, so that the quarter-warp float4 reads of 8 rows hit
+// distinct banks) and its chunk's input rows in shared memory with asynchronous copies; then a
+// thread takes kRows output rows (lane, lane + 32, ...) for the kSeqPerWarp sequences of its warp,
+// whose input rows are read as broadcasts: each float4 of W feeds kSeqPerWarp products and each
+// float4 of x feeds kRows, which sets the ratio of arithmetic to shared-memory reads.
+template <int kRows, int kSeqPerWarp>
+struct RowsTile {
+  static constexpr int kSlice = 32 * kRows;                           // output rows per CTA
+  static constexpr int kChunk = kSeqPerWarp * (kAdalnThreads / 32);   // sequences per CTA
+  static size_t smem_bytes(int IN) { return sizeof(float) * ((size_t)kSlice * (IN + 4) + (size_t)kChunk * IN); }
+};
 
-inline size_t rows_smem_bytes(int IN, int chunk) {
-  return sizeof(float) * ((size_t)kRowSlice * (IN + 4) + (size_t)chunk * IN);
-}
-
-template <bool kPhi, bool kSilu, int kSeqPerWarp>
+template <bool kPhi, bool kSilu, int kRows, int kSeqPerWarp>
 __global__ void __launch_bounds__(kAdalnThreads) adaln_rows_kernel(const float* __restrict__ Wt,
                                                                    const float* __restrict__ bias,
                                                                    const float* __restrict__ extra,
                                                                    const float* __restrict__ x, int B, int IN,
                                                                    int OUT, float* __restrict__ y,
                                                                    const int32_t* skip_if) {
-  constexpr int kChunk = kSeqPerWarp * (kAdalnThreads / 32);
+  using Tile = RowsTile<kRows, kSeqPerWarp>;
   extern __shared__ __align__(16) float s_dyn[];
   const int INP = IN + 4;
-  float* s_w = s_dyn;                          // [32][IN + 4]
-  float* s_x = s_dyn + kRowSlice * INP;        // [kChunk][IN]
+  float* s_w = s_dyn;                          // [kSlice][IN + 4]
+  float* s_x = s_dyn + Tile::kSlice * INP;     // [kChunk][IN]
   pdl_trigger();
   pdl_wait();
   if (skip_requested(skip_if)) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int o0 = blockIdx.x * kRowSlice, b0 = blockIdx.y * kChunk;
-  const int nrow = min(kRowSlice, OUT - o0), nb = min(kChunk, B - b0);
+  const int o0 = blockIdx.x * Tile::kSlice, b0 = blockIdx.y * Tile::kChunk;
+  const int nrow = min(Tile::kSlice, OUT - o0), nb = min(Tile::kChunk, B - b0);
   const int iv = IN / 4;
   for (int i = threadIdx.x; i < nrow * iv; i += blockDim.x) {
     const int r = i / iv, c = i - r * iv;
@@ -107,61 +109,82 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_rows_kernel(const float* 
   __syncthreads();
   const int bw = kSeqPerWarp * warp;   // this warp's first sequence of the chunk
   if (lane >= nrow || bw >= nb) return;
-  float acc[kSeqPerWarp];
+  float acc[kRows][kSeqPerWarp];
 #pragma unroll
-  for (int q = 0; q < kSeqPerWarp; ++q) acc[q] = 0.f;
-  const float* wrow = s_w + lane * INP;
+  for (int r = 0; r < kRows; ++r)
+#pragma unroll
+    for (int q = 0; q < kSeqPerWarp; ++q) acc[r][q] = 0.f;
+  // rows past the slice's end read a valid staged row (row 0); their results are not stored
+  const float* wrow[kRows];
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) wrow[r] = s_w + (lane + 32 * r < nrow ? lane + 32 * r : 0) * INP;
+  const float* xrow[kSeqPerWarp];
+#pragma unroll
+  for (int q = 0; q < kSeqPerWarp; ++q) xrow[q] = s_x + (bw + q < nb ? bw + q : bw) * IN;
   for (int k = 0; k < IN; k += 4) {
-    const float4 wv = *reinterpret_cast<const float4*>(wrow + k);
+    float4 wv[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) wv[r] = *reinterpret_cast<const float4*>(wrow[r] + k);
 #pragma unroll
     for (int q = 0; q < kSeqPerWarp; ++q) {
-      const int bq = bw + q < nb ? bw + q : bw;   // past the chunk's end: a valid row, result unused
-      const float4 u = *reinterpret_cast<const float4*>(s_x + bq * IN + k);
-      acc[q] = fmaf(wv.x, u.x, fmaf(wv.y, u.y, fmaf(wv.z, u.z, fmaf(wv.w, u.w, acc[q]))));
+      const float4 u = *reinterpret_cast<const float4*>(xrow[q] + k);
+#pragma unroll
+      for (int r = 0; r < kRows; ++r)
+        acc[r][q] = fmaf(wv[r].x, u.x, fmaf(wv[r].y, u.y, fmaf(wv[r].z, u.z, fmaf(wv[r].w, u.w, acc[r][q]))));
     }
   }
-  const int o = o0 + lane;
-  const float add = bias[o] + (extra ? extra[o] : 0.f);
 #pragma unroll
-  for (int q = 0; q < kSeqPerWarp; ++q) {
-    if (bw + q < nb) {
-      float v = acc[q] + add;
-      if (kSilu) v = silu_f(v);
-      y[(size_t)(b0 + bw + q) * OUT + o] = v;
+  for (int r = 0; r < kRows; ++r) {
+    if (lane + 32 * r >= nrow) break;
+    const int o = o0 + lane + 32 * r;
+    const float add = bias[o] + (extra ? extra[o] : 0.f);
+#pragma unroll
+    for (int q = 0; q < kSeqPerWarp; ++q) {
+      if (bw + q < nb) {
+        float v = acc[r][q] + add;
+        if (kSilu) v = silu_f(v);
+        y[(size_t)(b0 + bw + q) * OUT + o] = v;
+      }
     }
   }
 }
 
-// Chunk choice: the widest chunk (64, 16 or 8 sequences) that still gives at least one CTA per
-// SM, so that narrow layers (few 32-row slices) spread over more CTAs; 64-sequence chunks only
-// while the staged rows fit in kWideChunkSmem (inputs up to 256 wide).
-constexpr size_t kWideChunkSmem = 100 * 1024;
+// Tile choice: 64 rows x 32 sequences (2 rows and 4 sequences per thread) when the staged rows fit
+// in kWideTileSmem (inputs up to 256 wide) and the grid still has at least one CTA per SM (the
+// 6144-row output layer); else 32 rows x 16 or 8 sequences, the wider while it fills the SMs, so
+// that narrow layers (few row slices) spread over more CTAs.
+constexpr size_t kWideTileSmem = 100 * 1024;
 constexpr int kFillCtas = 148;
 
-template <bool kPhi, bool kSilu, int kSeqPerWarp>
-static cudaError_t launch_rows_spw(const float* Wt, const float* bias, const float* extra, const float* x, int B,
-                                   int IN, int OUT, float* y, const int32_t* skip_if, cudaStream_t stream) {
-  constexpr int kChunk = kSeqPerWarp * (kAdalnThreads / 32);
-  const dim3 grid((OUT + kRowSlice - 1) / kRowSlice, (B + kChunk - 1) / kChunk);
-  return launch_pdl(adaln_rows_kernel<kPhi, kSilu, kSeqPerWarp>, grid, dim3(kAdalnThreads),
-                    rows_smem_bytes(IN, kChunk), stream, Wt, bias, extra, x, B, IN, OUT, y, skip_if);
+template <bool kPhi, bool kSilu, int kRows, int kSeqPerWarp>
+static cudaError_t launch_rows_tile(const float* Wt, const float* bias, const float* extra, const float* x, int B,
+                                    int IN, int OUT, float* y, const int32_t* skip_if, cudaStream_t stream) {
+  using Tile = RowsTile<kRows, kSeqPerWarp>;
+  const dim3 grid((OUT + Tile::kSlice - 1) / Tile::kSlice, (B + Tile::kChunk - 1) / Tile::kChunk);
+  return launch_pdl(adaln_rows_kernel<kPhi, kSilu, kRows, kSeqPerWarp>, grid, dim3(kAdalnThreads),
+                    Tile::smem_bytes(IN), stream, Wt, bias, extra, x, B, IN, OUT, y, skip_if);
+}
+
+template <int kRows, int kSeqPerWarp>
+static long long tile_ctas(int B, int OUT) {
+  using Tile = RowsTile<kRows, kSeqPerWarp>;
+  return (long long)((OUT + Tile::kSlice - 1) / Tile::kSlice) * ((B + Tile::kChunk - 1) / Tile::kChunk);
 }
 
 template <bool kPhi, bool kSilu>
 static cudaError_t launch_rows(const float* Wt, const float* bias, const float* extra, const float* x, int B, int IN,
                                int OUT, float* y, const int32_t* skip_if, cudaStream_t stream) {
-  const long long rows = (OUT + kRowSlice - 1) / kRowSlice;
-  if (rows_smem_bytes(IN, 64) <= kWideChunkSmem && rows * ((B + 63) / 64) >= kFillCtas)
-    return launch_rows_spw<kPhi, kSilu, 8>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
-  if (rows * ((B + 15) / 16) >= kFillCtas)
-    return launch_rows_spw<kPhi, kSilu, 2>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
-  return launch_rows_spw<kPhi, kSilu, 1>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
+  if (RowsTile<2, 4>::smem_bytes(IN) <= kWideTileSmem && tile_ctas<2, 4>(B, OUT) >= kFillCtas)
+    return launch_rows_tile<kPhi, kSilu, 2, 4>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
+  if (tile_ctas<1, 2>(B, OUT) >= kFillCtas)
+    return launch_rows_tile<kPhi, kSilu, 1, 2>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
+  return launch_rows_tile<kPhi, kSilu, 1, 1>(Wt, bias, extra, x, B, IN, OUT, y, skip_if, stream);
 }
 
-template <bool kPhi, bool kSilu, int kSeqPerWarp>
+template <bool kPhi, bool kSilu, int kRows, int kSeqPerWarp>
 static bool set_rows_smem(int bytes) {
-  return cudaFuncSetAttribute(adaln_rows_kernel<kPhi, kSilu, kSeqPerWarp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              bytes) == cudaSuccess;
+  return cudaFuncSetAttribute(adaln_rows_kernel<kPhi, kSilu, kRows, kSeqPerWarp>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
 template <typename T>
@@ -288,13 +311,13 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
     if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
-      const int s8 = (int)kWideChunkSmem, s2 = (int)rows_smem_bytes(kMaxWidth, 16),
-                s1 = (int)rows_smem_bytes(kMaxWidth, 8);
-      if (!set_rows_smem<true, true, 8>(s8) || !set_rows_smem<false, true, 8>(s8) ||
-          !set_rows_smem<false, false, 8>(s8) || !set_rows_smem<true, true, 2>(s2) ||
-          !set_rows_smem<false, true, 2>(s2) || !set_rows_smem<false, false, 2>(s2) ||
-          !set_rows_smem<true, true, 1>(s1) || !set_rows_smem<false, true, 1>(s1) ||
-          !set_rows_smem<false, false, 1>(s1))
+      const int sw = (int)kWideTileSmem, s2 = (int)RowsTile<1, 2>::smem_bytes(kMaxWidth),
+                s1 = (int)RowsTile<1, 1>::smem_bytes(kMaxWidth);
+      if (!set_rows_smem<true, true, 2, 4>(sw) || !set_rows_smem<false, true, 2, 4>(sw) ||
+          !set_rows_smem<false, false, 2, 4>(sw) || !set_rows_smem<true, true, 1, 2>(s2) ||
+          !set_rows_smem<false, true, 1, 2>(s2) || !set_rows_smem<false, false, 1, 2>(s2) ||
+          !set_rows_smem<true, true, 1, 1>(s1) || !set_rows_smem<false, true, 1, 1>(s1) ||
+          !set_rows_smem<false, false, 1, 1>(s1))
         return TT_ERR_CUDA;
       __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
     }

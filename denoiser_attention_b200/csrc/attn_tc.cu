@@ -822,9 +822,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 // Merges the partials of groups cut between teams (flash-decoding combine):
 //   O = sum_j 2^(lse_j - M) O_j / sum_j 2^(lse_j - M),  M = max_j lse_j.
 // A CTA takes 32 query rows of one (group, query tile), 8 threads per row, each thread 16 of the
-// 128 dims: it reads its row's log2-sum-exps (the 8 threads of a row read the same words) and its
-// 64-byte slice of every contributor's row, issued together, 4 contributors at a time. CTAs of a
-// group that one team held whole return after reading the group's contributor range.
+// 128 dims: for 4 contributors at a time it loads their log2-sum-exps (the 8 threads of a row read
+// the same words) and its 64-byte slices of their rows together, and combines them against a
+// running maximum (a moving base rescales what was accumulated: exact, the same up to rounding as
+// the two-pass form). CTAs of a group that one team held whole return after reading the group's
+// contributor range.
 constexpr int kMergeRowsPerCta = 32;
 constexpr int kMergeThreads = 256;   // 8 threads per row
 
@@ -858,17 +860,17 @@ __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergePa
   const float* plse = reinterpret_cast<const float*>(p.ws + p.off_lse);
   const int n = (int)(c_hi - c_lo + 1);
   auto slot_of = [&](int j) { return ((size_t)u + (size_t)(c_lo + j)) * (size_t)p.nq + (size_t)qt; };
-  float mx = -INFINITY;
-  for (int j = 0; j < n; ++j) mx = fmaxf(mx, __ldg(plse + slot_of(j) * kRows + row));
+  // contributors 4 at a time, each batch's log2-sum-exps and 64-byte slices loaded together (one
+  // round trip per batch); the running base moves with the batch maximum (online combine)
   float4 acc[4] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f),
                    make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-  float wsum = 0.f;
+  float mx = -INFINITY, wsum = 0.f;
   for (int j0 = 0; j0 < n; j0 += 4) {
     float4 v[4][4];
     float wl[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      wl[q] = 0.f;
+      wl[q] = -INFINITY;
       if (j0 + q < n) {
         const size_t sl = slot_of(j0 + q);
         wl[q] = __ldg(plse + sl * kRows + row);
@@ -876,6 +878,20 @@ __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergePa
 #pragma unroll
         for (int c = 0; c < 4; ++c) v[q][c] = __ldg(src + c);
       }
+    }
+    const float bm = fmaxf(fmaxf(wl[0], wl[1]), fmaxf(wl[2], wl[3]));
+    if (bm > mx) {
+      // a new base: what was accumulated so far is scaled to it (factor 0 on the first batch)
+      const float f = ex2(mx - bm);
+      wsum *= f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[c].x *= f;
+        acc[c].y *= f;
+        acc[c].z *= f;
+        acc[c].w *= f;
+      }
+      mx = bm;
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
