@@ -7,7 +7,7 @@
 //                                          W->W, W->3D), each tiled over slices of 64 or 32
 //                                          weight rows x chunks of 32, 16 or 8 sequences, operands
 //                                          staged in shared memory with asynchronous copies
-//   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one CTA per token row
+//   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one warp per token row
 //   GATED_RESIDUAL   h + gate * f: a vectorised elementwise pass
 // All arithmetic is fp32 (the timestep sinusoid in fp64); bf16 tensors are widened on load and
 // rounded to nearest on store.
@@ -222,48 +222,80 @@ struct Io<__nv_bfloat16> {
   }
 };
 
-// One CTA per token row (b, s): y = h / sqrt(mean(h^2) + eps) * w * (1 + scale_b) + shift_b.
+// 8 consecutive floats (a 16-byte aligned address) into x[0..7], or 4 into x[0..3] (kN == 4)
+template <int kN>
+__device__ __forceinline__ void load_f32(const float* p, float* x) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  if constexpr (kN == 8) {
+    const float4 c = *reinterpret_cast<const float4*>(p + 4);
+    x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+  }
+}
+
+// One warp per token row (b, s): y = h / sqrt(mean(h^2) + eps) * w * (1 + scale_b) + shift_b. A
+// lane keeps up to kNormVec of its row's vectors in registers from the sum of squares to the
+// output (one read of h for rows up to 32 kNormVec vectors: D <= 2048 in bf16), the sum is a
+// warp-shuffle reduction, and w, scale and shift are read as float4.
+constexpr int kNormVec = 8;
+constexpr int kNormRowsPerCta = 4;
+
 template <typename T>
-__global__ void __launch_bounds__(kAdalnThreads) adaln_norm_modulate_kernel(const void* __restrict__ h,
-                                                                            const float* __restrict__ norm_w,
-                                                                            const float* __restrict__ mod,
-                                                                            int S, int D, float eps,
-                                                                            void* __restrict__ out,
-                                                                            const int32_t* skip_if) {
+__global__ void __launch_bounds__(32 * kNormRowsPerCta) adaln_norm_modulate_kernel(const void* __restrict__ h,
+                                                                                   const float* __restrict__ norm_w,
+                                                                                   const float* __restrict__ mod,
+                                                                                   int rows, int S, int D, float eps,
+                                                                                   void* __restrict__ out,
+                                                                                   const int32_t* skip_if) {
   constexpr int N = Io<T>::kN;
   pdl_trigger();
   pdl_wait();
   if (skip_requested(skip_if)) return;
-  const int row = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kNormRowsPerCta + (threadIdx.x >> 5);
+  if (row >= rows) return;
   const int b = row / S;
   const int nv = D / N;
   const size_t vbase = (size_t)row * nv;
   const float* shift = mod + (size_t)b * 3 * D;
   const float* scale = shift + D;
+  float xr[kNormVec][N];
   float ss = 0.f;
-  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+#pragma unroll
+  for (int i = 0; i < kNormVec; ++i) {
+    const int v = lane + 32 * i;
+    if (v < nv) {
+      Io<T>::load(h, vbase + v, xr[i]);
+#pragma unroll
+      for (int k = 0; k < N; ++k) ss = fmaf(xr[i][k], xr[i][k], ss);
+    }
+  }
+  for (int v = lane + 32 * kNormVec; v < nv; v += 32) {   // rows wider than the register cache
     float x[N];
     Io<T>::load(h, vbase + v, x);
 #pragma unroll
     for (int k = 0; k < N; ++k) ss = fmaf(x[k], x[k], ss);
   }
-  __shared__ float s_part[kAdalnThreads / 32];
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_part[w];
-  const float r = 1.0f / sqrtf(tot / (float)D + eps);
-  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+  const float r = 1.0f / sqrtf(warp_sum(ss) / (float)D + eps);
+  auto emit = [&](int v, float* x) {
+    const int j0 = v * N;
+    float w[N], sc[N], sh[N];
+    load_f32<N>(norm_w + j0, w);
+    load_f32<N>(scale + j0, sc);
+    load_f32<N>(shift + j0, sh);
+#pragma unroll
+    for (int k = 0; k < N; ++k) x[k] = fmaf(x[k] * r * w[k], 1.0f + sc[k], sh[k]);
+    Io<T>::store(out, vbase + v, x);
+  };
+#pragma unroll
+  for (int i = 0; i < kNormVec; ++i) {
+    const int v = lane + 32 * i;
+    if (v < nv) emit(v, xr[i]);
+  }
+  for (int v = lane + 32 * kNormVec; v < nv; v += 32) {
     float x[N];
     Io<T>::load(h, vbase + v, x);
-    const int j0 = v * N;
-#pragma unroll
-    for (int k = 0; k < N; ++k) {
-      const int j = j0 + k;
-      x[k] = fmaf(x[k] * r * norm_w[j], 1.0f + scale[j], shift[j]);
-    }
-    Io<T>::store(out, vbase + v, x);
+    emit(v, x);
   }
 }
 
@@ -283,12 +315,12 @@ __global__ void __launch_bounds__(kAdalnThreads) adaln_gated_residual_kernel(con
     const size_t row = v / nv_row;
     const int j0 = (int)(v - row * nv_row) * N;
     const int b = (int)(row / S);
-    const float* gate = mod + (size_t)b * 3 * D + 2 * D;
-    float x[N], y[N];
+    float x[N], y[N], g[N];
     Io<T>::load(h, v, x);
     Io<T>::load(f, v, y);
+    load_f32<N>(mod + (size_t)b * 3 * D + 2 * D + j0, g);
 #pragma unroll
-    for (int k = 0; k < N; ++k) x[k] = fmaf(gate[j0 + k], y[k], x[k]);
+    for (int k = 0; k < N; ++k) x[k] = fmaf(g[k], y[k], x[k]);
     Io<T>::store(out, v, x);
   }
 }
@@ -328,12 +360,14 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
       return TT_ERR_CUDA;
   } else if (a->op == TT_ADALN_NORM_MODULATE) {
     const int rows = B * a->block_size;
-    if (a->dtype == TT_BF16)
-      launch_pdl(adaln_norm_modulate_kernel<__nv_bfloat16>, dim3(rows), dim3(kAdalnThreads), 0, stream, a->h,
-                 a->norm_w, (const float*)a->mod, a->block_size, D, a->eps, a->out, a->skip_if);
-    else
-      launch_pdl(adaln_norm_modulate_kernel<float>, dim3(rows), dim3(kAdalnThreads), 0, stream, a->h, a->norm_w,
-                 (const float*)a->mod, a->block_size, D, a->eps, a->out, a->skip_if);
+    const dim3 grid((rows + kNormRowsPerCta - 1) / kNormRowsPerCta), block(32 * kNormRowsPerCta);
+    const cudaError_t e =
+        (a->dtype == TT_BF16)
+            ? launch_pdl(adaln_norm_modulate_kernel<__nv_bfloat16>, grid, block, 0, stream, a->h, a->norm_w,
+                         (const float*)a->mod, rows, a->block_size, D, a->eps, a->out, a->skip_if)
+            : launch_pdl(adaln_norm_modulate_kernel<float>, grid, block, 0, stream, a->h, a->norm_w,
+                         (const float*)a->mod, rows, a->block_size, D, a->eps, a->out, a->skip_if);
+    if (e != cudaSuccess) return TT_ERR_CUDA;
   } else {
     const int N = (a->dtype == TT_BF16) ? 8 : 4;
     const size_t nvec = (size_t)B * a->block_size * D / N;

@@ -99,6 +99,8 @@ static int validate_adaln(const tt_adaln_args_t* a) {
       const int W = (a->dtype == TT_BF16) ? 8 : 4;
       if (a->hidden % W != 0) return TT_ERR_UNSUPPORTED;
       if (!aligned16(a->h) || !aligned16(a->out) || (a->f && !aligned16(a->f))) return TT_ERR_UNSUPPORTED;
+      // mod and norm_w are read as float4
+      if (!aligned16(a->mod) || (a->norm_w && !aligned16(a->norm_w))) return TT_ERR_UNSUPPORTED;
       return TT_OK;
     }
     default:

@@ -143,7 +143,8 @@ int tt_denoise_attn(const tt_attn_args_t* args, void* workspace, size_t workspac
  *   h, out [B][S][D] E; norm_w [D] float.
  * op TT_ADALN_GATED_RESIDUAL (h, f, mod -> out):
  *   out[b][s] = h[b][s] + gate[b] * f[b][s]        h, f, out [B][S][D] E (out may alias h)
- * D must be a multiple of 8 for TT_BF16 and of 4 for TT_F32.
+ * D must be a multiple of 8 for TT_BF16 and of 4 for TT_F32; h, f, out, mod and norm_w 16-byte
+ * aligned (else TT_ERR_UNSUPPORTED).
  * ------------------------------------------------------------------------------------------- */
 typedef enum {
   TT_ADALN_COND = 0,

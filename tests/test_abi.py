@@ -144,6 +144,8 @@ def _adaln_args(**kw):
     (dict(op=B.TT_ADALN_NORM_MODULATE, hidden=6), B.TT_ERR_UNSUPPORTED),
     (dict(op=B.TT_ADALN_GATED_RESIDUAL, f=None), B.TT_ERR_INVALID_ARGUMENT),
     (dict(op=B.TT_ADALN_GATED_RESIDUAL, dtype=B.TT_BF16, hidden=260), B.TT_ERR_UNSUPPORTED),
+    (dict(op=B.TT_ADALN_NORM_MODULATE, norm_w=4100), B.TT_ERR_UNSUPPORTED),      # read as float4
+    (dict(op=B.TT_ADALN_GATED_RESIDUAL, mod=4104), B.TT_ERR_UNSUPPORTED),
 ])
 def test_adaln_host_validation(lib, kw, status):
     a = _adaln_args(**kw)
