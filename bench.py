@@ -78,6 +78,16 @@ def measured_peaks():
     return 6650.0, "of fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor peak in TFLOP/s for a kernel timed alone (the burst figure), and its source."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "of measured"
+    return 1590.0, "of fallback"
+
+
 # ------------------------------------------------------------------------------------------ clocks
 class ClockSampler:
     """Samples nvidia-smi clocks and throttle reasons in the background."""
@@ -464,6 +474,7 @@ def run_extras(args, dev, peak):
     import torch
     from denoiser_attention_b200 import api, synth
     out = {}
+    tpeak, tpeak_src = measured_tensor_peak()
     # ---- the decode step (8 sequences, ctx 4096): whole step and its kernels. Its attention leaves
     # SMs idle (528 key tiles over 148 CTAs), so the three branches on forked streams overlap well
     # here (for the batch workload they only take turns)
@@ -521,11 +532,13 @@ def run_extras(args, dev, peak):
         ms = isolated_ms(attn_op(step), sets, outs, torch.cuda.Stream(device=dev), reps=max(3, 200 // n_sets))
         kvb = kv_bytes_of(w.attn)
         key = name if S is None else f"{name}_S{S}"
+        tflops = attn_flops_of(w.attn) / (ms * 1e-3) / 1e12
         attn[key] = {"us": ms * 1e3, "kv_gbs": kvb / (ms * 1e-3) / 1e9, "frac": kvb / (ms * 1e-3) / 1e9 / peak,
-                     "tflops": attn_flops_of(w.attn) / (ms * 1e-3) / 1e12, "kv_bytes": kvb}
+                     "tflops": tflops, "tensor_frac": tflops / tpeak, "kv_bytes": kvb}
         del sets, outs, a
         torch.cuda.empty_cache()
     out["attention"] = attn
+    out["attention_peaks"] = {"hbm_gbs": peak, "bf16_tflops": tpeak, "tensor_peak_source": tpeak_src}
     # ---- the block-sweep unmask table: per S the unmask step time, and per (S, temperature,
     # gamma) the mean number of positions committed in the first refinement step (all masked)
     table = []
