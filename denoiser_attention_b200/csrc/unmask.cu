@@ -116,6 +116,9 @@ __device__ __forceinline__ long long owner_of(long long v, long long E, long lon
 }
 
 // Commit rule for one sequence, run by the whole CTA.
+// blocks up to this many positions rank by counting; longer ones sort
+constexpr int kRankLoopMax = 64;
+
 __device__ void commit_sequence(const UnmaskParams& p, int b, const float* conf_ws, const int32_t* arg_ws) {
   __shared__ float s_conf[1024];
   __shared__ uint8_t s_masked[1024];
@@ -149,16 +152,56 @@ __device__ void commit_sequence(const UnmaskParams& p, int b, const float* conf_
   }
   // a masked position commits iff its rank among masked positions (confidence descending,
   // position ascending) is below K; every position >= gamma ranks below n_ge <= K.
-  for (int l = tid; l < S; l += blockDim.x) {
-    if (!s_masked[l]) continue;
-    const float cl = s_conf[l];
-    int rank = 0;
-    for (int j = 0; j < S; ++j) {
-      if (!s_masked[j]) continue;
-      const float cj = s_conf[j];
-      rank += (cj > cl || (cj == cl && j < l)) ? 1 : 0;
+  if (S <= kRankLoopMax) {
+    // short blocks: each thread counts its positions' ranks directly (S comparisons each)
+    for (int l = tid; l < S; l += blockDim.x) {
+      if (!s_masked[l]) continue;
+      const float cl = s_conf[l];
+      int rank = 0;
+      for (int j = 0; j < S; ++j) {
+        if (!s_masked[j]) continue;
+        const float cj = s_conf[j];
+        rank += (cj > cl || (cj == cl && j < l)) ? 1 : 0;
+      }
+      if (rank < K) {
+        p.tokens[(size_t)b * S + l] = __ldcg(arg_ws + (size_t)b * S + l);
+        p.is_masked[(size_t)b * S + l] = 0;
+      }
     }
-    if (rank < K) {
+  } else {
+    // long blocks: a bitonic sort of 64-bit keys (confidence descending in the high word,
+    // position ascending in the low word; unmasked positions and the padding to a power of two
+    // sort last), then the first K sorted positions commit
+    __shared__ unsigned long long s_key[1024];
+    int P = 1;
+    while (P < S) P <<= 1;
+    for (int l = tid; l < P; l += blockDim.x) {
+      unsigned long long key = ~0ull;
+      if (l < S && s_masked[l]) {
+        const uint32_t u = __float_as_uint(s_conf[l]);
+        const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);   // ascending in the float's order
+        key = ((unsigned long long)(~ord) << 32) | (uint32_t)l;
+      }
+      s_key[l] = key;
+    }
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int jd = k >> 1; jd > 0; jd >>= 1) {
+        for (int i = tid; i < P; i += blockDim.x) {
+          const int ix = i ^ jd;
+          if (ix > i) {
+            const unsigned long long x = s_key[i], y = s_key[ix];
+            if ((x > y) == ((i & k) == 0)) {
+              s_key[i] = y;
+              s_key[ix] = x;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int r = tid; r < min(K, n_masked); r += blockDim.x) {
+      const int l = (int)(uint32_t)(s_key[r] & 0xffffffffull);
       p.tokens[(size_t)b * S + l] = __ldcg(arg_ws + (size_t)b * S + l);
       p.is_masked[(size_t)b * S + l] = 0;
     }

@@ -1,8 +1,8 @@
 """Eq. (1) attention on the GPU (through the C ABI) against the CPU fp64 oracle.
 
-Cases span several 64-token tiles with ragged tails, empty contexts (the first block), block
-sizes 1..64, grouped-query layouts with 1..64 query heads per kv head, paged KV in shuffled page
-order, the tiny fp32 workload, and the full-size decode, batch and ragged-paged workloads (the
+Cases span several 128-token key tiles with ragged tails, empty contexts (the first block), block
+sizes 1..64, grouped-query layouts with 1..128 query heads per kv head, an odd number of query
+tiles per group (the last CTA of a team then holds one), paged KV in shuffled page order, the tiny fp32 workload, and the full-size decode, batch and ragged-paged workloads (the
 last ones on sampled sequences where the whole batch would be slow for the oracle)."""
 import math
 
@@ -68,6 +68,9 @@ CASES = [
     # more than 32 groups with the group-aligned partition (on 148 SMs: 74 teams):
     (36, 16, 32, 2, 128, [300] * 36, torch.bfloat16, 0),    # 72 groups of 4 tiles, one team each
     (17, 16, 32, 2, 128, [1024] * 17, torch.bfloat16, 0),   # 34 groups of 9 tiles, chunks of 4 + 5
+    # three query tiles per group: G = 16, S = 24 (8 positions per tile); G = 128, S = 3 (one each)
+    (2, 24, 32, 2, 128, [300, 50], torch.bfloat16, 0),
+    (1, 3, 128, 1, 128, [200], torch.bfloat16, 0),
 ]
 
 
