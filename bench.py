@@ -658,7 +658,9 @@ def run_kernel(args):
         bufs, out, op, nbytes = lmhead_inputs(dev), None, lmhead_op(), 131072 * 2048 * 2
         desc = "x 8x16x2048, W 131072x2048 bf16"
     else:
-        w = synth.workload(args.workload)
+        # "name" or "name:S" (a block size for the sweep workload)
+        name, _, bs = args.workload.partition(":")
+        w = synth.workload(name, block_size=int(bs) if bs else None)
         if args.kernel == "attn":
             a = synth.attention_inputs(w.attn, seed=w.seed)
             bufs = api.StepBuffers(tau=None, h=None, f=None, q=a.q.to(dev), k_blk=a.k_blk.to(dev),
@@ -701,7 +703,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="the step's workload (default: the batch-generation workload, the headline)")
+                    help="the step's workload (default: the batch-generation workload, the headline); with "
+                         "--kernel also name:S, e.g. sweep_bf16:4")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the extra keys (decode step, attention per workload, block-sweep unmask table)")
     ap.add_argument("--schedule", choices=list(SCHEDULE_TEXT), default="branches",

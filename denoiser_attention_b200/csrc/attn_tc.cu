@@ -35,6 +35,8 @@
 // running maximum; only when a tile's maximum exceeds it by more than 8 (P > 256) does the
 // base move to the tile maximum, with O rescaled (exact: numerator and denominator share the
 // stale maximum).
+// Groups with a single query tile (G * S <= 128) run a second kernel, attn_tc1_kernel (namespace
+// `one` below), which puts both softmax warpgroups on that one tile.
 #include <cstdio>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -170,7 +172,8 @@ struct SegWalk {
   long long ustart;
   long long g, gend;
   GroupInfo gi;
-  __device__ void init(const TcParams& p, const Smem& sm, WsHeader* hdr) {
+  template <class Sm>
+  __device__ void init(const TcParams& p, const Sm& sm, WsHeader* hdr) {
     u = sm.u0;
     ustart = sm.u0_start;
     g = sm.range_begin;
@@ -206,6 +209,130 @@ __device__ __forceinline__ long long floor_div(long long a, long long b) {
 // Team owning global tile t when T tiles are cut into P <= T ranges [c*T/P, (c+1)*T/P).
 __device__ __forceinline__ long long owner_team(long long t, long long T, long long P) {
   return floor_div((t + 1) * P - 1, T);
+}
+
+// Warp 0 of every CTA: this team's tile range [range_begin, range_end) and the group where it
+// starts, written to the CTA's shared block; CTA 0 also records, per group, the teams that hold its
+// partials (for the merge kernel).
+template <class Sm>
+__device__ void partition_tiles(const TcParams& p, Sm& sm, int team, int lane, WsHeader* hdr) {
+  // 32-bit arithmetic where the values allow it: 64-bit division is a long instruction
+  // sequence, and this warp's chain of them sits before the first load
+  auto wsum = [](uint32_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+  };
+  long long T = 0;
+  int nmax = 0;
+  int n_first = 0;   // this lane's group in the first 32 (kept: one read of ctx_lens for those)
+  for (int base = 0; base < p.groups; base += 32) {
+    const int u = base + lane;
+    int n = 0;
+    if (u < p.groups) n = group_info(p, u, blockIdx.x == 0, hdr).ntiles;
+    if (base == 0) n_first = n;
+    nmax = max(nmax, n);
+    T += wsum((uint32_t)n);   // a group has fewer than 2^24 tiles (int32 lengths)
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nmax = max(nmax, __shfl_xor_sync(0xffffffffu, nmax, o));
+  auto ntiles_of = [&](int base, int u) -> int {
+    return (u < p.groups) ? (base == 0 ? n_first : group_info(p, u, false, hdr).ntiles) : 0;
+  };
+  // with fewer tiles than teams only the first T teams work (one tile each), so every working
+  // team owns a non-empty range and the teams of a group are consecutive
+  const long long Pu = T < p.teams ? T : p.teams;
+  uint32_t t_al = 0;   // chunk bound of the group-aligned partition; 0 = uniform
+  if (T > 0 && T < (1LL << 31) && p.groups <= p.teams) {
+    const uint32_t T32 = (uint32_t)T, teams32 = (uint32_t)p.teams, Pu32 = (uint32_t)Pu;
+    // candidates t in [ceil(T/teams), ceil(T/Pu) + kSegPenaltyTiles], at most kSegPenaltyTiles + 1
+    // of them (ceil(T/Pu) = ceil(T/teams) when Pu = teams, and both are 1 when Pu = T < teams):
+    // sum_u ceil(n_u / t) for all of them in one pass, independent divisions side by side
+    const uint32_t lo = (T32 - 1) / teams32 + 1;
+    uint32_t hi = (T32 - 1) / Pu32 + 1 + (uint32_t)kSegPenaltyTiles;
+    if (hi > (uint32_t)nmax) hi = (uint32_t)nmax;
+    constexpr int kCand = (int)kSegPenaltyTiles + 1;
+    uint32_t cnt[kCand];
+#pragma unroll
+    for (int k = 0; k < kCand; ++k) cnt[k] = 0;
+    for (int base = 0; base < p.groups; base += 32) {
+      const uint32_t n = (uint32_t)ntiles_of(base, base + lane);
+#pragma unroll
+      for (int k = 0; k < kCand; ++k) cnt[k] += (n + lo + k - 1) / (lo + k);
+    }
+#pragma unroll
+    for (int k = 0; k < kCand; ++k) cnt[k] = wsum(cnt[k]);
+    // the smallest feasible candidate (the count does not increase with t)
+#pragma unroll
+    for (int k = kCand - 1; k >= 0; --k)
+      if (lo + k <= hi && cnt[k] <= teams32) t_al = lo + k;
+  }
+  const bool aligned = t_al > 0;
+  long long rb = T, re = T;
+  if (!aligned && team < Pu) {
+    rb = floor_div(team * T, Pu);
+    re = floor_div((team + 1) * T, Pu);
+  }
+  long long acc = 0, cacc = 0;
+  int u0 = -1;
+  long long u0s = 0;
+  int2* crange_out = reinterpret_cast<int2*>(p.ws + p.off_crange);
+  const bool record = (blockIdx.x == 0);
+  for (int base = 0; base < p.groups && (u0 < 0 || record); base += 32) {
+    const int u = base + lane;
+    const int n = ntiles_of(base, u);
+    const int c = aligned ? (int)(((uint32_t)n + t_al - 1) / t_al) : 0;   // chunks (teams) of group u
+    int incl = n, cincl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      const int z = __shfl_up_sync(0xffffffffu, cincl, o);
+      if (lane >= o) {
+        incl += y;
+        cincl += z;
+      }
+    }
+    const long long lo = acc + incl - n, hi = acc + incl;   // tiles of group u
+    const long long c0 = cacc + cincl - c;                  // its first team (aligned)
+    if (record && u < p.groups) {
+      // n >= 1 (the block tile), so hi - 1 >= lo
+      crange_out[u] = aligned ? make_int2((int)c0, (int)(c0 + c - 1))
+                              : make_int2((int)owner_team(lo, T, Pu), (int)owner_team(hi - 1, T, Pu));
+    }
+    const bool mine = u < p.groups && (aligned ? (c0 <= team && team < c0 + c) : (lo <= rb && rb < hi));
+    const unsigned hit = __ballot_sync(0xffffffffu, mine);
+    if (hit && u0 < 0) {
+      const int src = __ffs(hit) - 1;
+      u0 = base + src;
+      u0s = __shfl_sync(0xffffffffu, lo, src);
+      const uint32_t nn = (uint32_t)__shfl_sync(0xffffffffu, n, src);
+      const uint32_t cc = (uint32_t)__shfl_sync(0xffffffffu, c, src);
+      const uint32_t j = (uint32_t)(team - __shfl_sync(0xffffffffu, c0, src));
+      if (aligned) {
+        // chunk j covers [j*nn/cc, (j+1)*nn/cc) of the group, from the quotient and remainder
+        // of nn/cc (j*nn may not fit 32 bits; j*r < cc^2 does)
+        const uint32_t q = nn / cc, r = nn - q * cc;
+        rb = u0s + (long long)j * q + (j * r) / cc;
+        re = u0s + (long long)(j + 1) * q + ((j + 1) * r) / cc;
+      }
+    }
+    acc += __shfl_sync(0xffffffffu, incl, 31);
+    cacc += __shfl_sync(0xffffffffu, cincl, 31);
+  }
+  if (lane == 0) {
+    sm.total_tiles = T;
+    sm.p_eff = aligned ? cacc : Pu;
+    sm.range_begin = rb;
+    sm.range_end = re;
+    sm.u0 = u0;
+    sm.u0_start = u0s;
+    sm.abort_flag = 0;
+    if (record) {
+      AttnMeta* meta = reinterpret_cast<AttnMeta*>(p.ws + p.off_meta);
+      meta->total_tiles = T;
+      meta->p_eff = aligned ? cacc : Pu;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
@@ -268,125 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   // (possible when groups <= teams): each group u is cut into ceil(n_u / t) near-equal chunks for
   // the smallest t with sum_u ceil(n_u / t) <= teams, one chunk per team, so no team runs two
   // segments. The aligned one is used when t <= ceil(T/P) + kSegPenaltyTiles.
-  if (warp == 0) {
-    // 32-bit arithmetic where the values allow it: 64-bit division is a long instruction
-    // sequence, and this warp's chain of them sits before the first load
-    auto wsum = [](uint32_t v) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      return v;
-    };
-    long long T = 0;
-    int nmax = 0;
-    int n_first = 0;   // this lane's group in the first 32 (kept: one read of ctx_lens for those)
-    for (int base = 0; base < p.groups; base += 32) {
-      const int u = base + lane;
-      int n = 0;
-      if (u < p.groups) n = group_info(p, u, blockIdx.x == 0, hdr).ntiles;
-      if (base == 0) n_first = n;
-      nmax = max(nmax, n);
-      T += wsum((uint32_t)n);   // a group has fewer than 2^24 tiles (int32 lengths)
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) nmax = max(nmax, __shfl_xor_sync(0xffffffffu, nmax, o));
-    auto ntiles_of = [&](int base, int u) -> int {
-      return (u < p.groups) ? (base == 0 ? n_first : group_info(p, u, false, hdr).ntiles) : 0;
-    };
-    // with fewer tiles than teams only the first T teams work (one tile each), so every working
-    // team owns a non-empty range and the teams of a group are consecutive
-    const long long Pu = T < p.teams ? T : p.teams;
-    uint32_t t_al = 0;   // chunk bound of the group-aligned partition; 0 = uniform
-    if (T > 0 && T < (1LL << 31) && p.groups <= p.teams) {
-      const uint32_t T32 = (uint32_t)T, teams32 = (uint32_t)p.teams, Pu32 = (uint32_t)Pu;
-      // candidates t in [ceil(T/teams), ceil(T/Pu) + kSegPenaltyTiles], at most kSegPenaltyTiles + 1
-      // of them (ceil(T/Pu) = ceil(T/teams) when Pu = teams, and both are 1 when Pu = T < teams):
-      // sum_u ceil(n_u / t) for all of them in one pass, independent divisions side by side
-      const uint32_t lo = (T32 - 1) / teams32 + 1;
-      uint32_t hi = (T32 - 1) / Pu32 + 1 + (uint32_t)kSegPenaltyTiles;
-      if (hi > (uint32_t)nmax) hi = (uint32_t)nmax;
-      constexpr int kCand = (int)kSegPenaltyTiles + 1;
-      uint32_t cnt[kCand];
-#pragma unroll
-      for (int k = 0; k < kCand; ++k) cnt[k] = 0;
-      for (int base = 0; base < p.groups; base += 32) {
-        const uint32_t n = (uint32_t)ntiles_of(base, base + lane);
-#pragma unroll
-        for (int k = 0; k < kCand; ++k) cnt[k] += (n + lo + k - 1) / (lo + k);
-      }
-#pragma unroll
-      for (int k = 0; k < kCand; ++k) cnt[k] = wsum(cnt[k]);
-      // the smallest feasible candidate (the count does not increase with t)
-#pragma unroll
-      for (int k = kCand - 1; k >= 0; --k)
-        if (lo + k <= hi && cnt[k] <= teams32) t_al = lo + k;
-    }
-    const bool aligned = t_al > 0;
-    long long rb = T, re = T;
-    if (!aligned && team < Pu) {
-      rb = floor_div(team * T, Pu);
-      re = floor_div((team + 1) * T, Pu);
-    }
-    long long acc = 0, cacc = 0;
-    int u0 = -1;
-    long long u0s = 0;
-    int2* crange_out = reinterpret_cast<int2*>(p.ws + p.off_crange);
-    const bool record = (blockIdx.x == 0);
-    for (int base = 0; base < p.groups && (u0 < 0 || record); base += 32) {
-      const int u = base + lane;
-      const int n = ntiles_of(base, u);
-      const int c = aligned ? (int)(((uint32_t)n + t_al - 1) / t_al) : 0;   // chunks (teams) of group u
-      int incl = n, cincl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        const int z = __shfl_up_sync(0xffffffffu, cincl, o);
-        if (lane >= o) {
-          incl += y;
-          cincl += z;
-        }
-      }
-      const long long lo = acc + incl - n, hi = acc + incl;   // tiles of group u
-      const long long c0 = cacc + cincl - c;                  // its first team (aligned)
-      if (record && u < p.groups) {
-        // n >= 1 (the block tile), so hi - 1 >= lo
-        crange_out[u] = aligned ? make_int2((int)c0, (int)(c0 + c - 1))
-                                : make_int2((int)owner_team(lo, T, Pu), (int)owner_team(hi - 1, T, Pu));
-      }
-      const bool mine = u < p.groups && (aligned ? (c0 <= team && team < c0 + c) : (lo <= rb && rb < hi));
-      const unsigned hit = __ballot_sync(0xffffffffu, mine);
-      if (hit && u0 < 0) {
-        const int src = __ffs(hit) - 1;
-        u0 = base + src;
-        u0s = __shfl_sync(0xffffffffu, lo, src);
-        const uint32_t nn = (uint32_t)__shfl_sync(0xffffffffu, n, src);
-        const uint32_t cc = (uint32_t)__shfl_sync(0xffffffffu, c, src);
-        const uint32_t j = (uint32_t)(team - __shfl_sync(0xffffffffu, c0, src));
-        if (aligned) {
-          // chunk j covers [j*nn/cc, (j+1)*nn/cc) of the group, from the quotient and remainder
-          // of nn/cc (j*nn may not fit 32 bits; j*r < cc^2 does)
-          const uint32_t q = nn / cc, r = nn - q * cc;
-          rb = u0s + (long long)j * q + (j * r) / cc;
-          re = u0s + (long long)(j + 1) * q + ((j + 1) * r) / cc;
-        }
-      }
-      acc += __shfl_sync(0xffffffffu, incl, 31);
-      cacc += __shfl_sync(0xffffffffu, cincl, 31);
-    }
-    if (lane == 0) {
-      sm.total_tiles = T;
-      sm.p_eff = aligned ? cacc : Pu;
-      sm.range_begin = rb;
-      sm.range_end = re;
-      sm.u0 = u0;
-      sm.u0_start = u0s;
-      sm.abort_flag = 0;
-      if (record) {
-        AttnMeta* meta = reinterpret_cast<AttnMeta*>(p.ws + p.off_meta);
-        meta->total_tiles = T;
-        meta->p_eff = aligned ? cacc : Pu;
-      }
-    }
-  }
+  if (warp == 0) partition_tiles(p, sm, team, lane, hdr);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
@@ -819,6 +828,588 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Groups with a single query tile (G * S <= 128, e.g. S <= 8 at G = 16): the two-stream kernel
+// above would run one softmax stream per CTA and leave the other warpgroup idle. This kernel
+// puts the tile's work on both: one query tile per CTA; the softmax split by key columns between
+// the two warpgroups (a thread owns one query row and 64 of a tile's 128 columns; the row's two
+// threads exchange their maxima once per tile and their sums once per segment through shared
+// memory and a named barrier of the warp pair); three S buffers in TMEM (O [0,128), S at 128,
+// 256, 384) so that the scores run three tiles ahead of the PV products, which the softmax of
+// the next tile therefore never waits for; warp 3 issues the QK products and warp 1 the PV
+// products (one thread each; a QK refills its S buffer once the PV that read P there has
+// completed); warp 0 loads the query tile and a 3-stage K ring, warp 2 a 2-stage V ring. The
+// partition of the key tiles, the segment walk, the output and the split-KV partials are those
+// of the two-stream kernel.
+namespace one {
+
+constexpr int kKStages = 3;       // K ring depth (= kSBufs: a stage's QK completion is also its S)
+constexpr int kVStages = 2;       // V ring depth
+constexpr int kSBufs = 3;         // S buffers in TMEM: QK runs this many tiles ahead of PV
+static_assert(kKStages == kSBufs, "k_empty[g % kSBufs] doubles as the S-ready barrier of tile g");
+constexpr int kHalves = 2;        // softmax warpgroups, each 64 of a tile's 128 key columns
+constexpr int kThreads = 128 + kHalves * kRows;
+constexpr int kLaunchRegs = 168, kProducerRegs = 88, kSoftmaxRegs = 208;
+static_assert(128 * kProducerRegs + 2 * 128 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS = 128;  // O at columns [0, 128), S buffer b at kTmemS + 128 b
+static_assert(kTmemS + 128 * kSBufs <= kTmemCols, "TMEM budget");
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemK = kQBytes;
+constexpr uint32_t kSmemV = kSmemK + kKStages * kKBytesPerStage;
+constexpr uint32_t kSmemBar = kSmemV + kVStages * kKBytesPerStage;
+// the two halves' exchanges (row maxima per tile, row sums per segment): values and the warps'
+// good flags, double-buffered by exchange parity
+constexpr uint32_t kSmemX = kSmemBar + 1024;
+constexpr uint32_t kXBytes = 2 * kHalves * kRows * 4 + 2 * kHalves * 4 * 4;
+constexpr uint32_t kSmemBytes = kSmemX + kXBytes + 1024;       // + alignment slack
+
+struct Smem {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  // k_empty[b] completes when the QK of a tile using K stage b = S buffer b has completed: the K
+  // stage is free and the tile's S is ready (one phase per tile using b)
+  uint64_t p_full[kSBufs];     // P of a tile is in S buffer b (and O rescaled): both halves' warps
+  uint64_t pv_done[kSBufs];    // O += P V of a tile using S buffer b has completed
+  uint64_t o_full;             // O of the segment is complete (one phase per segment)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  long long range_begin, range_end, total_tiles, p_eff;
+  int u0;
+  long long u0_start;
+};
+static_assert(sizeof(Smem) <= 1024, "barrier block");
+
+// Slot and phase parity of use n of an R-deep ring (a CTA's tile counters: n < 2^32), in 32-bit
+// arithmetic (a 64-bit division is a long instruction sequence, and these sit in every tile's chain).
+template <int R>
+__device__ __forceinline__ int ring_slot(long long n) {
+  return (int)((uint32_t)n % (uint32_t)R);
+}
+template <int R>
+__device__ __forceinline__ uint32_t ring_phase(long long n) {
+  return ((uint32_t)n / (uint32_t)R) & 1u;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attn_tc1_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>(smem + kSmemBar);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int team = blockIdx.x / p.nq;
+  const int qt = blockIdx.x % p.nq;                      // this CTA's query tile
+
+  // ---- 0. prologue that touches no input: barriers, TMEM, tensor-map prefetch. With a
+  // programmatic launch it overlaps the previous kernel; inputs are read after pdl_wait().
+  if (warp == 0 && lane == 0) {
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sm.v_full[i], 1);
+      mbar_init(&sm.v_empty[i], 1);
+    }
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(&sm.p_full[b], kHalves * kRows / 32);   // one arrival per softmax warp
+      mbar_init(&sm.pv_done[b], 1);
+    }
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.drain, 2);   // both MMA-issuing threads
+    fence_barrier_init();
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_kc);
+    prefetch_tmap(&p.tm_vc);
+    prefetch_tmap(&p.tm_kb);
+    prefetch_tmap(&p.tm_vb);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  pdl_trigger();
+  pdl_wait();
+  if (skip_requested(p.skip_if)) {
+    // early exit of a multi-step loop: nothing to do; release TMEM and leave
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(sm.tmem_base, kTmemCols);
+    }
+    return;
+  }
+
+  // ---- 1. this team's tile range and the group where it starts (warp 0); CTA 0 also records,
+  // per group, the teams that hold its partials (for the merge kernel).
+  // Two partitions of the T tiles (in group order) are considered. Uniform: team c takes
+  // [c*T/P, (c+1)*T/P), which balances tiles but lets ranges cross group boundaries. Group-aligned
+  // (possible when groups <= teams): each group u is cut into ceil(n_u / t) near-equal chunks for
+  // the smallest t with sum_u ceil(n_u / t) <= teams, one chunk per team, so no team runs two
+  // segments. The aligned one is used when t <= ceil(T/P) + kSegPenaltyTiles.
+  if (warp == 0) partition_tiles(p, sm, team, lane, hdr);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  const bool has_work = team < p.teams && sm.range_begin < sm.range_end && sm.u0 >= 0;
+
+  auto fail = [&](uint32_t detail) {
+    report_error(hdr, TT_ERR_DEVICE_TIMEOUT, detail);
+    *abort_flag = 1;
+  };
+
+  const uint32_t sQ = smem_u32(smem + kSmemQ);
+  const uint32_t sK = smem_u32(smem + kSmemK);
+  const uint32_t sV = smem_u32(smem + kSmemV);
+
+  if (warp < 4) {
+    setmaxnreg_dec<kProducerRegs>();
+  if (!has_work) {
+    // nothing to do (more teams than tiles, or a CTA beyond the last full team)
+  } else if (warp == 0 || warp == 2) {
+    // ======================= TMA producers: warp 0 loads the query tiles and the K ring, warp 2
+    // the V ring, so that neither ring waits for the other
+    if (lane == 0) {
+      const bool do_kq = (warp == 0);
+      const bool do_v = (warp == 2);
+      SegWalk w;
+      w.init(p, sm, hdr);
+      long long f = 0;
+      int qn = 0;
+      bool ok = true;
+      const uint32_t q_bytes = 2u * 128u * (uint32_t)p.G * (uint32_t)p.s_per_tile;   // one query tile
+      while (ok && !w.done()) {
+        int kb, ke;
+        w.segment(kb, ke);
+        const GroupInfo& gi = w.gi;
+        if (do_kq) {
+          if (qn > 0 && !mbar_wait_bounded(&sm.q_empty, (qn - 1) & 1, abort_flag)) {
+            fail(kDetailWaitQEmpty);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.q_full, q_bytes);
+          const int qrow = gi.b * p.S + qt * p.s_per_tile;
+          uint8_t* qdst = smem + kSmemQ;
+          tma_load_3d(qdst, &p.tm_q, &sm.q_full, 0, gi.kvh * p.G, qrow);
+          tma_load_3d(qdst + kQBytesPerDh, &p.tm_q, &sm.q_full, 64, gi.kvh * p.G, qrow);
+          ++qn;
+        }
+        for (int k = kb; k < ke; ++k, ++f) {
+          const CUtensorMap* mk;
+          const CUtensorMap* mv;
+          int row;
+          if (k < gi.nctx) {
+            const int t0 = k * kTile;
+            if (p.paged) {
+              int pg = p.page_table[(size_t)gi.b * p.max_pages + t0 / p.page_size];
+              if (pg < 0 || pg >= p.num_pages) {
+                report_error(hdr, TT_ERR_DEVICE, kDetailBadPage);
+                pg = 0;   // read a valid page instead; the result is unspecified, the error is set
+              }
+              row = pg * p.page_size + t0 % p.page_size;
+            } else {
+              row = gi.b * p.ctx_stride + t0;
+            }
+            mk = &p.tm_kc;
+            mv = &p.tm_vc;
+          } else {
+            row = gi.b * p.S;
+            mk = &p.tm_kb;
+            mv = &p.tm_vb;
+          }
+          if (do_kq) {
+            // K of a stage is free once its QK^T has read it
+            const int ks = ring_slot<kKStages>(f);
+            const uint32_t kround = (uint32_t)f / (uint32_t)kKStages;
+            if (kround > 0 && !mbar_wait_bounded(&sm.k_empty[ks], (kround - 1) & 1, abort_flag)) {
+              fail(kDetailWaitKvEmpty);
+              ok = false;
+              break;
+            }
+            uint8_t* kdst = smem + kSmemK + ks * kKBytesPerStage;
+            mbar_arrive_expect_tx(&sm.k_full[ks], kKBytesPerStage);
+            tma_load_3d(kdst, mk, &sm.k_full[ks], 0, gi.kvh, row);
+            tma_load_3d(kdst + kKVBoxBytes, mk, &sm.k_full[ks], 64, gi.kvh, row);
+          }
+          if (do_v) {
+            // V of a stage is free once its PV has read it
+            const int vs = ring_slot<kVStages>(f);
+            const uint32_t vround = (uint32_t)f / (uint32_t)kVStages;
+            if (vround > 0 && !mbar_wait_bounded(&sm.v_empty[vs], (vround - 1) & 1, abort_flag)) {
+              fail(kDetailWaitKvEmpty);
+              ok = false;
+              break;
+            }
+            uint8_t* vdst = smem + kSmemV + vs * kKBytesPerStage;
+            mbar_arrive_expect_tx(&sm.v_full[vs], kKBytesPerStage);
+            tma_load_3d(vdst, mv, &sm.v_full[vs], 0, gi.kvh, row);
+            tma_load_3d(vdst + kKVBoxBytes, mv, &sm.v_full[vs], 64, gi.kvh, row);
+          }
+        }
+        if (!ok) break;
+        w.advance(p, hdr);
+      }
+      // make sure every copy this thread issued has landed before the CTA can exit
+      const long long nf = f;
+      const uint64_t t0 = globaltimer_ns();
+      if (do_kq) {
+        for (long long jj = (nf > kKStages ? nf - kKStages : 0); jj < nf; ++jj)
+          while (!mbar_try_wait(&sm.k_full[jj % kKStages], (uint32_t)((jj / kKStages) & 1)) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        if (qn > 0)
+          while (!mbar_try_wait(&sm.q_full, (uint32_t)((qn - 1) & 1)) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+      }
+      if (do_v) {
+        for (long long jj = (nf > kVStages ? nf - kVStages : 0); jj < nf; ++jj)
+          while (!mbar_try_wait(&sm.v_full[jj % kVStages], (uint32_t)((jj / kVStages) & 1)) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+      }
+    }
+  } else if (warp == 1 || warp == 3) {
+    // ======================= MMA issuers: warp 1 the PV products, warp 3 the QK products (one
+    // thread each; each thread's products run in its issue order, the two threads' products
+    // interleave on the tensor pipe)
+    if (lane == 0) {
+      SegWalk w;
+      w.init(p, sm, hdr);
+      // descriptor bases; per-MMA descriptors add constant offsets to the start-address field
+      // (bits 0..13, 16-byte units), which shared-memory addresses below 256 KB never carry out of
+      const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sV, kKVBoxBytes, 1024);
+      long long f = 0;   // tiles of this CTA so far (all segments)
+      int seg = 0;
+      bool ok = true;
+      while (ok && !w.done()) {
+        int kb, ke;
+        w.segment(kb, ke);
+        const long long fs = f, fe = f + (ke - kb);   // this segment's tiles [fs, fe)
+        if (warp == 3) {
+          // S(g) = Q K(g)^T into S buffer g % kSBufs. That buffer held P of tile g - kSBufs: wait
+          // for its PV (pv_done is then exactly one phase behind: PV(g) needs this S first).
+          if (!mbar_wait_bounded(&sm.q_full, (uint32_t)(seg & 1), abort_flag)) {
+            fail(kDetailWaitQFull);
+            break;
+          }
+          for (; f < fe; ++f) {
+            const int b = ring_slot<kSBufs>(f);
+            if (f >= kSBufs) {
+              if (!mbar_wait_bounded(&sm.pv_done[b], ring_phase<kSBufs>(f - kSBufs), abort_flag)) {
+                fail(kDetailWaitPvDone);
+                ok = false;
+                break;
+              }
+            }
+            if (!mbar_wait_bounded(&sm.k_full[b], ring_phase<kKStages>(f), abort_flag)) {
+              fail(kDetailWaitKvFull);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d_tm = tmem + kTmemS + 128u * (uint32_t)b;
+            const uint64_t kd = dk0 + (uint64_t)((b * kKBytesPerStage) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off_q = ((kk >> 2) * kQBytesPerDh + (kk & 3) * 32) >> 4;
+              const uint32_t off_k = ((kk >> 2) * kKVBoxBytes + (kk & 3) * 32) >> 4;
+              mma_ss(d_tm, dq0 + off_q, kd + off_k, kIdescQK, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&sm.k_empty[b]);   // K stage free, S of tile f ready
+            if (f == fe - 1) tc_commit(&sm.q_empty);
+          }
+        } else {
+          // O (+)= P(f) V(f); P is in TMEM over the first 64 columns of S buffer f % kSBufs (keys
+          // 2c, 2c+1 in column c)
+          for (; f < fe; ++f) {
+            const int stage = ring_slot<kVStages>(f);
+            const int b = ring_slot<kSBufs>(f);
+            if (!mbar_wait_bounded(&sm.v_full[stage], ring_phase<kVStages>(f), abort_flag)) {
+              fail(kDetailWaitKvFull);
+              ok = false;
+              break;
+            }
+            // P of tile f written (and O rescaled) by both halves of the softmax
+            if (!mbar_wait_bounded(&sm.p_full[b], ring_phase<kSBufs>(f), abort_flag)) {
+              fail(kDetailWaitPFull);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t p_tm = tmem + kTmemS + 128u * (uint32_t)b;
+            const uint64_t vd = dv0 + (uint64_t)((stage * kKBytesPerStage) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts(tmem, p_tm + 8u * (uint32_t)kk, vd + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+                     (f == fs && kk == 0) ? 0u : 1u);
+            tc_commit(&sm.pv_done[b]);
+            tc_commit(&sm.v_empty[stage]);
+            if (f == fe - 1) tc_commit(&sm.o_full);
+          }
+        }
+        if (!ok) break;
+        ++seg;
+        w.advance(p, hdr);
+      }
+    }
+  }
+  } else {
+    setmaxnreg_inc<kSoftmaxRegs>();
+    // ======================= softmax + epilogue: warps 4-7 (half 0) and 8-11 (half 1). A thread
+    // owns one query row (its TMEM lane; lane quadrant = warp % 4) and 64 of a tile's 128 key
+    // columns; the two threads of a row (warps w and w + 4) exchange their maxima once per tile
+    // and their sums once per segment through shared memory and a named barrier of the pair.
+    // Leaving early: a failed bounded wait only marks the warp (good = false, error recorded,
+    // later waits return at once) and the work goes on; the pair leaves together after its next
+    // exchange, which carries both warps' marks, so neither is ever left alone at the barrier.
+    const int h = (warp - 4) >> 2;            // column half
+    const int quad = warp & 3;
+    const int t = 32 * quad + lane;           // query row
+    if (has_work) {
+      const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+      const uint32_t o_tm = tmem + lane_off + 64u * (uint32_t)h;
+      const int s_cnt = min(p.s_per_tile, p.S - qt * p.s_per_tile);   // block positions of this query tile
+      const int nrows = p.G * s_cnt;                                   // valid query rows (<= 128)
+      const float sc = p.scale_log2;
+      float* partials = reinterpret_cast<float*>(p.ws + p.off_partials);
+      float* plse = reinterpret_cast<float*>(p.ws + p.off_lse);
+      float* xv = reinterpret_cast<float*>(smem + kSmemX);             // [exchange parity][half][row]
+      int* xg = reinterpret_cast<int*>(xv + 2 * kHalves * kRows);      // [exchange parity][half][quadrant]
+      uint32_t xph = 0;                                                // exchanges so far
+      bool good = true;                                                // warp-uniform
+      // a bounded wait that records a failure instead of leaving
+      auto wait = [&](uint64_t* bar, uint32_t parity, uint32_t detail) {
+        bool got = true;
+        if (good) {
+          got = mbar_wait_bounded(bar, parity, abort_flag);
+          if (!got) fail(detail);
+        }
+        good = __all_sync(0xffffffffu, good && got);
+      };
+      // hands `v` to the row's other half and reads the other half's value into `other`; returns
+      // whether both warps of the pair are still good (the same answer in both)
+      auto exchange = [&](float v, float& other) -> bool {
+        float* slot = xv + (xph & 1u) * kHalves * kRows;
+        int* flg = xg + (xph & 1u) * kHalves * 4;
+        ++xph;
+        slot[h * kRows + t] = v;
+        if (lane == 0) flg[h * 4 + quad] = good ? 1 : 0;
+        named_barrier_sync(1 + quad, 64);
+        other = slot[(1 - h) * kRows + t];
+        return flg[(1 - h) * 4 + quad] != 0 && good;
+      };
+      SegWalk w;
+      w.init(p, sm, hdr);
+      long long f = 0;
+      int nseg = 0;
+      bool ok = true;
+      while (ok && !w.done()) {
+        int kb, ke;
+        w.segment(kb, ke);
+        const GroupInfo gi = w.gi;
+        float m_used = -INFINITY, l = 0.f;   // running base; this half's running sum
+        for (int k = kb; k < ke; ++k, ++f) {
+          const int valid = (k < gi.nctx) ? min(kTile, gi.L - k * kTile) : p.S;
+          const int b = ring_slot<kSBufs>(f);
+          const uint32_t s_tm = tmem + lane_off + kTmemS + 128u * (uint32_t)b;
+          wait(&sm.k_empty[b], ring_phase<kSBufs>(f), kDetailWaitSFull);
+          // (after a failed wait the work below still runs, on whatever TMEM holds: its results
+          // are discarded when the pair leaves at the exchange)
+          __syncwarp();   // lanes leave the wait one by one; the tcgen05 accesses are warp-collective
+          tc_fence_after();
+          uint32_t sr[64];
+          tmem_ld32(s_tm + 64u * (uint32_t)h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(s_tm + 64u * (uint32_t)h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+          const int valid_h = valid - 64 * h;   // valid keys among this half's columns
+          if (valid_h < 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c >= valid_h) sr[c] = __float_as_uint(-INFINITY);
+          }
+          float mx[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mx[q] = __uint_as_float(sr[q]);
+#pragma unroll
+          for (int c = 4; c + 8 <= 64; c += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) mx[q] = fmax3(mx[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + 4 + q]));
+          }
+          mx[0] = fmax3(mx[0], __uint_as_float(sr[60]), __uint_as_float(sr[61]));
+          mx[1] = fmax3(mx[1], __uint_as_float(sr[62]), __uint_as_float(sr[63]));
+          const float mh = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc;
+          // the row's tile maximum (both halves) decides the exponent base: a segment's first tile
+          // uses it; later tiles keep the running maximum m_used unless the tile exceeds it by more
+          // than 8 (P would exceed 256), in which case the base moves and O is rescaled. Both
+          // threads of a row see the same two values and take the same decision.
+          float mo;
+          if (!exchange(mh, mo)) {
+            ok = false;
+            break;
+          }
+          const float mt = fmaxf(mh, mo);
+          const bool first = (k == kb);
+          float m_new = m_used;
+          bool resc = false;
+          if (first) {
+            m_new = mt;
+          } else if (mt > m_used + 8.0f) {
+            m_new = mt;
+            resc = true;
+          }
+          // P = 2^(s * scale - base), written as bf16 pairs over columns [32 h, 32 h + 32) of the
+          // S buffer (the other half's S columns there were read before the exchange), summed in fp32
+          const uint32_t p_tm = s_tm + 32u * (uint32_t)h;
+          const uint64_t sc2 = pack_f32x2(sc, sc);
+          const uint64_t nb2 = pack_f32x2(-m_new, -m_new);
+          uint64_t acc2[2] = {pack_f32x2(0.f, 0.f), pack_f32x2(0.f, 0.f)};
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int c = 32 * q + 2 * jj;
+              const uint64_t x2 = ffma_f32x2(pack_u32x2(sr[c], sr[c + 1]), sc2, nb2);
+              const float p0 = ex2(lo_f32(x2)), p1 = ex2(hi_f32(x2));
+              acc2[jj & 1] = fadd_f32x2(acc2[jj & 1], pack_f32x2(p0, p1));
+              pk[jj] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(p_tm + 16u * (uint32_t)q, pk);
+          }
+          const uint64_t acc = fadd_f32x2(acc2[0], acc2[1]);
+          const float psum = lo_f32(acc) + hi_f32(acc);
+          const float factor = resc ? ex2(m_used - m_new) : 1.0f;
+          l = l * factor + psum;
+          tmem_wait_st();
+          if (!first && __any_sync(0xffffffffu, resc)) {
+            // O holds the products up to tile f - 1, the last of which may still be running: wait
+            // for it (the S of this tile came from a QK issued after the PV of tile f - kSBufs had
+            // completed, so pv_done of f - 1's buffer is at most one phase behind). Rows decide
+            // separately; the O accesses are warp-collective, so the warp rescales its 64 columns
+            // when any of its rows needs it (factor is 1 for the others).
+            const long long fp = f - 1;
+            wait(&sm.pv_done[ring_slot<kSBufs>(fp)], ring_phase<kSBufs>(fp), kDetailWaitPvDone);
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+              uint32_t orr[32];
+              tmem_ld32(o_tm + 32u * (uint32_t)cb, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * factor);
+              tmem_st32(o_tm + 32u * (uint32_t)cb, orr);
+            }
+            tmem_wait_st();
+          }
+          if (h == 0 && k < gi.nctx && valid < kTile) {
+            // Rows past the end of the context hold whatever the caller's slab or page holds
+            // there; P is 0 for them, but 0 * NaN would still poison O, so zero those V rows
+            // before the PV product reads them. The V tile must have landed first.
+            const int stage = ring_slot<kVStages>(f);
+            wait(&sm.v_full[stage], ring_phase<kVStages>(f), kDetailWaitKvFull);
+            uint8_t* vbase = smem + kSmemV + stage * kKBytesPerStage;
+            const int chunks_per_box = (kTile - valid) * 8;   // 16-byte chunks
+            for (int i = t; i < 2 * chunks_per_box; i += kRows) {
+              const int box = i / chunks_per_box, r = i - box * chunks_per_box;
+              *reinterpret_cast<uint4*>(vbase + box * kKVBoxBytes + (valid + r / 8) * 128 + (r % 8) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          }
+          m_used = m_new;
+          // every lane's TMEM stores (and O rescale) are complete and fenced before the warp's one
+          // arrival hands P to the MMA thread
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full[b]);
+        }
+        if (!ok) break;
+        // ---- epilogue of the segment: wait for the last PV product, then the row's sum over both
+        // halves, then this half's 64 dims of O / l
+        wait(&sm.o_full, (uint32_t)(nseg & 1), kDetailWaitPvDone);
+        float l_other;
+        if (!exchange(l, l_other)) {
+          ok = false;
+          break;
+        }
+        const float l_all = l + l_other;
+        __syncwarp();
+        tc_fence_after();
+        ++nseg;
+        const bool whole = (kb == 0) && (ke == gi.ntiles);
+        const bool row_valid = t < nrows;
+        const int s_idx = qt * p.s_per_tile + t / p.G;
+        const int hq = gi.kvh * p.G + t % p.G;
+        const float inv_l = 1.0f / l_all;
+        const float lse2 = m_used + log2f(l_all);
+        // partial slot unique per (group, team, query tile)
+        const size_t slot = ((size_t)w.u + (size_t)team) * (size_t)p.nq + (size_t)qt;
+        __nv_bfloat16* orow = p.out + (((size_t)gi.b * p.S + s_idx) * p.Hq + hq) * kD + 64 * h;
+        float* prow = partials + (slot * kRows + t) * kD + 64 * h;
+#pragma unroll 1
+        for (int cb = 0; cb < 2; ++cb) {
+          uint32_t orr[32];
+          tmem_ld32(o_tm + 32u * (uint32_t)cb, orr);
+          tmem_wait_ld();
+          if (row_valid) {
+            if (whole) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(orr[8 * q4 + 0]) * inv_l, __uint_as_float(orr[8 * q4 + 1]) * inv_l);
+                v.y = pack_bf16x2(__uint_as_float(orr[8 * q4 + 2]) * inv_l, __uint_as_float(orr[8 * q4 + 3]) * inv_l);
+                v.z = pack_bf16x2(__uint_as_float(orr[8 * q4 + 4]) * inv_l, __uint_as_float(orr[8 * q4 + 5]) * inv_l);
+                v.w = pack_bf16x2(__uint_as_float(orr[8 * q4 + 6]) * inv_l, __uint_as_float(orr[8 * q4 + 7]) * inv_l);
+                dst[q4] = v;
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(prow + cb * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                dst[q4] = make_float4(__uint_as_float(orr[4 * q4 + 0]) * inv_l, __uint_as_float(orr[4 * q4 + 1]) * inv_l,
+                                      __uint_as_float(orr[4 * q4 + 2]) * inv_l, __uint_as_float(orr[4 * q4 + 3]) * inv_l);
+            }
+          }
+        }
+        if (row_valid && h == 0) {
+          if (whole) {
+            if (p.lse) p.lse[((size_t)gi.b * p.Hq + hq) * p.S + s_idx] = lse2 * 0.69314718055994531f;
+          } else {
+            plse[slot * kRows + t] = lse2;
+          }
+        }
+        w.advance(p, hdr);
+      }
+    }
+  }
+
+  // ---- 3. teardown: all tensor-core work issued by the two MMA threads completes before TMEM
+  // is released (on the normal path it already has; on an abort path this drains it)
+  if ((warp == 1 || warp == 3) && lane == 0) {
+    tc_commit(&sm.drain);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace one
+
 // Merges the partials of groups cut between teams (flash-decoding combine):
 //   O = sum_j 2^(lse_j - M) O_j / sum_j 2^(lse_j - M),  M = max_j lse_j.
 // A CTA takes 32 query rows of one (group, query tile), 8 threads per row, each thread 16 of the
@@ -1033,7 +1624,7 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   p.off_partials = pl.off_partials;
   p.off_lse = pl.off_lse;
   p.skip_if = a->skip_if;
-  // the shared-memory opt-in is per device; set it once so no attribute call happens while a
+  // the shared-memory opt-ins are per device; set them once so no attribute call happens while a
   // caller captures the stream into a CUDA graph
   static unsigned long long attr_done = 0;   // bit per device ordinal (< 64)
   int dev = 0;
@@ -1041,17 +1632,28 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
     // The register raise of the softmax warpgroups waits until the block's pool (launch registers
-    // x threads) has room: refuse to launch unless the compiled kernel starts with enough.
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, attn_tc_kernel) != cudaSuccess) return TT_ERR_CUDA;
+    // x threads) has room: refuse to launch unless the compiled kernels start with enough.
+    cudaFuncAttributes fa{}, fa1{};
+    if (cudaFuncGetAttributes(&fa, attn_tc_kernel) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa1, one::attn_tc1_kernel) != cudaSuccess)
+      return TT_ERR_CUDA;
     if (fa.numRegs * kThreads < 128 * kProducerRegs + 2 * 128 * kSoftmaxRegs) return TT_ERR_UNSUPPORTED;
+    if (fa1.numRegs * one::kThreads < 128 * one::kProducerRegs + 2 * 128 * one::kSoftmaxRegs)
+      return TT_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(one::attn_tc1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)one::kSmemBytes) != cudaSuccess)
       return TT_ERR_CUDA;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  if (launch_pdl(attn_tc_kernel, dim3(pl.grid), dim3(kThreads), kSmemBytes, stream, p) != cudaSuccess)
-    return TT_ERR_CUDA;
+  // a group with one query tile: the one-tile kernel (both softmax warpgroups on that tile); the
+  // teams are single CTAs either way (ceil(1 / 2) = 1), so the plan and workspace are the same
+  const cudaError_t le =
+      (pl.qtiles == 1)
+          ? launch_pdl(one::attn_tc1_kernel, dim3(pl.grid), dim3(one::kThreads), one::kSmemBytes, stream, p)
+          : launch_pdl(attn_tc_kernel, dim3(pl.grid), dim3(kThreads), kSmemBytes, stream, p);
+  if (le != cudaSuccess) return TT_ERR_CUDA;
   MergeParams mp{};
   mp.S = p.S;
   mp.Hq = p.Hq;
