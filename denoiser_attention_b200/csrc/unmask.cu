@@ -235,6 +235,15 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// atomicAdd with acquire-release semantics at GPU scope: the writes before it are visible to a
+// thread that later acquires the same word, and the reads after it see what the earlier
+// releasers wrote
+__device__ __forceinline__ int atomic_add_acq_rel(int* ptr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+  return old;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskParams p) {
   using VT = VecTraits<T>;
@@ -264,6 +273,24 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
   __shared__ __align__(16) uint4 s_ring[kUnmaskRing][kUnmaskThreads];
   __shared__ int s_flag;
   const int warp = tid >> 5, lane = tid & 31;
+
+  // A row's part of the range is a segment. Each thread streams its vectors of the segment
+  // through its own ring, starting at slot 0; the first kUnmaskRing copies of a segment are
+  // issued here, for the next segment before the CTA reduces the finished one, so that those
+  // loads are in flight during the reduction.
+  auto prologue = [&](long long sg) {
+    const int rw = (int)(sg / p.vec_per_row);
+    const long long rb = (long long)rw * p.vec_per_row;
+    const long long se = min(vend, rb + p.vec_per_row);
+    const int n = (se - sg > tid) ? (int)((se - sg - tid + kUnmaskThreads - 1) / kUnmaskThreads) : 0;
+    const uint4* src = base + sg + tid;
+#pragma unroll
+    for (int i = 0; i < kUnmaskRing; ++i) {
+      if (i < n) cp_async16(&s_ring[i][tid], src + i * kUnmaskThreads);
+      cp_async_commit();
+    }
+  };
+  if (vbeg < vend) prologue(vbeg);
 
   for (long long seg = vbeg; seg < vend;) {
     const int row = (int)(seg / p.vec_per_row);
@@ -318,14 +345,13 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
     };
     // this thread's vectors vb + tid + i * kUnmaskThreads, i < nv, stream through its ring: the
     // copy of vector i + kUnmaskRing is issued once vector i has been consumed, so kUnmaskRing
-    // copies stay in flight (one commit group per index, empty past the end, keeps the count)
+    // copies stay in flight (one commit group per index, empty past the end, keeps the count);
+    // copies 0 .. kUnmaskRing - 1 were issued by prologue()
     const int nv = (ve - vb > tid) ? (ve - vb - tid + kUnmaskThreads - 1) / kUnmaskThreads : 0;
     auto issue = [&](int i) {
       if (i < nv) cp_async16(&s_ring[i % kUnmaskRing][tid], vp + vb + tid + i * kUnmaskThreads);
       cp_async_commit();
     };
-#pragma unroll
-    for (int i = 0; i < kUnmaskRing; ++i) issue(i);
     for (int i = 0; i < nv; ++i) {
       cp_async_wait<kUnmaskRing - 1>();   // the oldest copy (vector i) has landed
       const uint4 raw = s_ring[i % kUnmaskRing][tid];
@@ -333,6 +359,7 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
       issue(i + kUnmaskRing);
     }
     cp_async_wait<0>();
+    if (seg_end < vend) prologue(seg_end);
 
     // ---- CTA reduction (warp shuffles, then across warps), lowest index on ties
     const uint64_t accs = fadd_f32x2(acc[0], acc[1]);
@@ -356,12 +383,11 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
       if (c_hi > c_lo) {
         const size_t slot = (size_t)row + (size_t)cta;   // unique per (row, CTA) pair
         parts[slot] = UnmaskPartial{r.m, r.s, r.idx, 0};
-        __threadfence();
-        const int old = atomicAdd(row_cnt + row, 1);
+        // the ticket releases this CTA's partial and acquires those of the CTAs counted before it
+        const int old = atomic_add_acq_rel(row_cnt + row, 1);
         row_done = (old == (int)(c_hi - c_lo));
         if (row_done) {
           row_cnt[row] = 0;
-          __threadfence();
           const float4* pp = reinterpret_cast<const float4*>(parts);
           float4 q = __ldcg(pp + (size_t)row + (size_t)c_lo);
           r = RedState{q.x, q.y, __float_as_int(q.z)};
@@ -378,12 +404,12 @@ __global__ void __launch_bounds__(kUnmaskThreads) unmask_kernel(const UnmaskPara
         arg_ws[row] = r.idx;
         if (p.conf_out) p.conf_out[row] = conf;
         if (p.argmax_out) p.argmax_out[row] = r.idx;
-        __threadfence();
+        // releases this row's confidence and argmax; the sequence's last row acquires the others'
+        // (the CTA barrier below passes them on to the threads of commit_sequence)
         const int b = row / p.block_size;
-        const int old = atomicAdd(seq_cnt + b, 1);
+        const int old = atomic_add_acq_rel(seq_cnt + b, 1);
         if (old == p.block_size - 1) {
           seq_cnt[b] = 0;
-          __threadfence();
           last_of_seq = 1;
         }
       }
