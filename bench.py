@@ -380,9 +380,14 @@ def run_ours(args):
     ms_max = max_over_ranks(ms, dev)
     ms_per_step = ms_max / args.steps
 
-    # per-kernel durations from the events of a replay of the same M steps with event nodes
+    # per-kernel durations from the events of a replay of the same M steps with event nodes, run on
+    # one stream so that each event pair spans its own kernels only (with concurrent branches the
+    # unmask's pair would also span the attention it waits behind)
     del g, g_rem
+    schedule = run.step.schedule
+    run.step.schedule = "serial"
     g_ev, ev = run.capture(M, with_events=True)
+    run.step.schedule = schedule
     for _ in range(3):
         g_ev.replay()
     torch.cuda.synchronize()
@@ -424,7 +429,7 @@ def run_ours(args):
                        "seq_len": a.ctx_lens[0] + S, "parallelism": f"dp{world} (independent sequences)",
                        "l2": f"{M // 2} rotating input sets of {run_set_mb(inp, ad, logits):.1f} MB (> 4x L2 together)",
                        "schedule": args.schedule,
-                       "timing": f"CUDA graph of {M} steps replayed ({SCHEDULE_TEXT[args.schedule]}); per-kernel times from events in a second graph of the same steps, on the streams the kernels run on"},
+                       "timing": f"CUDA graph of {M} steps replayed ({SCHEDULE_TEXT[args.schedule]}); per-kernel times from events in a second graph of the same steps run on one stream"},
             "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                          "frac": attn_gbs / peak, "traffic": traffic, "kernel": "attn_tc_kernel",
                          "peak_source": peak_src, "algorithmic_bytes_per_launch": kv_bytes},
@@ -558,15 +563,21 @@ def run_extras(args, dev, peak):
                 table.append({"S": S, "temperature": 1.0 / inv_temp, "gamma": gamma,
                               "committed_per_step": float(nc.float().mean()),
                               "frac_above_gamma": float((conf >= gamma).float().mean())})
-        b = api.StepBuffers(tau=None, h=None, f=None, q=None, k_blk=None, v_blk=None, k_ctx=None, v_ctx=None,
-                            ctx_lens=None, page_table=None, logits=lg, tokens=t, is_masked=m)
+        # rotating copies of the logits, more than 4x L2 together, so that each launch reads HBM
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        n_sets = max(2, math.ceil(4 * l2 / (lg.numel() * lg.element_size())))
+        bs = [api.StepBuffers(tau=None, h=None, f=None, q=None, k_blk=None, v_blk=None, k_ctx=None, v_ctx=None,
+                              ctx_lens=None, page_table=None, logits=lg if k == 0 else lg.clone(), tokens=t.clone(),
+                              is_masked=m.clone()) for k in range(n_sets)]
         st = api.RefinementStep({}, gamma=0.8)
-        times[S] = isolated_ms(unmask_op(st), [b], [None], torch.cuda.Stream(device=dev), reps=50) * 1e3
-        del lg
+        times[S] = isolated_ms(unmask_op(st), bs, [None] * n_sets, torch.cuda.Stream(device=dev),
+                               reps=max(5, 200 // n_sets)) * 1e3
+        del lg, bs
         torch.cuda.empty_cache()
     out["sweep_unmask"] = {"unmask_us_by_S": times, "cells": table,
-                           "note": "committed tokens per step: mean over the 32 sequences of the first step "
-                                   "(every position masked), confidence sampler"}
+                           "note": "unmask time: graph of launches over rotating copies of the logits (more "
+                                   "than 4x L2 together); committed tokens per step: mean over the 32 sequences "
+                                   "of the first step (every position masked), confidence sampler"}
     # ---- the fused LM head + unmask on the decode shape (128 rows, D 2048, vocabulary 131072):
     # the 537 MB weight stream is the algorithmic traffic (larger than L2 by itself)
     lm = lmhead_inputs(dev)
