@@ -36,7 +36,9 @@
 // base move to the tile maximum, with O rescaled (exact: numerator and denominator share the
 // stale maximum).
 // Groups with a single query tile (G * S <= 128) run a second kernel, attn_tc1_kernel (namespace
-// `one` below), which puts both softmax warpgroups on that one tile.
+// `one` below), which puts both softmax warpgroups on that one tile; so do groups of two query
+// tiles (a team of two CTAs, one tile each) when the key tiles per SM, bounded from the context
+// capacity, are few (decode-sized work, where its faster pipeline fill and the smaller merge win).
 #include <cstdio>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -106,6 +108,10 @@ struct AttnMeta {
 // workload). The group-aligned partition is taken when its longest range is at most this much
 // above the uniform one's.
 constexpr long long kSegPenaltyTiles = 2;
+
+// Groups of two query tiles take the one-tile kernel when the key tiles (bounded from the context
+// capacity) are at most this many per SM.
+constexpr long long kOneTileMaxTilesPerSm = 32;
 
 struct TcParams {
   CUtensorMap tm_q, tm_kc, tm_vc, tm_kb, tm_vb;
@@ -1565,9 +1571,16 @@ AttnPlan attn_tc_plan(const tt_attn_args_t* a, int num_sms) {
   const int S = a->block_size;
   pl.s_per_tile = std::min(S, kRows / G);
   pl.qtiles = (S + pl.s_per_tile - 1) / pl.s_per_tile;        // nq
-  pl.team_size = (pl.qtiles + 1) / 2;                           // CTAs per team, two query tiles each
   pl.units = a->batch * a->num_kv_heads;                        // groups
   const int sms = std::max(1, num_sms);
+  // Groups of one query tile run the one-tile kernel. Groups of two do too (a team of two CTAs,
+  // one query tile each) when the CTAs would see few key tiles each: that kernel fills its
+  // pipeline sooner and a group is cut among fewer teams, so the merge has fewer partials. The
+  // lengths are on the device; the bound on the key tiles comes from the context capacity.
+  const long long cap = a->page_table ? (long long)a->max_pages_per_seq * a->page_size : (long long)a->ctx_stride;
+  const long long tiles_ub = (long long)pl.units * ((cap + kTile - 1) / kTile + 1);
+  pl.one_tile = (pl.qtiles == 1 || (pl.qtiles == 2 && tiles_ub <= kOneTileMaxTilesPerSm * (long long)sms)) ? 1 : 0;
+  pl.team_size = pl.one_tile ? pl.qtiles : (pl.qtiles + 1) / 2;   // CTAs per team
   const int teams = std::max(1, sms / pl.team_size);
   pl.grid = teams * pl.team_size;
   pl.slots = ((size_t)pl.units + (size_t)teams) * (size_t)pl.qtiles;
@@ -1647,10 +1660,10 @@ int attn_tc_launch(const tt_attn_args_t* a, const AttnPlan& pl, void* ws, cudaSt
       return TT_ERR_CUDA;
     __atomic_fetch_or(&attr_done, bit, __ATOMIC_ACQ_REL);
   }
-  // a group with one query tile: the one-tile kernel (both softmax warpgroups on that tile); the
-  // teams are single CTAs either way (ceil(1 / 2) = 1), so the plan and workspace are the same
+  // the plan's choice: the one-tile kernel (both softmax warpgroups on one query tile per CTA) or
+  // the two-stream kernel (two query tiles per CTA)
   const cudaError_t le =
-      (pl.qtiles == 1)
+      pl.one_tile
           ? launch_pdl(one::attn_tc1_kernel, dim3(pl.grid), dim3(one::kThreads), one::kSmemBytes, stream, p)
           : launch_pdl(attn_tc_kernel, dim3(pl.grid), dim3(kThreads), kSmemBytes, stream, p);
   if (le != cudaSuccess) return TT_ERR_CUDA;

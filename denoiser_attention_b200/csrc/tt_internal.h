@@ -47,7 +47,8 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream);
 struct AttnPlan {
   int grid;            // persistent CTAs
   int qtiles;          // query-row tiles per (sequence, kv head)
-  int team_size;       // CTAs per team (each CTA holds up to two query tiles of a group)
+  int team_size;       // CTAs per team (two-stream kernel: up to two query tiles of a group per CTA)
+  int one_tile;        // 1: attn_tc1_kernel, one query tile per CTA (teams of qtiles CTAs)
   int s_per_tile;      // block positions per query-row tile
   int units;           // groups: batch * kv heads
   size_t off_meta;     // total tiles and working CTAs of the partition
