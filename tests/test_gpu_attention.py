@@ -85,6 +85,35 @@ def test_attention_matches_oracle(cuda_lib, B, S, Hq, Hkv, d, lens, dtype, ps):
     np.testing.assert_allclose(np64(lse), ref_lse, atol=1e-4 if dtype == torch.bfloat16 else 1e-5)
 
 
+@pytest.mark.parametrize("B,S,lens,ps", [
+    (3, 16, [0, 100, 1000], 128),
+    (2, 16, [4100, 64], 256),
+    (2, 24, [300, 50], 128),     # three query tiles per group
+])
+def test_two_stream_kernel_on_short_contexts(cuda_lib, B, S, lens, ps):
+    # Groups of two query tiles run the one-tile kernel when the host's bound on the key tiles
+    # (from the page table's width) is small. A page table wider than the contexts need raises the
+    # bound above that limit, so these short contexts run the two-stream kernel; the entries past
+    # a sequence's pages are never read, and rows past the context end inside the last page hold
+    # NaN, which must not reach the output.
+    sh = synth.AttnShape(B, S, 32, 2, 128, lens, torch.bfloat16, page_size=ps, q_std=1 / math.sqrt(128))
+    inp = synth.attention_inputs(sh, seed=40 + B + S)
+    ref = _oracle(inp)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    units = B * 2
+    width = math.ceil(32 * sms / units * 128 / ps) + 2
+    assert units * (width * ps // 128 + 1) > 32 * sms
+    table = torch.full((B, width), -1, dtype=torch.int32)
+    table[:, :inp.page_table.shape[1]] = inp.page_table
+    for b, L in enumerate(lens):
+        if L % ps:
+            pg = int(table[b, L // ps])
+            inp.k_ctx[pg, L % ps:] = float("nan")
+            inp.v_ctx[pg, L % ps:] = float("nan")
+    inp.page_table = table
+    assert_close_attn(_run(inp), ref, torch.bfloat16, f"two-stream {B}x{S} lens={lens}")
+
+
 def test_attention_softmax_scale_and_large_logits(cuda_lib):
     # unscaled Q with softmax_scale 1/sqrt(d): logits of std ~1; and a sharp case (scale 1)
     for scale, q_std in ((1 / math.sqrt(128), 1.0), (1.0, 0.5)):
