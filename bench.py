@@ -266,7 +266,7 @@ class StepRun:
     def capture(self, n_steps, with_events):
         import torch
         mk = lambda: torch.cuda.Event(enable_timing=True, external=True)
-        ev = [(mk(), mk(), mk(), mk()) for _ in range(n_steps)] if with_events else None
+        ev = [tuple(mk() for _ in range(8)) for _ in range(n_steps)] if with_events else None
         g = torch.cuda.CUDAGraph()
         self.cap_stream.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(self.cap_stream):
@@ -393,6 +393,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     attn_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev), dev)
     unmask_ms = max_over_ranks(statistics.mean(e[2].elapsed_time(e[3]) for e in ev), dev)
+    cond_ms, normres_ms = (max_over_ranks(statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev), dev)
+                           for i in (4, 6))
     del g_ev
     # the same two kernels alone (own graphs over the same rotating input sets), for context: inside
     # the step they share the GPU with the other branches
@@ -440,6 +442,10 @@ def run_ours(args):
             "unmask_isolated_us": unmask_iso_ms * 1e3,
             "unmask_us": unmask_ms * 1e3, "unmask_steps_per_s": 1.0 / (unmask_ms * 1e-3),
             "unmask_logits_gbs": unmask_gbs, "unmask_frac": unmask_gbs / peak,
+            "step_breakdown_us": {"adaln_cond": cond_ms * 1e3, "norm_modulate_and_residual": normres_ms * 1e3,
+                                  "attention_and_merge": attn_ms * 1e3,
+                                  "unmask": unmask_ms * 1e3,
+                                  "note": "events around each launch group in a serial replay of the steps"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(t_c0 - 0.3, t_c1 + 0.1),
         }

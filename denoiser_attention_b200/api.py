@@ -117,6 +117,20 @@ def adaln_gated_residual(h, f, mod, out=None, ws_tag: str = "adaln", skip_if=Non
     return out
 
 
+def adaln_norm_modulate_residual(h, f, norm_w, mod, eps: float = 1e-5, out=None, out2=None, ws_tag: str = "adaln",
+                                 skip_if=None):
+    """(adaln_norm_modulate(h, norm_w, mod), adaln_gated_residual(h, f, mod)) in one launch that
+    reads h once."""
+    Bn, S, D = h.shape
+    out = torch.empty_like(h) if out is None else out
+    out2 = torch.empty_like(h) if out2 is None else out2
+    args = B.adaln_args(B.TT_ADALN_NORM_MODULATE_RESIDUAL, batch=Bn, block_size=S, hidden=D, dtype=h.dtype,
+                        eps=eps, h=h, norm_w=norm_w, f=f, mod=mod, out=out, out2=out2, skip_if=skip_if)
+    ws = workspace(256, h.device, ws_tag)
+    B.tt_adaln_modulate(args, ws)
+    return out, out2
+
+
 def unmask_step(logits, tokens, is_masked, *, gamma: float, inv_temperature: float = 1.0, mask_token_id: int = 3,
                 exclude_mask_token: bool = False, remaining_steps: int = 0, want_conf: bool = True,
                 ws_tag: str = "unmask", n_committed: Optional[torch.Tensor] = None,
@@ -227,9 +241,9 @@ class RefinementStep:
 
     SCHEDULES = ("branches", "attn_then_unmask", "unmask_then_attn", "serial")
 
-    # kernel launches per step: adaLN COND (3, one per MLP layer), RMSNorm prologue, attention and
-    # its split-KV merge, gated residual, unmask
-    LAUNCHES = 8
+    # kernel launches per step: adaLN COND (3, one per MLP layer), RMSNorm prologue with the gated
+    # residual, attention and its split-KV merge, unmask
+    LAUNCHES = 7
 
     def __init__(self, weights: Dict[str, torch.Tensor], *, gamma: float, inv_temperature: float = 1.0,
                  mask_token_id: int = 3, page_size: int = 0, ctx_stride: int = 0, softmax_scale: float = 1.0,
@@ -259,8 +273,9 @@ class RefinementStep:
 
     def run(self, b: StepBuffers, out_attn: Optional[torch.Tensor] = None, events=None, skip_if=None,
             all_done=None):
-        """Runs the step on the current stream. events: optional 4 timing events recorded around
-        the attention (0, 1) and the unmask (2, 3) launches, on the streams they run on.
+        """Runs the step on the current stream. events: optional timing events recorded around
+        the attention (0, 1) and the unmask (2, 3) launches, on the streams they run on, and, when
+        8 are given, around the COND (4, 5) and the RMSNorm + gated-residual (6, 7) launches.
         skip_if / all_done: optional int32 device words of a multi-step loop's early exit (every
         kernel of the step does nothing when *skip_if != 0; the unmask sets *all_done = 1 once no
         sequence has a masked position left). all_done must not be the word skip_if points to:
@@ -311,9 +326,13 @@ class RefinementStep:
         else:
             attention()
             unmask()
+        mark = (lambda i: events[i].record(main)) if events is not None and len(events) >= 8 else (lambda i: None)
+        mark(4)
         mod = adaln_cond(b.tau, w["w1"], w["b1"], w["w2"], w["b2"], w["w3"], w["b3"], w["layer_emb"], skip_if=skip_if)
-        y = adaln_norm_modulate(b.h, w["norm_w"], mod, eps=self.eps, skip_if=skip_if)
-        h_new = adaln_gated_residual(b.h, b.f, mod, skip_if=skip_if)
+        mark(5)
+        mark(6)
+        y, h_new = adaln_norm_modulate_residual(b.h, b.f, w["norm_w"], mod, eps=self.eps, skip_if=skip_if)
+        mark(7)
         if forked:
             join_a.record(s_attn)
             main.wait_event(join_a)

@@ -33,6 +33,7 @@ TT_SAMPLER_PREDICT_NOISE = 1
 TT_ADALN_COND = 0
 TT_ADALN_NORM_MODULATE = 1
 TT_ADALN_GATED_RESIDUAL = 2
+TT_ADALN_NORM_MODULATE_RESIDUAL = 3
 
 EXPORTED = [
     "tt_status_string", "tt_version",
@@ -69,7 +70,7 @@ class AdalnArgs(ctypes.Structure):
         ("mlp_width", _i32), ("dtype", _i32), ("eps", _f32),
         ("tau", _vp), ("w1", _vp), ("b1", _vp), ("w2", _vp), ("b2", _vp), ("w3", _vp), ("b3", _vp),
         ("layer_emb", _vp), ("mod", _vp), ("h", _vp), ("norm_w", _vp), ("f", _vp), ("out", _vp),
-        ("skip_if", _vp),
+        ("skip_if", _vp), ("out2", _vp),
     ]
 
 
@@ -225,14 +226,14 @@ def tt_denoise_attn(args: AttnArgs, workspace: torch.Tensor, stream=None) -> Non
 def adaln_args(op: int, *, batch: int, hidden: int, block_size: int = 0, freq_dim: int = 256,
                mlp_width: int = 256, dtype=torch.float32, eps: float = 1e-5, tau=None, w1=None, b1=None,
                w2=None, b2=None, w3=None, b3=None, layer_emb=None, mod=None, h=None, norm_w=None, f=None,
-               out=None, skip_if=None) -> AdalnArgs:
+               out=None, skip_if=None, out2=None) -> AdalnArgs:
     a = AdalnArgs()
     a.op, a.batch, a.block_size, a.hidden = op, batch, block_size, hidden
     a.freq_dim, a.mlp_width, a.dtype, a.eps = freq_dim, mlp_width, _dtype_code(dtype), float(eps)
     a.tau, a.w1, a.b1, a.w2, a.b2 = _ptr(tau), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)
     a.w3, a.b3, a.layer_emb, a.mod = _ptr(w3), _ptr(b3), _ptr(layer_emb), _ptr(mod)
     a.h, a.norm_w, a.f, a.out = _ptr(h), _ptr(norm_w), _ptr(f), _ptr(out)
-    a.skip_if = _ptr(skip_if)
+    a.skip_if, a.out2 = _ptr(skip_if), _ptr(out2)
     return a
 
 

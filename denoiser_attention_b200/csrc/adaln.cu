@@ -9,6 +9,7 @@
 //                                          staged in shared memory with asynchronous copies
 //   NORM_MODULATE    RMSNorm prologue modulated by (shift, scale): one warp per token row
 //   GATED_RESIDUAL   h + gate * f: a vectorised elementwise pass
+//   NORM_MODULATE_RESIDUAL  both from one read of h, in the RMSNorm kernel
 // All arithmetic is fp32 (the timestep sinusoid in fp64); bf16 tensors are widened on load and
 // rounded to nearest on store.
 #include <algorithm>
@@ -236,16 +237,21 @@ __device__ __forceinline__ void load_f32(const float* p, float* x) {
 // One warp per token row (b, s): y = h / sqrt(mean(h^2) + eps) * w * (1 + scale_b) + shift_b. A
 // lane keeps up to kNormVec of its row's vectors in registers from the sum of squares to the
 // output (one read of h for rows up to 32 kNormVec vectors: D <= 2048 in bf16), the sum is a
-// warp-shuffle reduction, and w, scale and shift are read as float4.
+// warp-shuffle reduction, and w, scale and shift are read as float4. With kResid the same pass
+// also writes out2 = h + gate_b * f, from the h already loaded: the vectors held in registers get
+// it while the sum of squares is formed, those of wider rows when they are read again for y (so
+// out2 may alias h).
 constexpr int kNormVec = 8;
 constexpr int kNormRowsPerCta = 4;
 
-template <typename T>
+template <typename T, bool kResid>
 __global__ void __launch_bounds__(32 * kNormRowsPerCta) adaln_norm_modulate_kernel(const void* __restrict__ h,
                                                                                    const float* __restrict__ norm_w,
                                                                                    const float* __restrict__ mod,
+                                                                                   const void* __restrict__ f,
                                                                                    int rows, int S, int D, float eps,
                                                                                    void* __restrict__ out,
+                                                                                   void* out2,
                                                                                    const int32_t* skip_if) {
   constexpr int N = Io<T>::kN;
   pdl_trigger();
@@ -259,6 +265,16 @@ __global__ void __launch_bounds__(32 * kNormRowsPerCta) adaln_norm_modulate_kern
   const size_t vbase = (size_t)row * nv;
   const float* shift = mod + (size_t)b * 3 * D;
   const float* scale = shift + D;
+  const float* gate = shift + 2 * D;
+  // out2 = h + gate * f for vector v whose h is x
+  auto residual = [&](int v, const float* x) {
+    float fv[N], g[N], o[N];
+    Io<T>::load(f, vbase + v, fv);
+    load_f32<N>(gate + v * N, g);
+#pragma unroll
+    for (int k = 0; k < N; ++k) o[k] = fmaf(g[k], fv[k], x[k]);
+    Io<T>::store(out2, vbase + v, o);
+  };
   float xr[kNormVec][N];
   float ss = 0.f;
 #pragma unroll
@@ -268,6 +284,7 @@ __global__ void __launch_bounds__(32 * kNormRowsPerCta) adaln_norm_modulate_kern
       Io<T>::load(h, vbase + v, xr[i]);
 #pragma unroll
       for (int k = 0; k < N; ++k) ss = fmaf(xr[i][k], xr[i][k], ss);
+      if constexpr (kResid) residual(v, xr[i]);
     }
   }
   for (int v = lane + 32 * kNormVec; v < nv; v += 32) {   // rows wider than the register cache
@@ -295,6 +312,7 @@ __global__ void __launch_bounds__(32 * kNormRowsPerCta) adaln_norm_modulate_kern
   for (int v = lane + 32 * kNormVec; v < nv; v += 32) {
     float x[N];
     Io<T>::load(h, vbase + v, x);
+    if constexpr (kResid) residual(v, x);
     emit(v, x);
   }
 }
@@ -358,15 +376,22 @@ int adaln_launch(const tt_adaln_args_t* a, void* ws, cudaStream_t stream) {
         launch_rows<false, false>(a->w3, a->b3, a->layer_emb, a2, B, W, OUT, a->mod, a->skip_if, stream) !=
             cudaSuccess)
       return TT_ERR_CUDA;
-  } else if (a->op == TT_ADALN_NORM_MODULATE) {
+  } else if (a->op == TT_ADALN_NORM_MODULATE || a->op == TT_ADALN_NORM_MODULATE_RESIDUAL) {
     const int rows = B * a->block_size;
     const dim3 grid((rows + kNormRowsPerCta - 1) / kNormRowsPerCta), block(32 * kNormRowsPerCta);
-    const cudaError_t e =
-        (a->dtype == TT_BF16)
-            ? launch_pdl(adaln_norm_modulate_kernel<__nv_bfloat16>, grid, block, 0, stream, a->h, a->norm_w,
-                         (const float*)a->mod, rows, a->block_size, D, a->eps, a->out, a->skip_if)
-            : launch_pdl(adaln_norm_modulate_kernel<float>, grid, block, 0, stream, a->h, a->norm_w,
-                         (const float*)a->mod, rows, a->block_size, D, a->eps, a->out, a->skip_if);
+    const bool resid = (a->op == TT_ADALN_NORM_MODULATE_RESIDUAL);
+    const float* mod = a->mod;
+    cudaError_t e;
+    if (a->dtype == TT_BF16)
+      e = resid ? launch_pdl(adaln_norm_modulate_kernel<__nv_bfloat16, true>, grid, block, 0, stream, a->h,
+                             a->norm_w, mod, a->f, rows, a->block_size, D, a->eps, a->out, a->out2, a->skip_if)
+                : launch_pdl(adaln_norm_modulate_kernel<__nv_bfloat16, false>, grid, block, 0, stream, a->h,
+                             a->norm_w, mod, a->f, rows, a->block_size, D, a->eps, a->out, a->out2, a->skip_if);
+    else
+      e = resid ? launch_pdl(adaln_norm_modulate_kernel<float, true>, grid, block, 0, stream, a->h, a->norm_w, mod,
+                             a->f, rows, a->block_size, D, a->eps, a->out, a->out2, a->skip_if)
+                : launch_pdl(adaln_norm_modulate_kernel<float, false>, grid, block, 0, stream, a->h, a->norm_w,
+                             mod, a->f, rows, a->block_size, D, a->eps, a->out, a->out2, a->skip_if);
     if (e != cudaSuccess) return TT_ERR_CUDA;
   } else {
     const int N = (a->dtype == TT_BF16) ? 8 : 4;

@@ -90,15 +90,20 @@ static int validate_adaln(const tt_adaln_args_t* a) {
       if (!aligned16(a->w1) || !aligned16(a->w2) || !aligned16(a->w3)) return TT_ERR_UNSUPPORTED;
       return TT_OK;
     case TT_ADALN_NORM_MODULATE:
-    case TT_ADALN_GATED_RESIDUAL: {
+    case TT_ADALN_GATED_RESIDUAL:
+    case TT_ADALN_NORM_MODULATE_RESIDUAL: {
+      const bool norm = (a->op != TT_ADALN_GATED_RESIDUAL), resid = (a->op != TT_ADALN_NORM_MODULATE);
       if (a->block_size < 1) return TT_ERR_INVALID_ARGUMENT;
       if (!a->h || !a->mod || !a->out) return TT_ERR_INVALID_ARGUMENT;
-      if (a->op == TT_ADALN_NORM_MODULATE && !a->norm_w) return TT_ERR_INVALID_ARGUMENT;
-      if (a->op == TT_ADALN_GATED_RESIDUAL && !a->f) return TT_ERR_INVALID_ARGUMENT;
-      if (a->op == TT_ADALN_NORM_MODULATE && !(a->eps >= 0.f)) return TT_ERR_INVALID_ARGUMENT;
+      if (norm && !a->norm_w) return TT_ERR_INVALID_ARGUMENT;
+      if (resid && !a->f) return TT_ERR_INVALID_ARGUMENT;
+      if (norm && !(a->eps >= 0.f)) return TT_ERR_INVALID_ARGUMENT;
+      if (a->op == TT_ADALN_NORM_MODULATE_RESIDUAL && (!a->out2 || a->out2 == a->out || a->out == a->f))
+        return TT_ERR_INVALID_ARGUMENT;
       const int W = (a->dtype == TT_BF16) ? 8 : 4;
       if (a->hidden % W != 0) return TT_ERR_UNSUPPORTED;
       if (!aligned16(a->h) || !aligned16(a->out) || (a->f && !aligned16(a->f))) return TT_ERR_UNSUPPORTED;
+      if (a->op == TT_ADALN_NORM_MODULATE_RESIDUAL && !aligned16(a->out2)) return TT_ERR_UNSUPPORTED;
       // mod and norm_w are read as float4
       if (!aligned16(a->mod) || (a->norm_w && !aligned16(a->norm_w))) return TT_ERR_UNSUPPORTED;
       return TT_OK;

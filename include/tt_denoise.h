@@ -143,13 +143,17 @@ int tt_denoise_attn(const tt_attn_args_t* args, void* workspace, size_t workspac
  *   h, out [B][S][D] E; norm_w [D] float.
  * op TT_ADALN_GATED_RESIDUAL (h, f, mod -> out):
  *   out[b][s] = h[b][s] + gate[b] * f[b][s]        h, f, out [B][S][D] E (out may alias h)
- * D must be a multiple of 8 for TT_BF16 and of 4 for TT_F32; h, f, out, mod and norm_w 16-byte
- * aligned (else TT_ERR_UNSUPPORTED).
+ * op TT_ADALN_NORM_MODULATE_RESIDUAL (h, f, norm_w, mod -> out, out2): both of the above from one
+ *   read of h: out = NORM_MODULATE's output, out2 = GATED_RESIDUAL's output. out2 may alias h; out
+ *   must not alias f or out2.
+ * D must be a multiple of 8 for TT_BF16 and of 4 for TT_F32; h, f, out, out2, mod and norm_w
+ * 16-byte aligned (else TT_ERR_UNSUPPORTED).
  * ------------------------------------------------------------------------------------------- */
 typedef enum {
   TT_ADALN_COND = 0,
   TT_ADALN_NORM_MODULATE = 1,
-  TT_ADALN_GATED_RESIDUAL = 2
+  TT_ADALN_GATED_RESIDUAL = 2,
+  TT_ADALN_NORM_MODULATE_RESIDUAL = 3
 } tt_adaln_op_t;
 
 typedef struct {
@@ -175,6 +179,7 @@ typedef struct {
   const void* f;
   void* out;
   const int32_t* skip_if;    /* optional device word: non-zero => the call does nothing */
+  void* out2;                /* NORM_MODULATE_RESIDUAL: the gated residual's output */
 } tt_adaln_args_t;
 
 size_t tt_adaln_workspace_bytes(const tt_adaln_args_t* args);

@@ -146,6 +146,12 @@ def _adaln_args(**kw):
     (dict(op=B.TT_ADALN_GATED_RESIDUAL, dtype=B.TT_BF16, hidden=260), B.TT_ERR_UNSUPPORTED),
     (dict(op=B.TT_ADALN_NORM_MODULATE, norm_w=4100), B.TT_ERR_UNSUPPORTED),      # read as float4
     (dict(op=B.TT_ADALN_GATED_RESIDUAL, mod=4104), B.TT_ERR_UNSUPPORTED),
+    # the fused RMSNorm + gated residual: a second output, not the first one, and y not over f
+    (dict(op=B.TT_ADALN_NORM_MODULATE_RESIDUAL, f=12288), B.TT_ERR_INVALID_ARGUMENT),           # out2 NULL
+    (dict(op=B.TT_ADALN_NORM_MODULATE_RESIDUAL, f=12288, out2=4096), B.TT_ERR_INVALID_ARGUMENT),
+    (dict(op=B.TT_ADALN_NORM_MODULATE_RESIDUAL, out2=8192), B.TT_ERR_INVALID_ARGUMENT),          # out == f
+    (dict(op=B.TT_ADALN_NORM_MODULATE_RESIDUAL, f=12288, out2=8200), B.TT_ERR_UNSUPPORTED),     # unaligned
+    (dict(op=B.TT_ADALN_NORM_MODULATE_RESIDUAL, f=12288, out2=8192, norm_w=None), B.TT_ERR_INVALID_ARGUMENT),
 ])
 def test_adaln_host_validation(lib, kw, status):
     a = _adaln_args(**kw)

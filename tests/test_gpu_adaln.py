@@ -20,6 +20,7 @@ def _dev(x):
     (3, 96, 64, 100, [0.0, 0.3, 0.999]),
     (64, 2048, 256, 256, [9 / 16] * 32 + [k / 16 for k in range(32)]),   # the batch workload's width
     (70, 64, 128, 1024, [((7 * k) % 17) / 16 for k in range(70)]),       # sequence chunks, widest layer
+    (70, 2040, 256, 256, [((5 * k) % 17) / 16 for k in range(70)]),      # 6120 output rows: a ragged last slice
 ])
 def test_cond_matches_oracle(cuda_lib, B, D, F, W, tau):
     a = synth.adaln_inputs(B, 2, D, tau, seed=D + W, dtype=torch.float32, freq_dim=F, mlp_width=W)
@@ -48,6 +49,31 @@ def test_norm_modulate_and_gated_residual(cuda_lib, dtype, B, S, D):
     else:
         assert_close_bf16_rounded(y, y_ref, "norm_modulate")
         assert_close_bf16_rounded(hn, h_ref, "gated_residual")
+
+
+@pytest.mark.parametrize("dtype,B,S,D", [(torch.float32, 1, 16, 256), (torch.bfloat16, 8, 16, 2048),
+                                         (torch.bfloat16, 2, 3, 8), (torch.float32, 3, 5, 4100),
+                                         (torch.bfloat16, 2, 4, 4160)])
+def test_norm_modulate_residual_fused(cuda_lib, dtype, B, S, D):
+    # one launch for both outputs, against the two oracle functions; D = 4100 (fp32) and 4160 (bf16)
+    # are wider than the rows a warp keeps in registers
+    a = synth.adaln_inputs(B, S, D, [0.5] * B, seed=S + D + 1, dtype=dtype)
+    g = torch.Generator().manual_seed(D + 1)
+    mod = (0.3 * torch.randn((B, 3, D), generator=g)).float()
+    y, hn = api.adaln_norm_modulate_residual(_dev(a.h), _dev(a.f), _dev(a.norm_w), _dev(mod), eps=1e-5)
+    y_ref = O.adaln_norm_modulate(np64(a.h), np64(a.norm_w), np64(mod), 1e-5)
+    h_ref = O.adaln_gated_residual(np64(a.h), np64(a.f), np64(mod))
+    if dtype == torch.float32:
+        assert np.abs(np64(y) - y_ref).max() <= 1e-5, np.abs(np64(y) - y_ref).max()
+        assert np.abs(np64(hn) - h_ref).max() <= 1e-5
+    else:
+        assert_close_bf16_rounded(y, y_ref, "fused norm_modulate")
+        assert_close_bf16_rounded(hn, h_ref, "fused gated_residual")
+    # the same with the residual written over h (rows both inside and beyond the register cache)
+    h = _dev(a.h).clone()
+    y2, _ = api.adaln_norm_modulate_residual(h, _dev(a.f), _dev(a.norm_w), _dev(mod), eps=1e-5, out2=h)
+    assert torch.equal(y2, y)
+    assert torch.equal(h, hn)
 
 
 def test_gated_residual_in_place(cuda_lib):
