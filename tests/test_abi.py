@@ -90,6 +90,35 @@ def test_attn_workspace_too_small(lib):
     assert lib.tt_denoise_attn(ctypes.byref(a), None, need, None) == B.TT_ERR_INVALID_ARGUMENT
 
 
+def _attn_ws_bytes(units, slots):
+    # header, the partition's totals, per group its first/last team, the split-KV partials
+    # [slots][128][128] and their log-sum-exps [slots][128], each start 256-byte aligned
+    off = 256
+    for nbytes in (16, 8 * units, 4 * slots * 128 * 128, 4 * slots * 128):
+        off = (off + nbytes + 255) // 256 * 256
+    return off
+
+
+@pytest.mark.parametrize("batch,stride,paged,one_tile", [
+    (8, 4096, False, True),       # decode shape: 528 key tiles at most, <= 32 per SM
+    (32, 8192, False, True),      # block sweep at S = 16: 4160 tiles
+    (64, 16384, False, False),    # batch shape: 16512 tiles, the two-stream kernel
+    (4, 0, True, False),          # paged, 480 pages of 256 per sequence: 7688 tiles at most
+])
+def test_attn_plan_picks_kernel_from_capacity(lib, batch, stride, paged, one_tile):
+    # Groups of two query tiles (G = 16, S = 16) run the one-tile kernel (teams of two CTAs) when the
+    # host's bound on the key tiles, from the context capacity, is at most 32 per SM; otherwise the
+    # two-stream kernel (one CTA per team). The workspace holds one partial per (group + team) and
+    # query tile, so its size shows the choice (148 SMs when no GPU is present).
+    kw = dict(batch=batch, ctx_stride=stride)
+    if paged:
+        kw.update(page_table=4096, page_size=256, max_pages_per_seq=480, num_pages=2048, ctx_stride=0)
+    a = _attn_args(**kw)
+    units, sms = batch * 2, 148
+    teams = sms // 2 if one_tile else sms
+    assert lib.tt_denoise_attn_workspace_bytes(ctypes.byref(a)) == _attn_ws_bytes(units, (units + teams) * 2)
+
+
 def _unmask_args(**kw):
     a = B.UnmaskArgs()
     a.batch, a.block_size, a.vocab, a.dtype = 2, 16, 1024, B.TT_BF16
